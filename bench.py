@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the WUSH-KV cache path on B200.
+
+One step = one decode step of one Qwen3-8B-shaped layer (32 query heads, 8 KV
+heads, head_dim 128, batch 16, ~8192 cached tokens, bf16 inputs, 2-bit QuEST
+INT, sink 64, recent 256, chunk 8):
+
+  append 1 post-RoPE token per sequence (key transform, fp16 recent window,
+  chunked flush with quantise + pack)  ->  query transform q' = T^{-T} q
+  ->  GQA decode attention over the packed cache + fp16 windows.
+
+The timed region cycles through `--copies` independent caches (one per
+"layer"), so each step reads cache bytes that are not in the 126 MB L2.
+
+    python bench.py [--steps K] [--warmup W] [--bits 2] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N   (independent replicas)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen3-8b-layer-b16-ctx8192"
+STEP_POOL = 32          # distinct per-step inputs, cycled
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--copies", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# byte model (algorithmic bytes)
+# ---------------------------------------------------------------------------
+
+def meta_bytes(quantizer: str) -> int:
+    return 2 if quantizer == "quest" else 4
+
+
+def decode_bytes(w, bits, state) -> int:
+    """KV bytes one decode reads (packed codes + per-token scales + fp16
+    windows) plus q' read and output write."""
+    _, ns, P, nr = state
+    per_unit = P * 2 * (16 * bits + meta_bytes(w.quantizer)) + (ns + nr) * 2 * 256
+    return w.units * per_unit + 2 * w.batch * w.n_q_heads * 128 * 4
+
+
+def append_bytes(w, bits, flushed: bool) -> int:
+    b = 2 * w.units * 128 * 2                 # bf16 k, v in
+    b += w.n_kv_heads * 128 * 128 * 4         # T_k
+    b += 2 * w.units * 128 * 2                # fp16 ring rows out
+    if flushed:
+        b += w.chunk * w.units * 2 * 256 + w.chunk * w.units * 2 * (16 * bits + meta_bytes(w.quantizer))
+    return b
+
+
+def qtransform_bytes(w) -> int:
+    return w.batch * w.n_q_heads * 128 * (2 + 4) + w.n_kv_heads * 128 * 128 * 4
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_inputs(w, torch, device):
+    """Prefill keys/values (context - 1 tokens) and a pool of per-step tokens."""
+    from bit_kv_cache_post_b200 import inputs as I
+    n = w.context - 1
+    k = np.stack([I.keys(w, 0, b, n) for b in range(w.batch)])       # [B, n, Hkv, 128]
+    v = np.stack([I.values(w, 0, b, n) for b in range(w.batch)])
+    kd = torch.from_numpy(k).to(device).to(torch.bfloat16)
+    vd = torch.from_numpy(v).to(device).to(torch.bfloat16)
+    del k, v
+    pool = []
+    for s in range(STEP_POOL):
+        ks, vs, qs = zip(*[I.step_tokens(w, 0, b, s) for b in range(w.batch)])
+        pool.append(tuple(torch.from_numpy(np.stack(x)).to(torch.bfloat16).pin_memory()
+                          for x in (ks, vs, qs)))          # [B,1,Hkv,128], [B,1,Hkv,128], [B,Hq,128]
+    return kd, vd, pool
+
+
+def window_state(n, w):
+    """(n, sink, packed, recent) token counts of one sequence (the byte model
+    follows the cache's window bookkeeping)."""
+    ns = min(n, w.sink)
+    m = n - ns
+    P = w.chunk * ((m - w.recent) // w.chunk) if m >= w.recent + w.chunk else 0
+    return n, ns, P, m - P
+
+
+def run_ours(args, rank, world, device, torch, dist):
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[WORKLOAD]
+    bits = args.bits
+    stream = torch.cuda.current_stream()
+    kd, vd, pool = build_inputs(w, torch, device)
+    total_steps = args.warmup + args.steps + args.e2e_steps
+    grow = math.ceil(total_steps / args.copies) + 8
+    cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, w.context + grow, bits=bits,
+                         sink=w.sink, recent=w.recent, chunk=w.chunk)
+    caches, Ts, TinvTs = [], [], []
+    for c in range(args.copies):
+        T, TinvT = I.key_transforms(w, c)
+        Ts.append(torch.from_numpy(T).to(device))
+        TinvTs.append(torch.from_numpy(TinvT).to(device))
+        cache = wk.Cache(cfg, device=device)
+        cache.append(kd, vd, Ts[-1])
+        caches.append(cache)
+    torch.cuda.synchronize()
+    del kd, vd
+    dev_pool = [tuple(x.to(device) for x in p) for p in pool]
+    qprime = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32, device=device)
+    out = torch.empty_like(qprime)
+
+    # host-side counts to account the algorithmic bytes of each step
+    counts = [c.tokens()[0] for c in caches]
+
+    def step_bytes(i):
+        c = i % args.copies
+        before = window_state(counts[c], w)
+        counts[c] += 1
+        after = window_state(counts[c], w)
+        dec = decode_bytes(w, bits, after)
+        rest = append_bytes(w, bits, after[2] > before[2]) + qtransform_bytes(w)
+        return dec, rest
+
+    def step(i, k, v, q, ev=None):
+        c = i % args.copies
+        if ev is not None:
+            ev[0].record(stream)
+        caches[c].append(k, v, Ts[c])
+        if ev is not None:
+            ev[1].record(stream)
+        wk.query_transform(q, TinvTs[c], out=qprime)
+        if ev is not None:
+            ev[2].record(stream)
+        caches[c].decode(qprime, out=out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step_bytes(i)
+        step(i, *dev_pool[i % STEP_POOL])
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, device resident inputs ----------------------
+    K = args.steps
+    dec_total = rest_total = 0
+    for i in range(args.warmup, args.warmup + K):
+        d, r = step_bytes(i)
+        dec_total += d
+        rest_total += r
+    counts_after = list(counts)
+    counts = [c.tokens()[0] for c in caches]          # restore, then replay live
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0.record(stream)
+        for j, i in enumerate(range(args.warmup, args.warmup + K)):
+            step(i, *dev_pool[i % STEP_POOL], ev=evs[j])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    counts = counts_after
+    ms = t0.elapsed_time(t1)
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    if dist is not None:
+        tt = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    launches_per_step = 3
+    status = max(c.device_status() for c in caches)
+
+    # ---- e2e: host buffers, copies inside the timed region --------------------
+    E = args.e2e_steps
+    host_out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory()
+    e_dec = 0
+    for i in range(args.warmup + K, args.warmup + K + E):
+        e_dec += sum(step_bytes(i))
+    h2d = sum(x.numel() * x.element_size() for x in pool[0])
+    d2h = host_out.numel() * 4
+    buf = [torch.empty_like(x, device=device) for x in dev_pool[0]]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.warmup + K, args.warmup + K + E):
+        for dst, src in zip(buf, pool[i % STEP_POOL]):
+            dst.copy_(src, non_blocking=True)
+        step(i, *buf)
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+
+    return dict(w=w, bits=bits, K=K, ms=ms, dec_total=dec_total, rest_total=rest_total,
+                dec_ms=dec_ms, app_ms=app_ms, clocks=clocks.summary(), launches=launches_per_step * K,
+                status=status, e2e=(E, e_ms, e_dec, h2d, d2h), copies=args.copies,
+                l2_bytes=sum(decode_bytes(w, bits, window_state(c, w)) for c in counts))
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_unit(w, bits):
+    """Single (sequence 0, KV head 0) oracle cache holding context - 1 tokens
+    (untimed set-up) and its step inputs."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from oracle import wushkv_oracle as O
+    n = w.context - 1
+    k = I.round_to(I.keys(w, 0, 0, n)[:, :1][None], w.dtype)
+    v = I.round_to(I.values(w, 0, 0, n)[:, :1][None], w.dtype)
+    T, TinvT = I.key_transform(w, 0, 0)
+    oc = O.OracleCache(O.CacheConfig(1, 1, w.group, w.context + 4096, bits=bits,
+                                     sink=w.sink, recent=w.recent, chunk=w.chunk))
+    oc.append(k, v, T[None].astype(np.float64))
+    return oc, T, TinvT
+
+
+def oracle_step(w, oc, T, TinvT, s, frac=1.0):
+    """Append one token, transform the group's queries and decode them over
+    the first `frac` of the unit's cached tokens.  Returns algorithmic bytes."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from oracle import wushkv_oracle as O
+    k, v, q = I.step_tokens(w, 0, 0, s % STEP_POOL)
+    oc.append(I.round_to(k[:, :1], w.dtype)[None], I.round_to(v[:, :1], w.dtype)[None],
+              T[None].astype(np.float64))
+    qp = O.transform_query(I.round_to(q[:w.group], w.dtype), TinvT.astype(np.float64))
+    ns, P, nr = oc.split()
+    if frac >= 1.0:
+        oc.decode(qp[None])
+        return decode_bytes(w, oc.cfg.bits, (oc.n, ns, P, nr)) // w.units
+    # a bounded sample: the same arithmetic over a prefix of the packed tokens
+    pt = max(4, int(P * frac)) // 4 * 4
+    Kd = O.quest_dequantize(oc.codes_k[0, :pt], oc.meta_k[0, :pt, 0], oc.cfg.bits)
+    Vd = O.quest_dequantize(oc.codes_v[0, :pt], oc.meta_v[0, :pt, 0], oc.cfg.bits)
+    O.attention_f64(qp, Kd, Vd, 1.0 / math.sqrt(128))
+    return pt * 2 * (16 * oc.cfg.bits + meta_bytes(w.quantizer))
+
+
+def _one_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except Exception:
+        class _N:
+            def __enter__(self): return self
+            def __exit__(self, *a): return False
+        return _N()
+
+
+def cpu_baseline(w, bits, budget_s=15.0):
+    from bit_kv_cache_post_b200 import inputs as I  # noqa: F401
+    with _one_thread():
+        oc, T, TinvT = oracle_unit(w, bits)
+        nbytes, reps = 0, 0
+        t = time.perf_counter()
+        while time.perf_counter() - t < budget_s or reps < 2:
+            nbytes += oracle_step(w, oc, T, TinvT, reps)
+            reps += 1
+        el = time.perf_counter() - t
+    return {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one (sequence, KV head) unit of {w.name}: {reps} steps of 1-token append "
+                      f"+ {w.group}-head decode over ~{w.context} tokens, {el:.1f} s, 1 thread"}
+
+
+def run_reference(args):
+    from bit_kv_cache_post_b200 import inputs as I
+    w = I.WORKLOADS[WORKLOAD]
+    with _one_thread():
+        oc, T, TinvT = oracle_unit(w, args.bits)
+        t = time.perf_counter()
+        oracle_step(w, oc, T, TinvT, 0)
+        t_full = time.perf_counter() - t
+        frac = min(1.0, 90.0 / max(1, args.steps + args.warmup) / max(t_full, 1e-6))
+        for s in range(args.warmup):
+            oracle_step(w, oc, T, TinvT, s, frac)
+        nbytes = 0
+        t = time.perf_counter()
+        for s in range(args.steps):
+            nbytes += oracle_step(w, oc, T, TinvT, s, frac)
+        el = time.perf_counter() - t
+    v = nbytes / el / 1e9
+    sample = (f"one (sequence, KV head) unit of {w.name}; each step appends 1 token and decodes "
+              f"{w.group} heads over {'all' if frac >= 1 else f'{frac:.3%} of the packed'} tokens; 1 thread")
+    return {"impl": "reference", "metric": BASELINE_METRIC, "value": v, "unit": "GB/s",
+            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_block(w, args.bits, None),
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+BASELINE_METRIC = "2-bit KV decode-attention GB/s (% of HBM peak); KV append tokens/s"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "of measured (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+    except Exception:
+        return 6650.0, "of fallback (6.65 TB/s)"
+
+
+def config_block(w, bits, copies):
+    c = {"workload": w.name, "layers": 1, "batch": w.batch, "n_q_heads": w.n_q_heads,
+         "n_kv_heads": w.n_kv_heads, "head_dim": 128, "context": w.context, "bits": bits,
+         "quantizer": "QuEST INT", "sink": w.sink, "recent": w.recent, "chunk": w.chunk,
+         "input_dtype": w.dtype, "step": "append 1 token/seq + query transform + decode"}
+    if copies is not None:
+        c["l2"] = (f"inputs larger than L2: {copies} independent caches cycled "
+                   "(one per layer), ~90 MB of cache bytes each")
+    return c
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    r = run_ours(args, rank, world, device, torch, dist)
+    w, bits, K = r["w"], r["bits"], r["K"]
+    step_bytes = r["dec_total"] + r["rest_total"]
+    value = world * step_bytes / (r["ms"] / 1e3) / 1e9
+    dec_avg_ms = float(np.mean(r["dec_ms"]))
+    achieved = (r["dec_total"] / K) / (dec_avg_ms / 1e3) / 1e9
+    peak, peak_src = peaks()
+    E, e_ms, e_dec, h2d, d2h = r["e2e"]
+    line = {
+        "metric": BASELINE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": r["ms"] / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config_block(w, bits, r["copies"]),
+        "decode_gbs": world * r["dec_total"] / (r["ms"] / 1e3) / 1e9,
+        "append_tokens_per_s": w.batch * K / (float(np.sum(r["app_ms"])) / 1e3),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "decode",
+                     "peak_source": peak_src, "frac_of_8tbs": achieved / 8000.0,
+                     "launch_ms": dec_avg_ms, "bytes_per_launch": r["dec_total"] / K},
+        "e2e": {"value": world * e_dec / (e_ms / 1e3) / 1e9 if E else None,
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": E, "counts": "step bytes / step time incl. pinned host<->device copies"},
+        "gpu_launches": r["launches"], "clocks": r["clocks"], "device_status": r["status"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, bits)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,449 @@
+// Host side of the libwushkv C ABI: configuration checks, cache layout, the
+// window/flush bookkeeping of each append, decode split policy, export and
+// status.  See include/wushkv.h for the contract of every entry point.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "wushkv_internal.cuh"
+
+struct wushkv_cache {
+  wushkv_config cfg;
+  wushkv_layout lay;
+  uint8_t* base;
+  size_t bytes;
+  int64_t n;        // tokens per sequence
+  double alpha;     // QuEST clip ratio in use
+};
+
+namespace {
+
+using namespace wushkv;
+
+// Decode split policy: tokens per CTA for the fp16 windows and for the
+// packed cache.  max_splits in the workspace is sized from these.
+constexpr int WIN_TOKENS_PER_SPLIT = 128;
+constexpr int PACK_TOKENS_PER_SPLIT = 512;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t packed_count(int64_t n, const wushkv_config& c) {
+  const int64_t ns = n < c.sink ? n : c.sink;
+  const int64_t m = n - ns;
+  return (m >= (int64_t)c.recent + c.chunk) ? (int64_t)c.chunk * ((m - c.recent) / c.chunk) : 0;
+}
+
+// ---- default QuEST clip ratio ------------------------------------------------
+// The clip ratio that minimises the mean squared error of the 2^b-level
+// mid-rise uniform quantiser on a unit Gaussian (Max, 1960), found as the
+// zero of the derivative of that error with respect to the clip ratio.  The
+// derivative only involves the moving levels c_i = (2i + 1) alpha / L:
+//   dMSE/dalpha = -2 sum_i (2i + 1)/L * int_{cell i} (x - c_i) phi(x) dx.
+double std_pdf(double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) * 0.3989422804014327; }
+double std_cdf(double x) {
+  if (std::isinf(x)) return x > 0 ? 1.0 : 0.0;
+  return 0.5 * std::erfc(-x * 0.7071067811865476);
+}
+double mse_slope(double alpha, int L) {
+  const double step = 2.0 * alpha / L;
+  double acc = 0.0;
+  for (int i = -L / 2; i < L / 2; ++i) {
+    const double lo = (i == -L / 2) ? -INFINITY : i * step;
+    const double hi = (i == L / 2 - 1) ? INFINITY : (i + 1) * step;
+    const double ci = (i + 0.5) * step;
+    const double first = (std_pdf(lo) - std_pdf(hi)) - ci * (std_cdf(hi) - std_cdf(lo));
+    acc += -2.0 * (2.0 * i + 1.0) / L * first;
+  }
+  return acc;
+}
+double gaussian_optimal_alpha(int bits) {
+  const int L = 1 << bits;
+  double lo = 0.25, hi = 16.0;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (mse_slope(mid, L) < 0) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// ---- configuration + layout ----------------------------------------------------
+wushkv_status check_config(const wushkv_config* c) {
+  if (!c) return WUSHKV_EINVAL;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->max_ctx < 1) return WUSHKV_EINVAL;
+  if (c->n_q_heads % c->n_kv_heads) return WUSHKV_EINVAL;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (c->head_dim != 128) return WUSHKV_EUNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return WUSHKV_EUNSUPPORTED;
+  if (c->bits < 2 || c->bits > 4) return WUSHKV_EUNSUPPORTED;
+  if (c->quantizer != WUSHKV_QUEST_INT && c->quantizer != WUSHKV_AFFINE_PCTCLIP) return WUSHKV_EINVAL;
+  if (c->sink < 0 || c->recent < 0 || c->chunk < 4) return WUSHKV_EINVAL;
+  if (c->sink % 4 || c->chunk % 4) return WUSHKV_EUNSUPPORTED;
+  if (c->quantizer == WUSHKV_QUEST_INT) {
+    if (c->quest_alpha < 0 || c->quest_alpha > (double)(1 << (c->bits - 1)) ||
+        std::isnan(c->quest_alpha))
+      return WUSHKV_EINVAL;
+  } else {
+    if (c->clip_lo_rank < 1 || c->clip_hi_rank > 128 || c->clip_lo_rank >= c->clip_hi_rank)
+      return WUSHKV_EINVAL;
+    if (c->clip_lo_rank > 8 || c->clip_hi_rank < 121) return WUSHKV_EUNSUPPORTED;
+  }
+  if ((int64_t)c->batch * c->n_kv_heads > 65535) return WUSHKV_EUNSUPPORTED;
+  return WUSHKV_OK;
+}
+
+int max_splits_for(const wushkv_config& c, int packed_capacity) {
+  const int win = (c.sink + c.recent + c.chunk + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
+  const int pack = (packed_capacity + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
+  return (win > 0 ? win : 1) + pack;
+}
+
+void make_layout(const wushkv_config& c, wushkv_layout* L) {
+  std::memset(L, 0, sizeof(*L));
+  const size_t U = (size_t)c.batch * c.n_kv_heads;
+  const int G = c.n_q_heads / c.n_kv_heads;
+  if (c.bits == 3) { L->n_planes = 2; L->plane_bits[0] = 2; L->plane_bits[1] = 1; }
+  else { L->n_planes = 1; L->plane_bits[0] = c.bits; }
+  L->packed_capacity = (int)align_up((size_t)c.max_ctx, 32);
+  size_t off = 0;
+  for (int p = 0; p < L->n_planes; ++p) {
+    L->plane_unit_stride[p] = (size_t)L->packed_capacity * 16 * L->plane_bits[p];
+    L->k_plane_off[p] = off; off = align_up(off + U * L->plane_unit_stride[p], 256);
+    L->v_plane_off[p] = off; off = align_up(off + U * L->plane_unit_stride[p], 256);
+  }
+  L->meta_bytes = c.quantizer == WUSHKV_QUEST_INT ? 2 : 4;
+  L->meta_unit_stride = align_up((size_t)L->packed_capacity * L->meta_bytes, 16);
+  L->k_meta_off = off; off = align_up(off + U * L->meta_unit_stride, 256);
+  L->v_meta_off = off; off = align_up(off + U * L->meta_unit_stride, 256);
+  L->sink_unit_stride = (size_t)c.sink * 128 * 2;
+  L->sink_k_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
+  L->sink_v_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
+  L->ring_slots = c.recent + c.chunk;
+  L->ring_unit_stride = (size_t)L->ring_slots * 128 * 2;
+  L->ring_k_off = off; off = align_up(off + U * L->ring_unit_stride, 256);
+  L->ring_v_off = off; off = align_up(off + U * L->ring_unit_stride, 256);
+  const int ms = max_splits_for(c, L->packed_capacity);
+  L->workspace_off = off;
+  L->workspace_bytes = U * (size_t)ms * G * (128 + 2) * sizeof(float) + U * sizeof(int);
+  off = align_up(off + L->workspace_bytes, 256);
+  L->status_off = off; off = align_up(off + 256, 256);
+  L->total_bytes = off;
+}
+
+DevCache dev_view(const wushkv_cache* h) {
+  const wushkv_config& c = h->cfg;
+  const wushkv_layout& L = h->lay;
+  DevCache d;
+  std::memset(&d, 0, sizeof(d));
+  for (int p = 0; p < L.n_planes; ++p) {
+    d.k_plane[p] = h->base + L.k_plane_off[p];
+    d.v_plane[p] = h->base + L.v_plane_off[p];
+    d.plane_unit_stride[p] = L.plane_unit_stride[p];
+    d.plane_bits[p] = L.plane_bits[p];
+  }
+  d.n_planes = L.n_planes;
+  d.bits = c.bits;
+  d.quantizer = c.quantizer;
+  d.k_meta = h->base + L.k_meta_off;
+  d.v_meta = h->base + L.v_meta_off;
+  d.meta_bytes = (int)L.meta_bytes;
+  d.meta_unit_stride = L.meta_unit_stride;
+  d.sink_k = reinterpret_cast<__half*>(h->base + L.sink_k_off);
+  d.sink_v = reinterpret_cast<__half*>(h->base + L.sink_v_off);
+  d.ring_k = reinterpret_cast<__half*>(h->base + L.ring_k_off);
+  d.ring_v = reinterpret_cast<__half*>(h->base + L.ring_v_off);
+  d.sink = c.sink; d.recent = c.recent; d.chunk = c.chunk; d.ring_slots = L.ring_slots;
+  d.packed_capacity = L.packed_capacity;
+  d.max_splits = max_splits_for(c, L.packed_capacity);
+  const size_t U = (size_t)c.batch * c.n_kv_heads;
+  d.partials = reinterpret_cast<float*>(h->base + L.workspace_off);
+  d.counters = reinterpret_cast<int*>(h->base + L.workspace_off +
+                                      U * (size_t)d.max_splits * (c.n_q_heads / c.n_kv_heads) *
+                                          (128 + 2) * sizeof(float));
+  d.status = reinterpret_cast<int*>(h->base + L.status_off);
+  d.units = (int)U;
+  d.n_kv_heads = c.n_kv_heads;
+  d.group = c.n_q_heads / c.n_kv_heads;
+  d.alpha = h->alpha;
+  d.r_lo = c.clip_lo_rank;
+  d.r_hi = c.clip_hi_rank;
+  return d;
+}
+
+wushkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA; }
+
+bool valid_dtype(int32_t d) { return d == WUSHKV_F16 || d == WUSHKV_BF16 || d == WUSHKV_F32; }
+
+}  // namespace
+
+extern "C" {
+
+double wushkv_default_quest_alpha(int32_t bits) {
+  if (bits < 2 || bits > 4) return 0.0;
+  static double cached[5] = {0, 0, 0, 0, 0};
+  if (cached[bits] == 0.0) cached[bits] = gaussian_optimal_alpha(bits);
+  return cached[bits];
+}
+
+const char* wushkv_strerror(int32_t s) {
+  switch (s) {
+    case WUSHKV_OK: return "ok";
+    case WUSHKV_EINVAL: return "invalid argument";
+    case WUSHKV_ECAPACITY: return "cache capacity exceeded";
+    case WUSHKV_EUNSUPPORTED: return "unsupported configuration";
+    case WUSHKV_ECUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+size_t wushkv_cache_bytes(const wushkv_config* cfg) {
+  if (check_config(cfg) != WUSHKV_OK) return 0;
+  wushkv_layout L;
+  make_layout(*cfg, &L);
+  return L.total_bytes;
+}
+
+wushkv_status wushkv_cache_create(const wushkv_config* cfg, void* dev_mem, size_t bytes,
+                                  void* stream, wushkv_cache** out) {
+  if (!out) return WUSHKV_EINVAL;
+  *out = nullptr;
+  const wushkv_status st = check_config(cfg);
+  if (st != WUSHKV_OK) return st;
+  if (!dev_mem || (reinterpret_cast<uintptr_t>(dev_mem) & 255)) return WUSHKV_EINVAL;
+  wushkv_layout L;
+  make_layout(*cfg, &L);
+  if (bytes < L.total_bytes) return WUSHKV_EINVAL;
+  wushkv_cache* h = new (std::nothrow) wushkv_cache;
+  if (!h) return WUSHKV_EINVAL;
+  h->cfg = *cfg;
+  h->lay = L;
+  h->base = static_cast<uint8_t*>(dev_mem);
+  h->bytes = bytes;
+  h->n = 0;
+  h->alpha = cfg->quest_alpha > 0 ? cfg->quest_alpha : wushkv_default_quest_alpha(cfg->bits);
+  const cudaError_t e = cudaMemsetAsync(dev_mem, 0, L.total_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) { delete h; return WUSHKV_ECUDA; }
+  *out = h;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_cache_destroy(wushkv_cache* cache) {
+  delete cache;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_cache_layout(const wushkv_cache* cache, wushkv_layout* out) {
+  if (!cache || !out) return WUSHKV_EINVAL;
+  *out = cache->lay;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t* n_tokens, int64_t* n_sink,
+                                  int64_t* n_packed, int64_t* n_recent) {
+  if (!cache) return WUSHKV_EINVAL;
+  const int64_t n = cache->n;
+  const int64_t ns = n < cache->cfg.sink ? n : cache->cfg.sink;
+  const int64_t P = packed_count(n, cache->cfg);
+  if (n_tokens) *n_tokens = n;
+  if (n_sink) *n_sink = ns;
+  if (n_packed) *n_packed = P;
+  if (n_recent) *n_recent = n - ns - P;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                            int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
+                            int32_t quantizer, void* stream) {
+  if (!cache || !k_rope_dev || !v_dev || !valid_dtype(in_dtype) || n_tok < 0) return WUSHKV_EINVAL;
+  const wushkv_config& c = cache->cfg;
+  if (bits != c.bits || quantizer != c.quantizer) return WUSHKV_EINVAL;
+  if (n_tok == 0) return WUSHKV_OK;
+  if (cache->n + n_tok > c.max_ctx) return WUSHKV_ECAPACITY;
+  const int64_t n0 = cache->n, n1 = n0 + n_tok;
+  const int64_t S = c.sink, W = c.recent + c.chunk;
+  const int64_t P0 = packed_count(n0, c), P1 = packed_count(n1, c);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  AppendArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.c = dev_view(cache);
+  a.k = k_rope_dev;
+  a.v = v_dev;
+  a.dtype = in_dtype;
+  a.T = T_k_dev;
+  a.n_tok = n_tok;
+  a.n0 = n0;
+  a.packed0 = P0;
+  a.packed1 = P1;
+
+  // Old recent tokens that this append flushes: [S + P0, min(S + P1, n0)).
+  const int64_t flush_end = (S + P1 < n0) ? S + P1 : n0;
+  const bool has_old_flush = (P1 > P0) && (S + P0 < n0);
+  const int64_t first = has_old_flush ? S + P0 : n0;
+  const int64_t q_begin = first / 4, q_end = (n1 + 3) / 4;
+  const int units = (int)((int64_t)c.batch * c.n_kv_heads);
+
+  auto launch = [&](int64_t qa, int64_t qb) -> cudaError_t {
+    if (qb <= qa) return cudaSuccess;
+    a.quad_begin = qa;
+    a.n_quads = qb - qa;
+    // enough CTAs to fill the GPU, up to 64 quads (256 tokens) per CTA
+    int64_t per = (a.n_quads * units) / 1184;
+    if (per < 1) per = 1;
+    if (per > 64) per = 64;
+    a.quads_per_cta = (int)per;
+    return launch_append(a, s);
+  };
+
+  cudaError_t e;
+  // New tokens may reuse ring slots that old flushed tokens are read from
+  // only when the touched span exceeds the ring; then flush first.
+  if (has_old_flush && (n1 - (S + P0) > W)) {
+    const int64_t q_mid = (flush_end + 3) / 4;
+    e = launch(q_begin, q_mid);
+    if (e == cudaSuccess) e = launch(q_mid, q_end);
+  } else {
+    e = launch(q_begin, q_end);
+  }
+  if (e != cudaSuccess) return WUSHKV_ECUDA;
+  cache->n = n1;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
+                                     float* q_out_dev, int32_t batch, int32_t n_q_heads,
+                                     int32_t n_kv_heads, void* stream) {
+  if (!q_dev || !T_k_invT_dev || !q_out_dev || !valid_dtype(q_dtype)) return WUSHKV_EINVAL;
+  if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads) return WUSHKV_EINVAL;
+  if (n_q_heads / n_kv_heads > 16) return WUSHKV_EUNSUPPORTED;
+  if ((int64_t)batch * n_kv_heads > 2147483647LL) return WUSHKV_EUNSUPPORTED;
+  return cuda_status(launch_query_transform(q_dev, q_dtype, T_k_invT_dev, q_out_dev, batch,
+                                            n_q_heads, n_kv_heads, static_cast<cudaStream_t>(stream)));
+}
+
+wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
+                            float scale, void* stream) {
+  if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
+  if (cache->n == 0) return WUSHKV_EINVAL;
+  if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
+  const wushkv_config& c = cache->cfg;
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.c = dev_view(cache);
+  a.q = q_prime_dev;
+  a.out = out_dev;
+  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
+  a.scale_log2 = sc * 1.4426950408889634f;
+  const int64_t n = cache->n;
+  a.n_sink = (int)(n < c.sink ? n : c.sink);
+  a.n_packed = (int)packed_count(n, c);
+  a.n_recent = (int)(n - a.n_sink - a.n_packed);
+  a.ring_first = (int)(a.n_packed % (c.recent + c.chunk));
+  const int win = a.n_sink + a.n_recent;
+  a.win_tokens_per_split = WIN_TOKENS_PER_SPLIT;
+  a.win_splits = (win + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
+  a.pack_tokens_per_split = PACK_TOKENS_PER_SPLIT;
+  a.pack_splits = (a.n_packed + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
+  if (a.win_splits + a.pack_splits > a.c.max_splits) return WUSHKV_EINVAL;
+  a.partials = a.c.partials;
+  a.counters = a.c.counters;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head, int32_t kv,
+                            int32_t tok0, int32_t ntok, uint8_t* codes_host, uint16_t* meta_host,
+                            uint16_t* fp16_host, int8_t* kinds_host) {
+  if (!cache) return WUSHKV_EINVAL;
+  const wushkv_config& c = cache->cfg;
+  const wushkv_layout& L = cache->lay;
+  if (seq < 0 || seq >= c.batch || head < 0 || head >= c.n_kv_heads || (kv != 0 && kv != 1))
+    return WUSHKV_EINVAL;
+  if (tok0 < 0 || ntok < 0 || (int64_t)tok0 + ntok > cache->n) return WUSHKV_EINVAL;
+  const size_t u = (size_t)seq * c.n_kv_heads + head;
+  const int64_t n = cache->n;
+  const int64_t ns = n < c.sink ? n : c.sink;
+  const int64_t P = packed_count(n, c);
+  const int W = L.ring_slots;
+  // copy the unit's regions to host
+  std::vector<std::vector<uint32_t>> planes(L.n_planes);
+  for (int p = 0; p < L.n_planes; ++p) {
+    planes[p].resize(L.plane_unit_stride[p] / 4);
+    const uint64_t off = (kv == 0 ? L.k_plane_off[p] : L.v_plane_off[p]) + u * L.plane_unit_stride[p];
+    if (cudaMemcpy(planes[p].data(), cache->base + off, L.plane_unit_stride[p], cudaMemcpyDeviceToHost))
+      return WUSHKV_ECUDA;
+  }
+  std::vector<uint16_t> meta(L.meta_unit_stride / 2);
+  if (cudaMemcpy(meta.data(), cache->base + (kv == 0 ? L.k_meta_off : L.v_meta_off) + u * L.meta_unit_stride,
+                 L.meta_unit_stride, cudaMemcpyDeviceToHost))
+    return WUSHKV_ECUDA;
+  std::vector<uint16_t> sink((size_t)c.sink * 128), ring((size_t)W * 128);
+  if (c.sink > 0 &&
+      cudaMemcpy(sink.data(), cache->base + (kv == 0 ? L.sink_k_off : L.sink_v_off) + u * L.sink_unit_stride,
+                 L.sink_unit_stride, cudaMemcpyDeviceToHost))
+    return WUSHKV_ECUDA;
+  if (cudaMemcpy(ring.data(), cache->base + (kv == 0 ? L.ring_k_off : L.ring_v_off) + u * L.ring_unit_stride,
+                 L.ring_unit_stride, cudaMemcpyDeviceToHost))
+    return WUSHKV_ECUDA;
+  const int mb = (int)L.meta_bytes / 2;
+  for (int i = 0; i < ntok; ++i) {
+    const int64_t t = tok0 + i;
+    int kind;
+    if (t < ns) kind = 0;
+    else if (t < ns + P) kind = 1;
+    else kind = 2;
+    if (kinds_host) kinds_host[i] = (int8_t)kind;
+    if (kind == 1) {
+      const int64_t pk = t - c.sink;
+      uint8_t code[128] = {0};
+      int shift = 0;
+      for (int p = 0; p < L.n_planes; ++p) {
+        const int w = L.plane_bits[p], F = 8 / w;
+        const uint32_t mask = (1u << w) - 1u;
+        for (int d = 0; d < 128; ++d) {
+          uint32_t wd;
+          int bit;
+          if (kv == 0) {
+            const int ks = d / 32, rem = d % 32, h2 = rem / 16, c4 = (rem % 16) / 4, beta = d % 4;
+            const int rho = 4 * h2 + ks;
+            wd = planes[p][(size_t)pk * 4 * w + c4 * w + rho / F];
+            bit = 8 * beta + w * (rho % F);
+          } else {
+            const int mt = d / 16, rem = d % 16, rh = rem / 8, r = rem % 8;
+            const int rho = 2 * mt + rh, beta = (int)(pk % 4);
+            wd = planes[p][(size_t)(pk / 4) * 16 * w + r * 2 * w + rho / F];
+            bit = 8 * beta + w * (rho % F);
+          }
+          code[d] |= (uint8_t)(((wd >> bit) & mask) << shift);
+        }
+        shift += w;
+      }
+      if (codes_host) std::memcpy(codes_host + (size_t)i * 128, code, 128);
+      if (meta_host) {
+        meta_host[2 * i] = meta[(size_t)pk * mb];
+        meta_host[2 * i + 1] = mb == 2 ? meta[(size_t)pk * mb + 1] : 0;
+      }
+      if (fp16_host) std::memset(fp16_host + (size_t)i * 128, 0, 256);
+    } else {
+      const uint16_t* row = kind == 0 ? &sink[(size_t)t * 128]
+                                      : &ring[(size_t)((t - c.sink) % W) * 128];
+      if (fp16_host) std::memcpy(fp16_host + (size_t)i * 128, row, 256);
+      if (codes_host) std::memset(codes_host + (size_t)i * 128, 0, 128);
+      if (meta_host) { meta_host[2 * i] = 0; meta_host[2 * i + 1] = 0; }
+    }
+  }
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_device_status(const wushkv_cache* cache, int32_t clear, int32_t* out) {
+  if (!cache || !out) return WUSHKV_EINVAL;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, cache->base + cache->lay.status_off, 4, cudaMemcpyDeviceToHost))
+    return WUSHKV_ECUDA;
+  if (clear && cudaMemset(cache->base + cache->lay.status_off, 0, 4)) return WUSHKV_ECUDA;
+  *out = v;
+  return WUSHKV_OK;
+}
+
+}  // extern "C"

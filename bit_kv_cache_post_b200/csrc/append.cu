@@ -1,0 +1,203 @@
+// Append path: key transform after RoPE, fp16 sink/recent windows, chunked
+// flush of the recent window into the packed cache with per-token
+// quantisation and bit packing.
+//
+// Method source: summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化"
+// (ai-papers-daily), sections 工作参考价值 and 方法关键点: the key transform
+// follows RMSNorm and RoPE and costs one d x d product per new token; the
+// first 64 and the latest 256 tokens stay in fp16; the recent window is
+// quantised in chunks of 8 (or 16).
+//
+// One CTA (128 threads, one per dim) handles a run of 4-token quads of one
+// unit (sequence, KV head).  Quads are the packing granule of the V layout,
+// so a quad that reaches the packed cache is quantised and packed whole.
+#include "wushkv_internal.cuh"
+
+namespace wushkv {
+
+namespace {
+
+constexpr int TT_LD = 129;  // padded row of the transposed transform in smem
+
+__device__ __forceinline__ float load_in(const void* p, int dtype, size_t i) {
+  if (dtype == WUSHKV_F16) return __half2float(static_cast<const __half*>(p)[i]);
+  if (dtype == WUSHKV_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  return static_cast<const float*>(p)[i];
+}
+
+__device__ __forceinline__ float round_f16(float x) { return __half2float(__float2half_rn(x)); }
+
+// Token classes inside one append.
+enum : int { TOK_SKIP = 0, TOK_NEW = 1, TOK_FLUSH_OLD = 2 };
+
+__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* Tt = reinterpret_cast<float*>(smem_raw);          // [128][TT_LD] = T^T
+  float* kin = Tt + D * TT_LD;                             // [4][128] raw keys
+  float* k16 = kin + 4 * D;                                // [4][128] fp16 keys
+  float* v16 = k16 + 4 * D;                                // [4][128] fp16 values
+  uint8_t* codes = reinterpret_cast<uint8_t*>(v16 + 4 * D);  // [4][128]
+  __shared__ int kind_s[4];
+
+  const DevCache& c = a.c;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.y;
+  const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
+  const int64_t n0 = a.n0, n1 = a.n0 + a.n_tok;
+  const int64_t S = c.sink, P0 = a.packed0, P1 = a.packed1;
+  const int W = c.ring_slots;
+
+  const int64_t q_first = a.quad_begin + (int64_t)blockIdx.x * a.quads_per_cta;
+  const int64_t q_last = min(q_first + a.quads_per_cta, a.quad_begin + a.n_quads);
+  if (q_first >= q_last) return;
+
+  // Stage T^T of this head once per CTA if any new key needs the product.
+  const bool has_new = (4 * q_last > n0) && (4 * q_first < n1);
+  const bool transform = (a.T != nullptr) && has_new;
+  if (transform) {
+    const float* T = a.T + (size_t)h * D * D;
+    for (int idx = tid; idx < D * D; idx += 128) {
+      const int i = idx >> 7, j = idx & 127;
+      Tt[j * TT_LD + i] = T[idx];
+    }
+  }
+
+  const size_t plane_u0 = (size_t)u * c.plane_unit_stride[0];
+  const size_t plane_u1 = (size_t)u * c.plane_unit_stride[1];
+
+  for (int64_t Q = q_first; Q < q_last; ++Q) {
+    __syncthreads();  // previous quad's smem consumers are done
+    // ---- gather the quad's four tokens -------------------------------------
+    for (int j = 0; j < 4; ++j) {
+      const int64_t t = 4 * Q + j;
+      int kind = TOK_SKIP;
+      if (t >= n0 && t < n1) kind = TOK_NEW;
+      else if (t < n0 && t >= S + P0 && t < S + P1) kind = TOK_FLUSH_OLD;
+      if (tid == 0) kind_s[j] = kind;
+      if (kind == TOK_NEW) {
+        const size_t row = (((size_t)b * a.n_tok + (size_t)(t - n0)) * c.n_kv_heads + h) * D;
+        kin[j * D + tid] = load_in(a.k, a.dtype, row + tid);
+        v16[j * D + tid] = round_f16(load_in(a.v, a.dtype, row + tid));
+      } else if (kind == TOK_FLUSH_OLD) {
+        const int slot = (int)((t - S) % W);
+        const size_t off = ((size_t)u * W + slot) * D + tid;
+        k16[j * D + tid] = __half2float(c.ring_k[off]);
+        v16[j * D + tid] = __half2float(c.ring_v[off]);
+      }
+    }
+    __syncthreads();
+    // ---- key transform k' = T k (fp32 FMA), one output dim per thread ------
+    for (int j = 0; j < 4; ++j) {
+      if (kind_s[j] != TOK_NEW) continue;
+      float acc;
+      if (transform) {
+        acc = 0.f;
+        const float* kj = kin + j * D;
+#pragma unroll 8
+        for (int jj = 0; jj < D; ++jj) acc = fmaf(Tt[jj * TT_LD + tid], kj[jj], acc);
+      } else {
+        acc = kin[j * D + tid];
+      }
+      k16[j * D + tid] = round_f16(acc);
+    }
+    __syncthreads();
+    // ---- destinations --------------------------------------------------------
+    const int64_t t0 = 4 * Q;
+    const bool packed_quad = (t0 >= S) && (t0 + 4 <= S + P1) &&
+                             (kind_s[0] | kind_s[1] | kind_s[2] | kind_s[3]) != TOK_SKIP;
+    if (!packed_quad) {
+      for (int j = 0; j < 4; ++j) {
+        if (kind_s[j] != TOK_NEW) continue;
+        const int64_t t = t0 + j;
+        if (t < S) {
+          const size_t off = ((size_t)u * S + (size_t)t) * D + tid;
+          c.sink_k[off] = __float2half_rn(k16[j * D + tid]);
+          c.sink_v[off] = __float2half_rn(v16[j * D + tid]);
+        } else {
+          const int slot = (int)((t - S) % W);
+          const size_t off = ((size_t)u * W + slot) * D + tid;
+          c.ring_k[off] = __float2half_rn(k16[j * D + tid]);
+          c.ring_v[off] = __float2half_rn(v16[j * D + tid]);
+        }
+      }
+      continue;
+    }
+    // ---- quantise + pack a whole quad -------------------------------------------
+    const int64_t pk = t0 - S;  // packed index of the quad's first token
+    for (int kv = 0; kv < 2; ++kv) {
+      const float* src = (kv == 0 ? k16 : v16) + warp * D;
+      float x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = src[4 * lane + i];
+      uint8_t cd[4];
+      uint8_t* meta = (kv == 0 ? c.k_meta : c.v_meta) + (size_t)u * c.meta_unit_stride +
+                      (size_t)(pk + warp) * c.meta_bytes;
+      if (c.quantizer == WUSHKV_QUEST_INT) {
+        __half dl;
+        quest_warp(x, c.bits, c.alpha, cd, dl);
+        if (lane == 0) *reinterpret_cast<__half*>(meta) = dl;
+      } else {
+        __half s, lo;
+        affine_warp(x, c.bits, c.r_lo, c.r_hi, cd, s, lo);
+        if (lane == 0) *reinterpret_cast<__half2*>(meta) = __halves2half2(s, lo);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) codes[warp * D + 4 * lane + i] = cd[i];
+      __syncthreads();
+      for (int p = 0; p < c.n_planes; ++p) {
+        const int w = c.plane_bits[p], P = 8 / w;
+        uint8_t* base = (kv == 0 ? c.k_plane[p] : c.v_plane[p]) + (p == 0 ? plane_u0 : plane_u1);
+        if (kv == 0) {
+          // four K rows, 4w words each: warp = token, lane = word
+          if (lane < 4 * w) {
+            uint32_t word = 0;
+            for (int s = 0; s < P; ++s)
+              for (int beta = 0; beta < 4; ++beta) {
+                const int dim = k_field_dim(lane, w, s, beta);
+                word |= plane_value(codes[warp * D + dim], c.bits, p) << (8 * beta + w * s);
+              }
+            reinterpret_cast<uint32_t*>(base + (size_t)(pk + warp) * 16 * w)[lane] = word;
+          }
+        } else {
+          // one V quad, 16w words
+          if (tid < 16 * w) {
+            uint32_t word = 0;
+            for (int s = 0; s < P; ++s) {
+              const int dim = v_field_dim(tid, w, s);
+              for (int beta = 0; beta < 4; ++beta)
+                word |= plane_value(codes[beta * D + dim], c.bits, p) << (8 * beta + w * s);
+            }
+            reinterpret_cast<uint32_t*>(base + (size_t)(pk / 4) * 64 * w)[tid] = word;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+}  // namespace
+
+size_t append_smem_bytes() {
+  return (size_t)(D * TT_LD + 3 * 4 * D) * sizeof(float) + 4 * D;
+}
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
+  const size_t smem = append_smem_bytes();
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int attr_done[64] = {0};
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  if (a.n_quads <= 0) return cudaSuccess;
+  const int64_t gx = (a.n_quads + a.quads_per_cta - 1) / a.quads_per_cta;
+  dim3 grid((unsigned)gx, (unsigned)a.c.units);
+  append_kernel<<<grid, 128, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace wushkv

@@ -1,0 +1,235 @@
+// Internal declarations shared by the libwushkv kernels and host code.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "wushkv.h"
+
+namespace wushkv {
+
+constexpr int D = 128;           // head_dim
+constexpr unsigned FULL = 0xffffffffu;
+
+// Device-visible view of one cache buffer.
+struct DevCache {
+  uint8_t* k_plane[2];
+  uint8_t* v_plane[2];
+  uint64_t plane_unit_stride[2];     // bytes per unit (K and V alike)
+  int n_planes;
+  int plane_bits[2];
+  int bits;
+  int quantizer;
+  uint8_t* k_meta;
+  uint8_t* v_meta;
+  int meta_bytes;                    // 2 (QuEST delta) or 4 (affine scale, lo)
+  uint64_t meta_unit_stride;         // bytes per unit
+  __half* sink_k;
+  __half* sink_v;
+  __half* ring_k;
+  __half* ring_v;
+  int sink, recent, chunk, ring_slots;
+  int packed_capacity;
+  float* partials;                   // split-K workspace
+  int* counters;                     // one arrival counter per unit
+  int max_splits;
+  int* status;                       // sticky device error word
+  int units, n_kv_heads, group;
+  double alpha;                      // QuEST clip ratio
+  int r_lo, r_hi;                    // affine ranks (1-indexed)
+};
+
+// Status bits a kernel may set in the sticky word.
+enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2 };
+
+// ---------------------------------------------------------------------------
+// Exact-rounding helpers
+// ---------------------------------------------------------------------------
+
+// float64 -> fp16, round to nearest even, rounded once.  Written from the
+// IEEE 754 binary16 definition: pick the fp16 quantum (2^(e-10), or 2^-24 in
+// the subnormal range), round |x| / quantum to the nearest even integer in
+// float64 (exact: power-of-two scaling), and rebuild.  The rebuilt value is
+// an fp16 value, so the final float -> half conversion is exact.
+__device__ __forceinline__ __half f64_to_f16_rn(double x) {
+  double a = fabs(x);
+  if (!(a > 0.0)) return __float2half_rn((float)x);          // 0, -0, NaN
+  if (a >= 65520.0) return __float2half_rn(x > 0 ? INFINITY : -INFINITY);
+  int e = ilogb(a);                                          // floor(log2 a)
+  if (e < -14) e = -14;
+  double q = rint(ldexp(a, 10 - e));                         // ties to even
+  double v = ldexp(q, e - 10);
+  return __float2half_rn((float)(x < 0 ? -v : v));
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Per-token quantisers on one warp.  Lane l holds dims 4l..4l+3 of the token
+// as float values that are exactly fp16 values.
+// ---------------------------------------------------------------------------
+
+// QuEST INT: RMS-based scale, symmetric mid-rise grid, bin-centre
+// reconstruction (review "[논문리뷰] WUSH-KV ...", Key Terms, QuEST entry).
+// delta = fp16(alpha * rms / 2^(bits-1)); code = clamp(floor(x/delta + L/2)).
+__device__ __forceinline__ void quest_warp(const float x[4], int bits, double alpha,
+                                           uint8_t code[4], __half& delta) {
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ss = __fma_rn((double)x[i], (double)x[i], ss);
+  ss = warp_sum_f64(ss);
+  const double rms = __dsqrt_rn(ss / 128.0);
+  const double dd = __dmul_rn(alpha, rms) / (double)(1 << (bits - 1));
+  delta = f64_to_f16_rn(dd);
+  const float d32 = __half2float(delta);
+  const int L = 1 << bits;
+  const float inv = __frcp_rn(d32);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float t = __fadd_rn(__fmul_rn(x[i], inv), (float)(L / 2));
+    t = fminf(fmaxf(floorf(t), 0.f), (float)(L - 1));
+    code[i] = (d32 == 0.f) ? (uint8_t)(L / 2) : (uint8_t)(int)t;
+  }
+}
+
+// k-th smallest (1-indexed, k <= 8) of the warp's 128 values; ties are
+// removed one occurrence per round, so the result is the order statistic.
+__device__ __forceinline__ float warp_kth_smallest(const float x[4], int k) {
+  const int lane = threadIdx.x & 31;
+  unsigned taken = 0;
+  float m = 0.f;
+  for (int round = 0; round < k; ++round) {
+    float lm = INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (!(taken >> i & 1)) lm = fminf(lm, x[i]);
+    float g = lm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g = fminf(g, __shfl_xor_sync(FULL, g, o));
+    const unsigned who = __ballot_sync(FULL, lm == g);
+    if (lane == __ffs(who) - 1) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (!(taken >> i & 1) && x[i] == g) { taken |= 1u << i; break; }
+    }
+    m = g;
+  }
+  return m;
+}
+
+__device__ __forceinline__ float warp_kth_largest(const float x[4], int k) {
+  float y[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) y[i] = -x[i];
+  return -warp_kth_smallest(y, k);
+}
+
+// Percentile-clipped affine quantiser (summary page 方法关键点, 4th bullet):
+// lo/hi = order statistics r_lo, r_hi; s = fp16((hi - lo) / (L - 1));
+// code = clamp(rint((x - lo) / s)).  Zeros are canonicalised to +0.
+__device__ __forceinline__ void affine_warp(const float x[4], int bits, int r_lo, int r_hi,
+                                            uint8_t code[4], __half& s_out, __half& lo_out) {
+  const int L = 1 << bits;
+  float lo = warp_kth_smallest(x, r_lo);
+  float hi = warp_kth_largest(x, 129 - r_hi);
+  lo = __fadd_rn(lo, 0.f);
+  hi = __fadd_rn(hi, 0.f);
+  lo_out = __float2half_rn(lo);
+  const float s32 = __fdiv_rn(__fsub_rn(hi, lo), (float)(L - 1));
+  s_out = __float2half_rn(s32);
+  const float sd = __half2float(s_out);
+  const float lo_h = __half2float(lo_out);
+  const float inv = __frcp_rn(sd);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float t = __fmul_rn(__fsub_rn(x[i], lo_h), inv);
+    t = fminf(fmaxf(rintf(t), 0.f), (float)(L - 1));
+    code[i] = (sd == 0.f) ? (uint8_t)0 : (uint8_t)(int)t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Packed format index maps (see the layout comment in wushkv.h)
+// ---------------------------------------------------------------------------
+
+// K row: dim of field s, byte beta of word wi in a plane of width w.
+__device__ __forceinline__ int k_field_dim(int wi, int w, int s, int beta) {
+  const int P = 8 / w;
+  const int c = wi / w, sub = wi % w;
+  const int rho = sub * P + s;
+  const int h = rho >> 2, ks = rho & 3;
+  return 32 * ks + 4 * c + 16 * h + beta;
+}
+
+// V quad: dim of field s, byte beta (token) of word wi (= r*2w + j).
+__device__ __forceinline__ int v_field_dim(int wi, int w, int s) {
+  const int P = 8 / w;
+  const int r = wi / (2 * w), j = wi % (2 * w);
+  const int rho = j * P + s;
+  const int mt = rho >> 1, rh = rho & 1;
+  return 16 * mt + r + 8 * rh;
+}
+
+// Value of plane p (width w) of a code: 3-bit codes split into a 2-bit low
+// plane and a 1-bit high plane.
+__device__ __forceinline__ uint32_t plane_value(uint32_t code, int bits, int p) {
+  if (bits == 3) return p == 0 ? (code & 3u) : (code >> 2);
+  return code;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in the .cu files)
+// ---------------------------------------------------------------------------
+struct AppendArgs {
+  DevCache c;
+  const void* k;           // [B][n_tok][Hkv][128]
+  const void* v;
+  int dtype;
+  const float* T;          // [Hkv][128][128] or null
+  int n_tok;
+  int64_t n0;              // tokens before this append
+  int64_t packed0, packed1;  // packed counts before / after
+  int64_t quad_begin;      // first absolute quad (4 tokens) handled
+  int64_t n_quads;         // quads handled by this launch
+  int quads_per_cta;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+
+cudaError_t launch_query_transform(const void* q, int dtype, const float* TinvT, float* out,
+                                   int batch, int n_q_heads, int n_kv_heads, cudaStream_t s);
+
+struct DecodeArgs {
+  DevCache c;
+  const float* q;          // [B][Hq][128] fp32
+  float* out;              // [B][Hq][128] fp32
+  float scale_log2;        // scale * log2(e)
+  int n_sink, n_packed, n_recent;
+  int ring_first;          // ring slot of the oldest recent token
+  int win_splits;          // CTAs per unit for sink + recent tokens
+  int win_tokens_per_split;
+  int pack_splits;         // CTAs per unit for packed tokens
+  int pack_tokens_per_split;
+  float* partials;         // workspace for split partials
+  int* counters;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace wushkv

@@ -1,0 +1,214 @@
+/*
+ * wushkv.h -- C ABI of libwushkv.so: the online hot path of WUSH-KV
+ * ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms",
+ * arXiv 2609.38121) on NVIDIA B200 (sm_100a).
+ *
+ * Method facts this library implements (sources are the summary pages of the
+ * paper; page titles and sections are named at each call below):
+ *   - every KV head owns an invertible d x d key transform T_k applied after
+ *     RoPE (k' = T_k k, one d x d product per new token), and queries use its
+ *     inverse transpose (q' = T_k^{-T} q) so that q'.k' = q.k;
+ *   - values arrive already transformed (the value transform is folded into
+ *     W_V and W_O offline), so the cache stores them as given;
+ *   - keys and values are quantised per token to 2, 3 or 4 bits with QuEST
+ *     INT (RMS-based scale, bin-centre reconstruction) or a percentile-clipped
+ *     affine quantiser, and bit-packed;
+ *   - the first `sink` tokens and the latest `recent` tokens stay in fp16;
+ *     the recent window is flushed to the packed cache `chunk` tokens at a
+ *     time;
+ *   - decoding is grouped-query attention over the packed cache plus the
+ *     fp16 windows.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named *_dev are device pointers; *_host are host pointers.
+ *     The library borrows them for the duration of the call (asynchronous
+ *     calls: until the work on `stream` completes).  It never allocates
+ *     device memory: the caller allocates the cache buffer
+ *     (wushkv_cache_bytes) and every input and output.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Compute calls are asynchronous on it.
+ *   - Argument errors are detected on the host before any launch and
+ *     returned synchronously; nothing is written in that case.  CUDA launch
+ *     errors return WUSHKV_ECUDA.  Errors found inside kernels set a sticky
+ *     device status word read by wushkv_device_status.
+ *   - head_dim is 128.  KV head of query head h is floor(h / G), G =
+ *     n_q_heads / n_kv_heads (contiguous groups).
+ *   - One cache object holds one layer for `batch` sequences that all hold
+ *     the same number of tokens (every append adds n_tok to each sequence).
+ *   - A "unit" is one (sequence b, KV head h); unit index u = b*n_kv_heads+h.
+ */
+#ifndef WUSHKV_H
+#define WUSHKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WUSHKV_API __attribute__((visibility("default")))
+#else
+#define WUSHKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WUSHKV_OK = 0,
+  WUSHKV_EINVAL = 1,        /* bad argument (NULL pointer, mismatched bits, ...) */
+  WUSHKV_ECAPACITY = 2,     /* append would exceed max_ctx; nothing written   */
+  WUSHKV_EUNSUPPORTED = 3,  /* valid but not built (head_dim != 128, ...)     */
+  WUSHKV_ECUDA = 4          /* a CUDA runtime call failed                     */
+} wushkv_status;
+
+typedef enum { WUSHKV_QUEST_INT = 0, WUSHKV_AFFINE_PCTCLIP = 1 } wushkv_quantizer;
+typedef enum { WUSHKV_F16 = 0, WUSHKV_BF16 = 1, WUSHKV_F32 = 2 } wushkv_dtype;
+
+/* Cache configuration (one layer).
+ *   batch, n_kv_heads, n_q_heads: GQA shape; n_q_heads % n_kv_heads == 0 and
+ *     G = n_q_heads / n_kv_heads in {1, 2, 4, 8}.
+ *   head_dim: must be 128.
+ *   max_ctx: tokens per sequence the cache can hold (>= 1).
+ *   bits: 2, 3 or 4.  quantizer: wushkv_quantizer.
+ *   sink, recent, chunk: window sizes (summary page "WUSH-KV：数据自适应变换的
+ *     KV Cache 低比特量化", sections 工作参考价值 and 方法关键点: 64, 256 and
+ *     8 or 16).  sink % 4 == 0, chunk % 4 == 0, chunk >= 4, recent >= 0.
+ *   quest_alpha: QuEST clip ratio (clip range +-alpha * RMS); 0 selects the
+ *     Gaussian-MSE-optimal default for `bits` (wushkv_default_quest_alpha).
+ *     Must satisfy 0 < alpha <= 2^(bits-1).
+ *   clip_lo_rank, clip_hi_rank: affine quantiser order statistics (1-indexed
+ *     ranks among the 128 values; default 2 and 127).  Supported:
+ *     1 <= lo <= 8, 121 <= hi <= 128.
+ */
+typedef struct {
+  int32_t batch, n_kv_heads, n_q_heads, head_dim, max_ctx, bits;
+  int32_t quantizer;
+  int32_t sink, recent, chunk;
+  double quest_alpha;
+  int32_t clip_lo_rank, clip_hi_rank;
+} wushkv_config;
+
+typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
+
+/* Byte layout of a cache buffer (offsets from the buffer base).  Exposed so
+ * that callers can checkpoint, inspect or move the cache.  Packed format:
+ *   planes: 2-bit codes -> one 2-bit plane, 4-bit -> one 4-bit plane, 3-bit
+ *     -> a 2-bit plane of (code & 3) and a 1-bit plane of (code >> 2).  A
+ *     plane of width w packs 8/w fields per byte; field s of byte beta of a
+ *     little-endian 32-bit word is at bit 8*beta + w*s.
+ *   K (token rows, 16*w bytes per token per plane): c in 0..3, h in 0..1,
+ *     ks in 0..3, beta in 0..3, rho = 4h + ks: word c*w + rho/(8/w), field
+ *     rho % (8/w), dim 32ks + 4c + 16h + beta.
+ *   V (4-token quads, 64*w bytes per quad per plane): r in 0..7, rho in
+ *     0..15 (mt = rho/2, rh = rho%2), beta in 0..3: word r*2w + rho/(8/w),
+ *     field rho % (8/w), dim 16mt + r + 8rh, token 4*quad + beta.
+ *   meta: per token, fp16 delta (QuEST, 2 bytes) or fp16 (scale, lo) pair
+ *     (affine, 4 bytes); K and V separately.
+ *   sink, ring: fp16 [unit][slot][128]; ring slot of post-sink token t is
+ *     (t - sink) mod (recent + chunk). */
+typedef struct {
+  int32_t n_planes;
+  int32_t plane_bits[2];
+  int32_t packed_capacity;          /* token slots per unit in the packed region */
+  uint64_t k_plane_off[2], v_plane_off[2];
+  uint64_t plane_unit_stride[2];    /* bytes per unit, K and V alike */
+  uint64_t k_meta_off, v_meta_off;
+  uint32_t meta_bytes;              /* per token: 2 (QuEST) or 4 (affine) */
+  uint64_t meta_unit_stride;
+  uint64_t sink_k_off, sink_v_off, sink_unit_stride;
+  uint64_t ring_k_off, ring_v_off, ring_unit_stride;
+  int32_t ring_slots;               /* recent + chunk */
+  uint64_t workspace_off, workspace_bytes;
+  uint64_t status_off;
+  uint64_t total_bytes;
+} wushkv_layout;
+
+/* Bytes of device memory a cache with this configuration needs (0 if the
+ * configuration is invalid).  Includes the split-K decode workspace and the
+ * device status word. */
+WUSHKV_API size_t wushkv_cache_bytes(const wushkv_config* cfg);
+
+/* Create a cache over caller-allocated device memory `dev_mem` of `bytes`
+ * bytes (>= wushkv_cache_bytes(cfg), 256-byte aligned).  Zeroes the buffer
+ * asynchronously on `stream`.  On success *out receives a host handle that
+ * owns only host metadata (free it with wushkv_cache_destroy; the device
+ * buffer stays the caller's).  Errors: EINVAL, EUNSUPPORTED, ECUDA. */
+WUSHKV_API wushkv_status wushkv_cache_create(const wushkv_config* cfg, void* dev_mem, size_t bytes,
+                                  void* stream, wushkv_cache** out);
+WUSHKV_API wushkv_status wushkv_cache_destroy(wushkv_cache* cache);
+
+/* Fill *out with the byte layout of this cache. */
+WUSHKV_API wushkv_status wushkv_cache_layout(const wushkv_cache* cache, wushkv_layout* out);
+
+/* Current token counts per sequence: total, sink, packed, recent (host-side
+ * bookkeeping, no synchronisation).  Any pointer may be NULL. */
+WUSHKV_API wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t* n_tokens, int64_t* n_sink,
+                                  int64_t* n_packed, int64_t* n_recent);
+
+/* Append n_tok tokens to every sequence.
+ *   Source: summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
+ *   方法关键点 (key transform after RoPE, one d x d product per new token;
+ *   quantiser choice; sink/recent windows with chunked flush).
+ *   k_rope_dev: [batch][n_tok][n_kv_heads][128] post-RoPE keys, dtype in_dtype.
+ *   v_dev:      [batch][n_tok][n_kv_heads][128] values (already in the
+ *               transformed value space), dtype in_dtype.
+ *   T_k_dev:    [n_kv_heads][128][128] fp32 row-major, k'_i = sum_j T[i][j] k_j;
+ *               NULL means the keys are already transformed (no product).
+ *   bits, quantizer: must equal the cache's configuration (EINVAL otherwise).
+ * Every key and value is rounded once to fp16; tokens landing in the sink or
+ * recent window are stored as those fp16 values, tokens that the window
+ * policy sends to the packed cache are quantised from them.  The resulting
+ * state depends only on the token count, not on how appends were batched.
+ * ECAPACITY if n_tokens + n_tok > max_ctx (nothing written). */
+WUSHKV_API wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                            int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
+                            int32_t quantizer, void* stream);
+
+/* q' = T_k^{-T} q for every query head, with the transform of its KV group.
+ *   Source: same page, 方法关键点 and 工作参考价值 (one d x d product per
+ *   query; inverse transpose keeps q'.k' = q.k).
+ *   q_dev:        [batch][n_q_heads][128], dtype q_dtype.
+ *   T_k_invT_dev: [n_kv_heads][128][128] fp32 row-major, q'_i = sum_j M[i][j] q_j.
+ *   q_out_dev:    [batch][n_q_heads][128] fp32 (kept fp32 for the decode). */
+WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
+                                     float* q_out_dev, int32_t batch, int32_t n_q_heads,
+                                     int32_t n_kv_heads, void* stream);
+
+/* GQA decode attention of one query per query head over the whole cache.
+ *   Source: review "[논문리뷰] WUSH-KV ..." (secrett2633), Key Terms (GQA);
+ *   dequantisation happens inside the score and PV loops.
+ *   q_prime_dev: [batch][n_q_heads][128] fp32 transformed queries.
+ *   out_dev:     [batch][n_q_heads][128] fp32 = softmax(scale q'.k'^T) v
+ *                in the transformed value space.
+ *   scale: softmax scale; 0 selects 1/sqrt(128).
+ * Uses the cache's workspace region for split-K partials; calls on the same
+ * cache must therefore be stream-ordered.  EINVAL if the cache is empty. */
+WUSHKV_API wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
+                            float scale, void* stream);
+
+/* Copy tokens [tok0, tok0 + ntok) of unit (seq, head), K (kv = 0) or V
+ * (kv = 1), to host memory.  Synchronous (waits for the device).
+ *   codes_host: [ntok][128] uint8, unpacked codes (0 for window tokens); or NULL.
+ *   meta_host:  [ntok][2] uint16 fp16 bits: (delta, 0) for QuEST, (scale, lo)
+ *               for affine (0 for window tokens); or NULL.
+ *   fp16_host:  [ntok][128] uint16 fp16 bits of window tokens (0 for packed
+ *               tokens); or NULL.
+ *   kinds_host: [ntok] int8: 0 sink, 1 packed, 2 recent; or NULL. */
+WUSHKV_API wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head, int32_t kv,
+                            int32_t tok0, int32_t ntok, uint8_t* codes_host, uint16_t* meta_host,
+                            uint16_t* fp16_host, int8_t* kinds_host);
+
+/* Read (and with clear != 0, reset) the sticky device status word;
+ * synchronises the device.  0 means no kernel reported an error. */
+WUSHKV_API wushkv_status wushkv_device_status(const wushkv_cache* cache, int32_t clear, int32_t* out);
+
+/* Gaussian-MSE-optimal QuEST clip ratio for 2, 3 or 4 bits (0 otherwise). */
+WUSHKV_API double wushkv_default_quest_alpha(int32_t bits);
+
+/* Static description of a status code. */
+WUSHKV_API const char* wushkv_strerror(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WUSHKV_H */

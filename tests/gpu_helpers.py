@@ -1,0 +1,98 @@
+"""Shared helpers of the GPU parity tests: build the CUDA cache and the
+oracle cache from the same seeded inputs and read raw device regions."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from oracle import wushkv_oracle as O
+
+
+def torch_dtype(name):
+    import torch
+    return {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[name]
+
+
+def rounded(x: np.ndarray, name: str) -> np.ndarray:
+    """float32 values after rounding to the input dtype (what both sides read)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch_dtype(name)).float().numpy()
+
+
+def to_dev(x: np.ndarray, name: str):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch_dtype(name)).cuda().contiguous()
+
+
+def region(cache, off: int, nbytes: int) -> np.ndarray:
+    """Raw bytes [off, off + nbytes) of a cache buffer as uint8."""
+    start = cache.base_ptr - cache.buffer.data_ptr() + off
+    return cache.buffer[start:start + nbytes].cpu().numpy()
+
+
+def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
+    """The packed plane bytes of unit u for its first n_packed tokens, as
+    uint32 arrays shaped like the oracle's pack_* output."""
+    L = cache.layout()
+    out = []
+    for p in range(L.n_planes):
+        w = L.plane_bits[p]
+        base = (L.k_plane_off[p] if kv == 0 else L.v_plane_off[p]) + u * L.plane_unit_stride[p]
+        raw = region(cache, base, n_packed * 16 * w).view(np.uint32)
+        out.append(raw.reshape(n_packed, 4 * w) if kv == 0 else raw.reshape(n_packed // 4, 16 * w))
+    return out
+
+
+def unit_meta(cache, u: int, kv: int, n_packed: int) -> np.ndarray:
+    L = cache.layout()
+    base = (L.k_meta_off if kv == 0 else L.v_meta_off) + u * L.meta_unit_stride
+    raw = region(cache, base, n_packed * L.meta_bytes).view(np.float16)
+    return raw.reshape(n_packed, L.meta_bytes // 2)
+
+
+def unit_window(cache, u: int, kv: int, which: str) -> np.ndarray:
+    L = cache.layout()
+    if which == "sink":
+        off = (L.sink_k_off if kv == 0 else L.sink_v_off) + u * L.sink_unit_stride
+        n = L.sink_unit_stride
+    else:
+        off = (L.ring_k_off if kv == 0 else L.ring_v_off) + u * L.ring_unit_stride
+        n = L.ring_unit_stride
+    return region(cache, off, n).view(np.float16).reshape(-1, 128)
+
+
+def oracle_cfg(cfg) -> O.CacheConfig:
+    return O.CacheConfig(batch=cfg.batch, n_kv_heads=cfg.n_kv_heads, n_q_heads=cfg.n_q_heads,
+                         max_ctx=cfg.max_ctx, bits=cfg.bits, quantizer=cfg.quantizer,
+                         sink=cfg.sink, recent=cfg.recent, chunk=cfg.chunk,
+                         alpha=(cfg.quest_alpha or None), r_lo=cfg.clip_lo_rank,
+                         r_hi=cfg.clip_hi_rank)
+
+
+def compare_cache_bitexact(cache, oc: O.OracleCache, units=None):
+    """Every byte of the packed planes, meta, sink and recent rows of the
+    given units equals the oracle's."""
+    ns, P, nr = oc.split()
+    assert cache.tokens() == (oc.n, ns, P, nr)
+    L = cache.layout()
+    for u in (range(oc.cfg.units) if units is None else units):
+        for kv in (0, 1):
+            want = oc.packed_k(u) if kv == 0 else oc.packed_v(u)
+            got = unit_packed_planes(cache, u, kv, P)
+            for p in range(L.n_planes):
+                assert np.array_equal(got[p], want[p]), (u, kv, p)
+            meta = unit_meta(cache, u, kv, P)
+            om = (oc.meta_k if kv == 0 else oc.meta_v)[u, :P, :meta.shape[1]]
+            assert np.array_equal(meta.view(np.uint16), om.view(np.uint16)), (u, kv)
+            sink = unit_window(cache, u, kv, "sink")[:ns]
+            osink = (oc.sink_k if kv == 0 else oc.sink_v)[u, :ns]
+            assert np.array_equal(sink.view(np.uint16), osink.view(np.uint16)), (u, kv)
+            ring = unit_window(cache, u, kv, "ring")[oc.recent_order()]
+            oring = (oc.ring_k if kv == 0 else oc.ring_v)[u, oc.recent_order()]
+            assert np.array_equal(ring.view(np.uint16), oring.view(np.uint16)), (u, kv)
+
+
+def rel_rms_err(got: np.ndarray, want: np.ndarray) -> float:
+    """max |got - want| / RMS(want)."""
+    return float(np.abs(got - want).max() / math.sqrt(float(np.mean(want ** 2))))
