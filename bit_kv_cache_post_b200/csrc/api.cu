@@ -447,3 +447,79 @@ wushkv_status wushkv_device_status(const wushkv_cache* cache, int32_t clear, int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at decode time: code running inside a
+// host allocator hook, plug-ins whose host application owns every device
+// allocation, or engines that forbid allocation after start-up.  For them
+// the split-K partials and arrival counters of the decode live in this
+// file-scope device array instead of the cache buffer's workspace.  The
+// array is a fixed 8 MiB and stays resident on every GPU that loads the
+// library until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(8) << 20;
+constexpr size_t NOALLOC_COUNTER_BYTES = size_t(65536) * sizeof(int);  // one per unit
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch, looked up once per device.  In host
+// code the symbol itself is only a host-side stand-in for the array.
+void* g_noalloc_addr[64] = {nullptr};
+
+}  // namespace
+
+extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const wushkv_cache* cache,
+                                                float* out_dev, float scale, void* stream) {
+  if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
+  if (cache->n == 0) return WUSHKV_EINVAL;
+  if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSHKV_ECUDA;
+  if (dev < 0 || dev >= 64) return WUSHKV_EUNSUPPORTED;
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return WUSHKV_ECUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  const wushkv_config& c = cache->cfg;
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.c = dev_view(cache);
+  a.q = q_prime_dev;
+  a.out = out_dev;
+  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
+  a.scale_log2 = sc * 1.4426950408889634f;
+  const int64_t n = cache->n;
+  a.n_sink = (int)(n < c.sink ? n : c.sink);
+  a.n_packed = (int)packed_count(n, c);
+  a.n_recent = (int)(n - a.n_sink - a.n_packed);
+  a.ring_first = (int)(a.n_packed % (c.recent + c.chunk));
+  const int win = a.n_sink + a.n_recent;
+  a.win_tokens_per_split = WIN_TOKENS_PER_SPLIT;
+  a.win_splits = (win + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
+  a.pack_tokens_per_split = PACK_TOKENS_PER_SPLIT;
+  a.pack_splits = (a.n_packed + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
+  const int total = a.win_splits + a.pack_splits;
+  if (total > a.c.max_splits) return WUSHKV_EINVAL;
+  // The partials of this call are packed densely: stride = this call's splits.
+  a.c.max_splits = total;
+  const size_t units = (size_t)a.c.units;
+  const size_t partial_bytes = units * (size_t)total * a.c.group * (128 + 2) * sizeof(float);
+  if (units * sizeof(int) > NOALLOC_COUNTER_BYTES ||
+      partial_bytes > NOALLOC_SCRATCH_BYTES - NOALLOC_COUNTER_BYTES)
+    return WUSHKV_ECAPACITY;
+  unsigned char* base = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+  a.counters = reinterpret_cast<int*>(base);
+  a.partials = reinterpret_cast<float*>(base + NOALLOC_COUNTER_BYTES);
+  a.c.counters = a.counters;
+  a.c.partials = a.partials;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: arrival counters must
+  // start at zero.
+  if (cudaMemsetAsync(a.counters, 0, units * sizeof(int), s) != cudaSuccess) return WUSHKV_ECUDA;
+  return cuda_status(launch_decode(a, s));
+}

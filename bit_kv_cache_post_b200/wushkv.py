@@ -20,6 +20,7 @@ EXPORTED = [
     "wushkv_cache_bytes", "wushkv_cache_create", "wushkv_cache_destroy", "wushkv_cache_layout",
     "wushkv_cache_tokens", "wushkv_append", "wushkv_query_transform", "wushkv_decode",
     "wushkv_export", "wushkv_device_status", "wushkv_default_quest_alpha", "wushkv_strerror",
+    "wushkv_decode_noalloc",
 ]
 
 
@@ -77,6 +78,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_append.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, vp]
     lib.wushkv_query_transform.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp]
     lib.wushkv_decode.argtypes = [vp, vp, vp, ctypes.c_float, vp]
+    lib.wushkv_decode_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_export.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.wushkv_device_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
     lib.wushkv_default_quest_alpha.argtypes = [i32]
@@ -194,6 +196,17 @@ class Cache:
             out = torch.empty_like(q_prime)
         _check(load().wushkv_decode(q_prime.data_ptr(), self._handle, out.data_ptr(), scale,
                                     _stream_ptr(stream)), "wushkv_decode")
+        return out
+
+    def decode_noalloc(self, q_prime, out=None, scale: float = 0.0, stream=None):
+        """As decode(), for callers that cannot allocate device memory: the
+        split-K scratch lives in the library's fixed 8 MiB device array."""
+        import torch
+        assert q_prime.is_contiguous() and q_prime.dtype == torch.float32
+        if out is None:
+            out = torch.empty_like(q_prime)
+        _check(load().wushkv_decode_noalloc(q_prime.data_ptr(), self._handle, out.data_ptr(),
+                                            scale, _stream_ptr(stream)), "wushkv_decode_noalloc")
         return out
 
     def export(self, seq: int, head: int, kv: int, tok0: int, ntok: int):

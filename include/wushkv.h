@@ -186,6 +186,31 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
 WUSHKV_API wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream);
 
+/* Decode for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a deployment convenience around wushkv_decode.
+ * Some callers cannot call cudaMalloc when they decode -- code running inside
+ * a host application's allocator hook, plug-ins whose host owns every device
+ * allocation, or serving engines that forbid allocation after start-up.
+ * This entry point takes the same inputs and writes the same output as
+ * wushkv_decode, but keeps its split-K partials and arrival counters in a
+ * fixed 8 MiB array inside the library (a file-scope __device__ array that
+ * every GPU which loads the library holds until the process exits) instead of
+ * the cache buffer's workspace.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array, which keeps the previous call's
+ *     contents; each call zeroes its arrival counters first.  Calls that
+ *     overlap on the GPU (other streams, threads or caches) race: issue
+ *     them one after another.
+ *   - WUSHKV_ECAPACITY, with nothing launched, when this call's partials
+ *     (units x splits x G x 520 bytes) exceed 8 MiB minus 256 KiB of
+ *     counters, or the cache has more than 65536 units.
+ * Other errors as wushkv_decode. */
+WUSHKV_API wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const wushkv_cache* cache,
+                                               float* out_dev, float scale, void* stream);
+
 /* Copy tokens [tok0, tok0 + ntok) of unit (seq, head), K (kv = 0) or V
  * (kv = 1), to host memory.  Synchronous (waits for the device).
  *   codes_host: [ntok][128] uint8, unpacked codes (0 for window tokens); or NULL.
