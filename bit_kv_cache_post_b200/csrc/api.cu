@@ -22,10 +22,15 @@ namespace {
 
 using namespace wushkv;
 
-// Decode split policy: tokens per CTA for the fp16 windows and for the
-// packed cache.  max_splits in the workspace is sized from these.
-constexpr int WIN_TOKENS_PER_SPLIT = 128;
-constexpr int PACK_TOKENS_PER_SPLIT = 512;
+// Decode split policy: each unit is cut into `splits` CTAs of equal bytes
+// (window groups of 32 fp16 tokens, packed blocks of 64 tokens) so that the
+// grid fills one wave of resident CTAs; no split is smaller than
+// MIN_SPLIT_BYTES.  The workspace holds up to max(1, MAX_GRID / units)
+// splits per unit.
+constexpr int WIN_GROUP = 32;
+constexpr int PACK_BLOCK = 64;
+constexpr int64_t MIN_SPLIT_BYTES = 32 * 1024;
+constexpr int MAX_GRID = 2048;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -95,9 +100,11 @@ wushkv_status check_config(const wushkv_config* c) {
 }
 
 int max_splits_for(const wushkv_config& c, int packed_capacity) {
-  const int win = (c.sink + c.recent + c.chunk + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
-  const int pack = (packed_capacity + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
-  return (win > 0 ? win : 1) + pack;
+  const int items = (c.sink + c.recent + c.chunk + WIN_GROUP - 1) / WIN_GROUP +
+                    (packed_capacity + PACK_BLOCK - 1) / PACK_BLOCK;
+  const int units = c.batch * c.n_kv_heads;
+  const int cap = MAX_GRID / units > 1 ? MAX_GRID / units : 1;
+  return items < cap ? (items > 1 ? items : 1) : cap;
 }
 
 void make_layout(const wushkv_config& c, wushkv_layout* L) {
@@ -106,7 +113,7 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
   const int G = c.n_q_heads / c.n_kv_heads;
   if (c.bits == 3) { L->n_planes = 2; L->plane_bits[0] = 2; L->plane_bits[1] = 1; }
   else { L->n_planes = 1; L->plane_bits[0] = c.bits; }
-  L->packed_capacity = (int)align_up((size_t)c.max_ctx, 32);
+  L->packed_capacity = (int)align_up((size_t)c.max_ctx, 128);
   size_t off = 0;
   for (int p = 0; p < L->n_planes; ++p) {
     L->plane_unit_stride[p] = (size_t)L->packed_capacity * 16 * L->plane_bits[p];
@@ -175,6 +182,61 @@ DevCache dev_view(const wushkv_cache* h) {
 wushkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? WUSHKV_OK : WUSHKV_ECUDA; }
 
 bool valid_dtype(int32_t d) { return d == WUSHKV_F16 || d == WUSHKV_BF16 || d == WUSHKV_F32; }
+
+// Fill the decode arguments of the cache's current state: window/packed
+// counts and the split plan.  Returns false if the cache is empty.
+int device_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
+bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale, DecodeArgs* a) {
+  const wushkv_config& c = h->cfg;
+  std::memset(a, 0, sizeof(*a));
+  a->c = dev_view(h);
+  a->q = q;
+  a->out = out;
+  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
+  a->scale_log2 = sc * 1.4426950408889634f;
+  const int64_t n = h->n;
+  if (n == 0) return false;
+  a->n_sink = (int)(n < c.sink ? n : c.sink);
+  a->n_packed = (int)packed_count(n, c);
+  a->n_recent = (int)(n - a->n_sink - a->n_packed);
+  a->ring_first = (int)(a->n_packed % (c.recent + c.chunk));
+  a->win_groups = (a->n_sink + a->n_recent + WIN_GROUP - 1) / WIN_GROUP;
+  a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
+  a->cost_w = (int64_t)WIN_GROUP * 2 * 128 * 2;
+  a->cost_p = (int64_t)PACK_BLOCK * 2 * (16 * c.bits + (int)h->lay.meta_bytes);
+  const int64_t bytes = a->win_groups * a->cost_w + a->pack_blocks * a->cost_p;
+  const int units = a->c.units;
+  static int occ[5][9][2] = {};
+  int& o = occ[c.bits][a->c.group][c.quantizer];
+  if (!o) {
+    o = decode_ctas_per_sm(c.bits, a->c.group, c.quantizer);
+    if (o <= 0) o = 1;
+  }
+  const int64_t wave = (int64_t)device_sms() * o;
+  int64_t s = wave / units;
+  const int64_t items = a->win_groups + a->pack_blocks;
+  const int64_t by_size = (bytes + MIN_SPLIT_BYTES - 1) / MIN_SPLIT_BYTES;
+  if (s > items) s = items;
+  if (s > by_size) s = by_size;
+  if (s > a->c.max_splits) s = a->c.max_splits;
+  if (s < 1) s = 1;
+  a->splits = (int)s;
+  a->partials = a->c.partials;
+  a->counters = a->c.counters;
+  return true;
+}
 
 }  // namespace
 
@@ -326,29 +388,9 @@ wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const f
 wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream) {
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
-  if (cache->n == 0) return WUSHKV_EINVAL;
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
-  const wushkv_config& c = cache->cfg;
   DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.c = dev_view(cache);
-  a.q = q_prime_dev;
-  a.out = out_dev;
-  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
-  a.scale_log2 = sc * 1.4426950408889634f;
-  const int64_t n = cache->n;
-  a.n_sink = (int)(n < c.sink ? n : c.sink);
-  a.n_packed = (int)packed_count(n, c);
-  a.n_recent = (int)(n - a.n_sink - a.n_packed);
-  a.ring_first = (int)(a.n_packed % (c.recent + c.chunk));
-  const int win = a.n_sink + a.n_recent;
-  a.win_tokens_per_split = WIN_TOKENS_PER_SPLIT;
-  a.win_splits = (win + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
-  a.pack_tokens_per_split = PACK_TOKENS_PER_SPLIT;
-  a.pack_splits = (a.n_packed + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
-  if (a.win_splits + a.pack_splits > a.c.max_splits) return WUSHKV_EINVAL;
-  a.partials = a.c.partials;
-  a.counters = a.c.counters;
+  if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
   return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -485,26 +527,9 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return WUSHKV_ECUDA;
     g_noalloc_addr[dev] = p;
   }
-  const wushkv_config& c = cache->cfg;
   DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.c = dev_view(cache);
-  a.q = q_prime_dev;
-  a.out = out_dev;
-  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
-  a.scale_log2 = sc * 1.4426950408889634f;
-  const int64_t n = cache->n;
-  a.n_sink = (int)(n < c.sink ? n : c.sink);
-  a.n_packed = (int)packed_count(n, c);
-  a.n_recent = (int)(n - a.n_sink - a.n_packed);
-  a.ring_first = (int)(a.n_packed % (c.recent + c.chunk));
-  const int win = a.n_sink + a.n_recent;
-  a.win_tokens_per_split = WIN_TOKENS_PER_SPLIT;
-  a.win_splits = (win + WIN_TOKENS_PER_SPLIT - 1) / WIN_TOKENS_PER_SPLIT;
-  a.pack_tokens_per_split = PACK_TOKENS_PER_SPLIT;
-  a.pack_splits = (a.n_packed + PACK_TOKENS_PER_SPLIT - 1) / PACK_TOKENS_PER_SPLIT;
-  const int total = a.win_splits + a.pack_splits;
-  if (total > a.c.max_splits) return WUSHKV_EINVAL;
+  if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
+  const int total = a.splits;
   // The partials of this call are packed densely: stride = this call's splits.
   a.c.max_splits = total;
   const size_t units = (size_t)a.c.units;

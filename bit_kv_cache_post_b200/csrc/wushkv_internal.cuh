@@ -223,13 +223,14 @@ struct DecodeArgs {
   float scale_log2;        // scale * log2(e)
   int n_sink, n_packed, n_recent;
   int ring_first;          // ring slot of the oldest recent token
-  int win_splits;          // CTAs per unit for sink + recent tokens
-  int win_tokens_per_split;
-  int pack_splits;         // CTAs per unit for packed tokens
-  int pack_tokens_per_split;
-  float* partials;         // workspace for split partials
-  int* counters;
+  int splits;              // CTAs per unit
+  int win_groups;          // ceil((n_sink + n_recent) / 32)
+  int pack_blocks;         // ceil(n_packed / 64)
+  int64_t cost_w, cost_p;  // bytes of one window group / one packed block
+  float* partials;         // split partials [unit][max_splits][G][130]
+  int* counters;           // arrival counter per unit
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+int decode_ctas_per_sm(int bits, int group, int quantizer);
 
 }  // namespace wushkv

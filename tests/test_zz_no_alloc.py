@@ -60,12 +60,16 @@ def test_noalloc_matches_decode_two_calls(wk):
 
 
 def test_noalloc_rejects_oversize_scratch(wk):
-    """128 units x G 8 x ~35 splits of partials exceed the fixed array."""
+    """2048 units x G 8 need at least one split each: 2048 x 8 x 520 B of
+    partials exceed the fixed array, so the call is refused, not run."""
     import torch
     lib = wk.load()
-    cache = _filled_cache(wk, 16, 8, 8, 16384, 2)
-    q = torch.zeros((16, 64, 128), dtype=torch.float32, device="cuda")
+    cache = _filled_cache(wk, 256, 8, 8, 16, 2)
+    q = torch.zeros((256, 64, 128), dtype=torch.float32, device="cuda")
     out = torch.zeros_like(q)
     st = lib.wushkv_decode_noalloc(q.data_ptr(), cache.handle, out.data_ptr(), ctypes.c_float(0.0),
                                    None)
     assert st == wk.ECAPACITY
+    cache.decode(q, out=out)            # the regular entry point serves it
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
