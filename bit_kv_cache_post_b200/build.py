@@ -23,6 +23,7 @@ FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC,-fvisibility=hidden",
+    "-diag-suppress", "177",
     "-shared",
 ]
 

@@ -22,14 +22,15 @@ namespace {
 
 using namespace wushkv;
 
-// Decode split policy: each unit is cut into `splits` CTAs of equal bytes
-// (window groups of 32 fp16 tokens, packed blocks of 64 tokens) so that the
-// grid fills one wave of resident CTAs; no split is smaller than
-// MIN_SPLIT_BYTES.  The workspace holds up to max(1, MAX_GRID / units)
-// splits per unit.
+// Decode work split: the units' bytes (window groups of 32 fp16 tokens,
+// packed blocks of 64 tokens) are shared equally among the CTAs of one wave
+// (stream-K); a CTA gets at least MIN_CTA_BYTES.  A unit is touched by at
+// most ceil(grid / units) + 1 CTAs, each writing one partial, so the
+// workspace holds max(3, MAX_GRID / units + 2) partials per unit and the
+// grid never exceeds (max_splits - 1) * units.
 constexpr int WIN_GROUP = 32;
 constexpr int PACK_BLOCK = 64;
-constexpr int64_t MIN_SPLIT_BYTES = 32 * 1024;
+constexpr int64_t MIN_CTA_BYTES = 32 * 1024;
 constexpr int MAX_GRID = 2048;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -100,11 +101,10 @@ wushkv_status check_config(const wushkv_config* c) {
 }
 
 int max_splits_for(const wushkv_config& c, int packed_capacity) {
-  const int items = (c.sink + c.recent + c.chunk + WIN_GROUP - 1) / WIN_GROUP +
-                    (packed_capacity + PACK_BLOCK - 1) / PACK_BLOCK;
+  (void)packed_capacity;
   const int units = c.batch * c.n_kv_heads;
-  const int cap = MAX_GRID / units > 1 ? MAX_GRID / units : 1;
-  return items < cap ? (items > 1 ? items : 1) : cap;
+  const int ms = MAX_GRID / units + 2;
+  return ms > 3 ? ms : 3;
 }
 
 void make_layout(const wushkv_config& c, wushkv_layout* L) {
@@ -216,23 +216,20 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
   a->cost_w = (int64_t)WIN_GROUP * 2 * 128 * 2;
   a->cost_p = (int64_t)PACK_BLOCK * 2 * (16 * c.bits + (int)h->lay.meta_bytes);
-  const int64_t bytes = a->win_groups * a->cost_w + a->pack_blocks * a->cost_p;
-  const int units = a->c.units;
+  const int64_t unit_bytes = a->win_groups * a->cost_w + a->pack_blocks * a->cost_p;
+  const int64_t units = a->c.units;
   static int occ[5][9][2] = {};
   int& o = occ[c.bits][a->c.group][c.quantizer];
   if (!o) {
     o = decode_ctas_per_sm(c.bits, a->c.group, c.quantizer);
     if (o <= 0) o = 1;
   }
-  const int64_t wave = (int64_t)device_sms() * o;
-  int64_t s = wave / units;
-  const int64_t items = a->win_groups + a->pack_blocks;
-  const int64_t by_size = (bytes + MIN_SPLIT_BYTES - 1) / MIN_SPLIT_BYTES;
-  if (s > items) s = items;
-  if (s > by_size) s = by_size;
-  if (s > a->c.max_splits) s = a->c.max_splits;
-  if (s < 1) s = 1;
-  a->splits = (int)s;
+  int64_t grid = (int64_t)device_sms() * o;
+  const int64_t by_size = units * unit_bytes / MIN_CTA_BYTES;
+  if (grid > by_size) grid = by_size;
+  if (grid > (int64_t)(a->c.max_splits - 1) * units) grid = (int64_t)(a->c.max_splits - 1) * units;
+  if (grid < 1) grid = 1;
+  a->grid = (int)grid;
   a->partials = a->c.partials;
   a->counters = a->c.counters;
   return true;
@@ -454,7 +451,8 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
           } else {
             const int mt = d / 16, rem = d % 16, rh = rem / 8, r = rem % 8;
             const int rho = 2 * mt + rh, beta = (int)(pk % 4);
-            wd = planes[p][(size_t)(pk / 4) * 16 * w + r * 2 * w + rho / F];
+            const int quad = (int)(pk / 4);
+            wd = planes[p][(size_t)quad * 16 * w + v_word_index(quad, r, rho / F, w)];
             bit = 8 * beta + w * (rho % F);
           }
           code[d] |= (uint8_t)(((wd >> bit) & mask) << shift);
@@ -529,8 +527,9 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   }
   DecodeArgs a;
   if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
-  const int total = a.splits;
-  // The partials of this call are packed densely: stride = this call's splits.
+  // Partials are packed densely: a unit is touched by at most
+  // ceil(grid / units) + 1 CTAs of this call.
+  const int total = (a.grid + a.c.units - 1) / a.c.units + 1;
   a.c.max_splits = total;
   const size_t units = (size_t)a.c.units;
   const size_t partial_bytes = units * (size_t)total * a.c.group * (128 + 2) * sizeof(float);

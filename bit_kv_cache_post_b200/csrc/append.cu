@@ -159,15 +159,17 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
             reinterpret_cast<uint32_t*>(base + (size_t)(pk + warp) * 16 * w)[lane] = word;
           }
         } else {
-          // one V quad, 16w words
+          // one V quad, 16w words: thread tid builds unit word (r, j)
           if (tid < 16 * w) {
+            const int r = tid / (2 * w), j = tid % (2 * w);
             uint32_t word = 0;
             for (int s = 0; s < P; ++s) {
               const int dim = v_field_dim(tid, w, s);
               for (int beta = 0; beta < 4; ++beta)
                 word |= plane_value(codes[beta * D + dim], c.bits, p) << (8 * beta + w * s);
             }
-            reinterpret_cast<uint32_t*>(base + (size_t)(pk / 4) * 64 * w)[tid] = word;
+            const int quad = (int)(pk / 4);
+            reinterpret_cast<uint32_t*>(base + (size_t)quad * 64 * w)[v_word_index(quad, r, j, w)] = word;
           }
         }
       }

@@ -42,7 +42,7 @@ struct DevCache {
 };
 
 // Status bits a kernel may set in the sticky word.
-enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2 };
+enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2, DEV_ERR_TIMEOUT = 4 };
 
 // ---------------------------------------------------------------------------
 // Exact-rounding helpers
@@ -188,6 +188,15 @@ __device__ __forceinline__ int v_field_dim(int wi, int w, int s) {
   return 16 * mt + r + 8 * rh;
 }
 
+// Flat word index in a V quad of unit word j of row unit r (plane width w):
+// the 2w words of row r sit at unit position (r + 2 (quad mod 4)) mod 8; a
+// 4-bit unit is split into two 16-byte halves 128 bytes apart.
+__host__ __device__ __forceinline__ int v_word_index(int quad, int r, int j, int w) {
+  const int pos = (r + 2 * (quad & 3)) & 7;
+  if (w == 4) return j < 4 ? 4 * pos + j : 32 + 4 * pos + (j - 4);
+  return 2 * w * pos + j;
+}
+
 // Value of plane p (width w) of a code: 3-bit codes split into a 2-bit low
 // plane and a 1-bit high plane.
 __device__ __forceinline__ uint32_t plane_value(uint32_t code, int bits, int p) {
@@ -223,7 +232,7 @@ struct DecodeArgs {
   float scale_log2;        // scale * log2(e)
   int n_sink, n_packed, n_recent;
   int ring_first;          // ring slot of the oldest recent token
-  int splits;              // CTAs per unit
+  int grid;                // CTAs (stream-K shares of the units' bytes)
   int win_groups;          // ceil((n_sink + n_recent) / 32)
   int pack_blocks;         // ceil(n_packed / 64)
   int64_t cost_w, cost_p;  // bytes of one window group / one packed block

@@ -100,8 +100,12 @@ typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
  *     ks in 0..3, beta in 0..3, rho = 4h + ks: word c*w + rho/(8/w), field
  *     rho % (8/w), dim 32ks + 4c + 16h + beta.
  *   V (4-token quads, 64*w bytes per quad per plane): r in 0..7, rho in
- *     0..15 (mt = rho/2, rh = rho%2), beta in 0..3: word r*2w + rho/(8/w),
- *     field rho % (8/w), dim 16mt + r + 8rh, token 4*quad + beta.
+ *     0..15 (mt = rho/2, rh = rho%2), beta in 0..3: unit word j = rho/(8/w),
+ *     field rho % (8/w), dim 16mt + r + 8rh, token 4*quad + beta.  Row unit
+ *     r sits at position pos = (r + 2*(quad mod 4)) mod 8 of its quad: word
+ *     2w*pos + j for w <= 2; for w = 4 word 4pos + j (j < 4) or
+ *     32 + 4pos + j - 4 (j >= 4).  (This spreads a warp's reads of a quad
+ *     over all shared-memory banks.)
  *   meta: per token, fp16 delta (QuEST, 2 bytes) or fp16 (scale, lo) pair
  *     (affine, 4 bytes); K and V separately.
  *   sink, ring: fp16 [unit][slot][128]; ring slot of post-sink token t is

@@ -329,8 +329,12 @@ def affine_dequantize(codes: np.ndarray, s_h: np.ndarray, lo_h: np.ndarray) -> n
 #       word = c*w + rho // P, field s = rho % P, dim = 32ks + 4c + 16h + beta.
 #   V quads (4 consecutive tokens, 8*2w words per plane): for r in 0..7,
 #     rho in 0..15 (mt = rho // 2, rh = rho % 2), beta in 0..3:
-#       word index = r*2w + rho // P, field s = rho % P,
+#       unit word j = rho // P, field s = rho % P,
 #       dim = 16mt + r + 8rh, token = 4*quad + beta.
+#     The 2w words of row unit r are stored at unit position
+#     pos = (r + 2*(quad mod 4)) mod 8 of the quad: w = 1 -> words 2pos + j;
+#     w = 2 -> words 4pos + j; w = 4 -> words 4pos + j for j < 4 and
+#     32 + 4pos + (j - 4) for j >= 4.  (quad = quad index within the unit.)
 # ---------------------------------------------------------------------------
 
 def plane_widths(bits: int) -> list[int]:
@@ -382,40 +386,58 @@ def unpack_k_rows(planes: list[np.ndarray], bits: int) -> np.ndarray:
     return codes.astype(np.uint8)
 
 
+def v_word_index(quad: int, r: int, j: int, w: int) -> int:
+    """Flat word index in a V quad of unit word j of row unit r."""
+    pos = (r + 2 * (quad % 4)) % 8
+    if w == 4:
+        return 4 * pos + j if j < 4 else 32 + 4 * pos + (j - 4)
+    return 2 * w * pos + j
+
+
 def pack_v_quads(codes: np.ndarray, bits: int) -> list[np.ndarray]:
-    """codes [NQ, 4, 128] (4 consecutive tokens per quad) -> one uint32
-    array [NQ, 8 * 2w] per plane."""
+    """codes [NQ, 4, 128] (4 consecutive tokens per quad; quad index = first
+    axis) -> one uint32 array [NQ, 16w] per plane."""
     out = []
+    nq = codes.shape[0]
     for w, vals in zip(plane_widths(bits), _plane_values(codes, bits)):
         P = 8 // w
-        words = np.zeros(codes.shape[:-2] + (8, 2 * w), dtype=np.uint32)
+        unit = np.zeros((nq, 8, 2 * w), dtype=np.uint32)
         for r in range(8):
             for rho in range(16):
                 mt, rh = rho // 2, rho % 2
                 dim = 16 * mt + r + 8 * rh
                 word, s = rho // P, rho % P
                 for beta in range(4):
-                    words[..., r, word] |= vals[..., beta, dim] << np.uint32(8 * beta + w * s)
-        out.append(words.reshape(codes.shape[:-2] + (16 * w,)))
+                    unit[:, r, word] |= vals[:, beta, dim] << np.uint32(8 * beta + w * s)
+        words = np.zeros((nq, 16 * w), dtype=np.uint32)
+        for q in range(nq):
+            for r in range(8):
+                for j in range(2 * w):
+                    words[q, v_word_index(q, r, j, w)] = unit[q, r, j]
+        out.append(words)
     return out
 
 
 def unpack_v_quads(planes: list[np.ndarray], bits: int) -> np.ndarray:
     """Inverse of :func:`pack_v_quads`: -> codes [NQ, 4, 128]."""
-    nq = planes[0].shape[:-1]
-    codes = np.zeros(nq + (4, HEAD_DIM), dtype=np.uint32)
+    nq = planes[0].shape[0]
+    codes = np.zeros((nq, 4, HEAD_DIM), dtype=np.uint32)
     shift = 0
     for w, flat in zip(plane_widths(bits), planes):
         P, mask = 8 // w, np.uint32((1 << w) - 1)
-        words = flat.reshape(nq + (8, 2 * w))
+        words = np.zeros((nq, 8, 2 * w), dtype=np.uint32)
+        for q in range(nq):
+            for r in range(8):
+                for j in range(2 * w):
+                    words[q, r, j] = flat[q, v_word_index(q, r, j, w)]
         for r in range(8):
             for rho in range(16):
                 mt, rh = rho // 2, rho % 2
                 dim = 16 * mt + r + 8 * rh
                 word, s = rho // P, rho % P
                 for beta in range(4):
-                    f = (words[..., r, word] >> np.uint32(8 * beta + w * s)) & mask
-                    codes[..., beta, dim] |= f << np.uint32(shift)
+                    f = (words[:, r, word] >> np.uint32(8 * beta + w * s)) & mask
+                    codes[:, beta, dim] |= f << np.uint32(shift)
         shift += w
     return codes.astype(np.uint8)
 

@@ -122,8 +122,8 @@ def test_pack_positions_golden():
             c[0, dim] = code
             planes = O.pack_k_rows(c, bits)
         else:
-            c = np.zeros((1, 4, 128), np.uint8)
-            c[0, tok, dim] = code
+            c = np.zeros((tok // 4 + 1, 4, 128), np.uint8)
+            c[tok // 4, tok % 4, dim] = code
             planes = O.pack_v_quads(c, bits)
         words = planes[plane].reshape(-1)
         nz = np.flatnonzero(words)
