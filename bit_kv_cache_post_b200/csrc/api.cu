@@ -31,6 +31,10 @@ using namespace wushkv;
 constexpr int WIN_GROUP = 32;
 constexpr int PACK_BLOCK = 64;
 constexpr int64_t MIN_CTA_BYTES = 32 * 1024;
+// Window tokens (plain fp16 rows) take fewer instructions per byte than
+// packed tokens; the split weighs their bytes by 1 / WINDOW_COST_DIVISOR so
+// that CTAs and warps receive equal time rather than equal bytes.
+constexpr int64_t WINDOW_COST_DIVISOR = 3;
 constexpr int MAX_GRID = 2048;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -214,7 +218,7 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   a->ring_first = (int)(a->n_packed % (c.recent + c.chunk));
   a->win_groups = (a->n_sink + a->n_recent + WIN_GROUP - 1) / WIN_GROUP;
   a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
-  a->cost_w = (int64_t)WIN_GROUP * 2 * 128 * 2;
+  a->cost_w = (int64_t)WIN_GROUP * 2 * 128 * 2 / WINDOW_COST_DIVISOR;
   a->cost_p = (int64_t)PACK_BLOCK * 2 * (16 * c.bits + (int)h->lay.meta_bytes);
   const int64_t unit_bytes = a->win_groups * a->cost_w + a->pack_blocks * a->cost_p;
   const int64_t units = a->c.units;

@@ -35,6 +35,7 @@ constexpr int WGRP = 32;        // window tokens per group
 constexpr int PS_LD = PB + 16;  // bytes per row of the per-warp P tile
 constexpr int NSTAGE = 2;       // per-warp copy stages
 constexpr uint32_t WAIT_POLLS = 1u << 22;
+constexpr unsigned FULL_MASK = 0xffffffffu;
 
 // Bytes of one packed block in a stage: K planes, V planes, K meta, V meta.
 template <int BITS>
@@ -255,26 +256,24 @@ struct PackedState {
 // Lane = 4r + c.  Score m-tile rows r, r+8 are tokens; columns are (head,
 // term) pairs, so thread c owns head 4nt + c of n-tile nt.  PV m-tile rows
 // are dims 16mt + r (+8); the PV B operand comes back through the warp's P
-// tile in shared memory.
-template <int BITS, int G, bool AFFINE>
-__device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, const unsigned char* st,
-                                     int blk, int warp, int lane, const uint32_t (&qb)[(G + 3) / 4][4][2],
-                                     const float (&qscale)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4],
-                                     PackedState<(G + 3) / 4>& S) {
+// tile in shared memory.  FULL: all 64 tokens of the block are cached.
+template <int BITS, int G, bool AFFINE, bool FULL>
+__device__ __forceinline__ void packed_block_compute(
+    const DecodeArgs& a, Smem<BITS, G>& sh, const unsigned char* st, int blk, int warp, int lane,
+    const uint32_t (&qb)[(G + 3) / 4][4][2], const float (&qscale)[(G + 3) / 4],
+    const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], PackedState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   using SL = StageLayout<BITS>;
-  constexpr int MB = AFFINE ? 4 : 2;
   const int r = lane >> 2, c4 = lane & 3;
-  const float beta = 0.5f - (float)(1 << (BITS - 1));
-  const int tb = blk * PB;
+  const int nvalid = a.n_packed - blk * PB;  // used when !FULL
 
   // ---- scores ----------------------------------------------------------------
   float sc[4][2][NT];
   float vs[4][2], vo[4][2];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
-    KWords<BITS> kw0 = stage_k_words<BITS>(st, 16 * mt + r, c4);
-    KWords<BITS> kw1 = stage_k_words<BITS>(st, 16 * mt + r + 8, c4);
+    const KWords<BITS> kw0 = stage_k_words<BITS>(st, 16 * mt + r, c4);
+    const KWords<BITS> kw1 = stage_k_words<BITS>(st, 16 * mt + r + 8, c4);
     int acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
@@ -288,22 +287,30 @@ __device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, con
 #pragma unroll
     for (int th = 0; th < 2; ++th) {
       const int t = 16 * mt + r + 8 * th;
-      const bool valid = tb + t < a.n_packed;
-      const float2 km = load_meta<AFFINE>(st + SL::K_META, t, beta);
-      const float2 vm = load_meta<AFFINE>(st + SL::V_META, t, beta);
-      vs[mt][th] = vm.x;
-      vo[mt][th] = vm.y;
+      float ks_, ko_;
+      if constexpr (AFFINE) {
+        const float2 km = __half22float2(*reinterpret_cast<const __half2*>(st + SL::K_META + 4 * t));
+        const float2 vm = __half22float2(*reinterpret_cast<const __half2*>(st + SL::V_META + 4 * t));
+        ks_ = km.x; ko_ = km.y; vs[mt][th] = vm.x; vo[mt][th] = vm.y;
+      } else {
+        ks_ = __half2float(*reinterpret_cast<const __half*>(st + SL::K_META + 2 * t));
+        ko_ = 0.f;
+        vs[mt][th] = __half2float(*reinterpret_cast<const __half*>(st + SL::V_META + 2 * t));
+        vo[mt][th] = 0.f;
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const float dot = qscale[nt] * (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
-        const float s = fmaf(km.x, dot, km.y * qsum[nt]);
-        sc[mt][th][nt] = valid ? s : -INFINITY;
+        const float xf = (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
+        float s;
+        if constexpr (AFFINE) s = fmaf(ks_, qscale[nt] * xf, ko_ * qsum[nt]);
+        else s = ks_ * fmaf(qscale[nt], xf, qoff[nt]);   // delta * (q.c + beta sum q)
+        if constexpr (!FULL) s = (t < nvalid) ? s : -INFINITY;
+        sc[mt][th][nt] = s;
       }
     }
   }
-  (void)MB;
 
-  // ---- online softmax, P terms -------------------------------------------------
+  // ---- online softmax; P as 16-bit fixed point in two byte terms ---------------
   uint8_t* ps = &sh.ps[warp][0][0];
   float al[NT], sp[NT];
 #pragma unroll
@@ -311,9 +318,9 @@ __device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, con
     float bm = -INFINITY;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) bm = fmaxf(bm, fmaxf(sc[mt][0][nt], sc[mt][1][nt]));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, 4));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, 8));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, 16));
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
     const float mn = fmaxf(S.m[nt], bm);
     al[nt] = exp2f(S.m[nt] - mn);
     S.m[nt] = mn;
@@ -322,32 +329,33 @@ __device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, con
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        const bool valid = sc[mt][th][nt] != -INFINITY;
-        const float p = valid ? exp2f(sc[mt][th][nt] - mn) : 0.f;
-        const float pt = p * vs[mt][th];
+        const float p = exp2f(sc[mt][th][nt] - mn);   // masked tokens: exp2(-inf) = 0
+        float pt = p * vs[mt][th];
+        if constexpr (!FULL) pt = (16 * mt + r + 8 * th < nvalid) ? pt : 0.f;
         ls += p;
-        es = fmaf(p, vo[mt][th], es);
+        if constexpr (AFFINE) es = fmaf(p, vo[mt][th], es);
+        else es += pt;                                 // times beta at the end
         pm = fmaxf(pm, pt);
         sc[mt][th][nt] = pt;
       }
-    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 4));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 8));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 16));
+    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 4));
+    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 8));
+    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 16));
     sp[nt] = pm;
     S.l[nt] = fmaf(S.l[nt], al[nt], ls);
     S.e[nt] = fmaf(S.e[nt], al[nt], es);
-    const float inv = pm > 0.f ? 255.f / pm : 0.f;
+    const float inv = pm > 0.f ? 65535.f / pm : 0.f;
+    const int col = nt * 8 + 2 * c4;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        const float uu = fminf(sc[mt][th][nt] * inv, 255.f);
-        const float q0 = floorf(uu);
-        const float q1 = fminf(rintf((uu - q0) * 255.f), 255.f);
-        const int col = nt * 8 + 2 * c4;
+        // 1.5 * 2^23 + rint(pt * 65535 / pm): the low 16 mantissa bits are the
+        // rounded value; its high byte is term 0, its low byte term 1.
+        const uint32_t bits = __float_as_uint(fmaf(sc[mt][th][nt], inv, 12582912.f));
         const int t = 16 * mt + r + 8 * th;
-        ps[col * PS_LD + t] = (uint8_t)q0;
-        ps[(col + 1) * PS_LD + t] = (uint8_t)q1;
+        ps[col * PS_LD + t] = (uint8_t)(bits >> 8);
+        ps[(col + 1) * PS_LD + t] = (uint8_t)bits;
       }
   }
   __syncwarp();
@@ -372,8 +380,14 @@ __device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, con
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const uint32_t a0 = v_frag<BITS>(v0, 2 * mt), a1 = v_frag<BITS>(v0, 2 * mt + 1);
-      const uint32_t a2 = v_frag<BITS>(v1, 2 * mt), a3 = v_frag<BITS>(v1, 2 * mt + 1);
+      uint32_t a0, a1, a2, a3;
+      if constexpr (BITS == 3) {
+        a0 = v_frag<BITS>(v0, 2 * mt); a1 = v_frag<BITS>(v0, 2 * mt + 1);
+        a2 = v_frag<BITS>(v1, 2 * mt); a3 = v_frag<BITS>(v1, 2 * mt + 1);
+      } else {
+        a0 = v_frag_scaled<BITS>(v0, 2 * mt); a1 = v_frag_scaled<BITS>(v0, 2 * mt + 1);
+        a2 = v_frag_scaled<BITS>(v1, 2 * mt); a3 = v_frag_scaled<BITS>(v1, 2 * mt + 1);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_u8u8(pacc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }
@@ -381,11 +395,11 @@ __device__ void packed_block_compute(const DecodeArgs& a, Smem<BITS, G>& sh, con
   __syncwarp();
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float f = sp[nt] * (1.f / 65025.f);
+    const float f = sp[nt] * (1.f / 65535.f);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      S.o[nt][mt][0] = fmaf(S.o[nt][mt][0], al[nt], f * (float)(pacc[mt][nt][0] * 255 + pacc[mt][nt][1]));
-      S.o[nt][mt][1] = fmaf(S.o[nt][mt][1], al[nt], f * (float)(pacc[mt][nt][2] * 255 + pacc[mt][nt][3]));
+      S.o[nt][mt][0] = fmaf(S.o[nt][mt][0], al[nt], f * (float)(pacc[mt][nt][0] * 256 + pacc[mt][nt][1]));
+      S.o[nt][mt][1] = fmaf(S.o[nt][mt][1], al[nt], f * (float)(pacc[mt][nt][2] * 256 + pacc[mt][nt][3]));
     }
   }
 }
@@ -399,7 +413,8 @@ __device__ void packed_blocks(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
   uint32_t qb[NT][4][2];
-  float qscale[NT], qsum[NT];
+  float qscale[NT], qsum[NT], qoff[NT];
+  const float beta = 0.5f - (float)(1 << (BITS - 1));
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int gcol = nt * 4 + (r >> 1), term = r & 1;
@@ -410,6 +425,7 @@ __device__ void packed_blocks(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int
         qb[nt][ks][h] = *reinterpret_cast<const uint32_t*>(&sh.qterm[gcol][term][32 * ks + 16 * h + 4 * c4]);
     qscale[nt] = sh.qscale[nt * 4 + c4];
     qsum[nt] = sh.qsum[nt * 4 + c4];
+    qoff[nt] = beta * qsum[nt];
     S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) S.o[nt][mt][0] = S.o[nt][mt][1] = 0.f;
@@ -435,8 +451,12 @@ __device__ void packed_blocks(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int
       for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
       return;
     }
-    packed_block_compute<BITS, G, AFFINE>(a, sh, sh.stage[warp][stg], pb0 + i, warp, lane, qb, qscale,
-                                          qsum, S);
+    if ((pb0 + i + 1) * PB <= a.n_packed)
+      packed_block_compute<BITS, G, AFFINE, true>(a, sh, sh.stage[warp][stg], pb0 + i, warp, lane, qb,
+                                                  qscale, qoff, qsum, S);
+    else
+      packed_block_compute<BITS, G, AFFINE, false>(a, sh, sh.stage[warp][stg], pb0 + i, warp, lane, qb,
+                                                   qscale, qoff, qsum, S);
     __syncwarp();
     if (lane == 0 && i + NSTAGE < nblk) {
       fence_proxy_async();
@@ -521,13 +541,16 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
         lt += __shfl_xor_sync(FULL, lt, o);
         et += __shfl_xor_sync(FULL, et, o);
       }
+      if constexpr (!AFFINE) et *= 0.5f - (float)(1 << (BITS - 1));  // sum p*delta*beta
       const int g = nt * 4 + c4;
       if (g < G) {
         if (r == 0) { sh.sm[NW + warp][g] = S.m[nt]; sh.sl[NW + warp][g] = lt; }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          so_p[warp][g][16 * mt + r] = S.o[nt][mt][0] + et;
-          so_p[warp][g][16 * mt + r + 8] = S.o[nt][mt][1] + et;
+          const float s0 = BITS == 3 ? 1.f : v_row_scale<BITS == 3 ? 2 : BITS>(2 * mt);
+          const float s1 = BITS == 3 ? 1.f : v_row_scale<BITS == 3 ? 2 : BITS>(2 * mt + 1);
+          so_p[warp][g][16 * mt + r] = fmaf(S.o[nt][mt][0], s0, et);
+          so_p[warp][g][16 * mt + r + 8] = fmaf(S.o[nt][mt][1], s1, et);
         }
       }
     }

@@ -38,21 +38,6 @@ template <> struct KWords<2> { uint2 lo; };
 template <> struct KWords<3> { uint2 lo; uint32_t hi; };
 template <> struct KWords<4> { uint4 w; };
 
-template <int BITS>
-__device__ __forceinline__ KWords<BITS> load_k_words(const uint8_t* p0, const uint8_t* p1, int tok,
-                                                     int c4) {
-  KWords<BITS> r;
-  if constexpr (BITS == 2) {
-    r.lo = __ldg(reinterpret_cast<const uint2*>(p0 + (size_t)tok * 32) + c4);
-  } else if constexpr (BITS == 3) {
-    r.lo = __ldg(reinterpret_cast<const uint2*>(p0 + (size_t)tok * 32) + c4);
-    r.hi = __ldg(reinterpret_cast<const uint32_t*>(p1 + (size_t)tok * 16) + c4);
-  } else {
-    r.w = __ldg(reinterpret_cast<const uint4*>(p0 + (size_t)tok * 64) + c4);
-  }
-  return r;
-}
-
 // A fragment register of k-step ks, half h (k columns 16h + 4c .. +3).
 template <int BITS>
 __device__ __forceinline__ uint32_t k_frag(const KWords<BITS>& w, int ks, int h) {
@@ -75,23 +60,6 @@ template <> struct VWords<2> { uint4 lo; };
 template <> struct VWords<3> { uint4 lo; uint2 hi; };
 template <> struct VWords<4> { uint4 a, b; };
 
-template <int BITS>
-__device__ __forceinline__ VWords<BITS> load_v_words(const uint8_t* p0, const uint8_t* p1, int quad,
-                                                     int r) {
-  VWords<BITS> v;
-  if constexpr (BITS == 2) {
-    v.lo = __ldg(reinterpret_cast<const uint4*>(p0 + (size_t)quad * 128) + r);
-  } else if constexpr (BITS == 3) {
-    v.lo = __ldg(reinterpret_cast<const uint4*>(p0 + (size_t)quad * 128) + r);
-    v.hi = __ldg(reinterpret_cast<const uint2*>(p1 + (size_t)quad * 64) + r);
-  } else {
-    const uint4* q = reinterpret_cast<const uint4*>(p0 + (size_t)quad * 256) + 2 * r;
-    v.a = __ldg(q);
-    v.b = __ldg(q + 1);
-  }
-  return v;
-}
-
 __device__ __forceinline__ uint32_t pick4(const uint4& w, int j) {
   return j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
 }
@@ -109,6 +77,28 @@ __device__ __forceinline__ uint32_t v_frag(const VWords<BITS>& v, int rho) {
     const uint32_t word = (rho >> 1) < 4 ? pick4(v.a, rho >> 1) : pick4(v.b, (rho >> 1) - 4);
     return (word >> (4 * (rho & 1))) & 0x0F0F0F0Fu;
   }
+}
+
+// As v_frag, but masked in place (no shift): the codes come out multiplied
+// by 2^(w * field).  For 2- and 4-bit planes the field of a PV row is fixed
+// (rho = 2mt + rh), so every dim row carries one power-of-two factor that is
+// removed once from the final output (v_row_scale).
+template <int BITS>
+__device__ __forceinline__ uint32_t v_frag_scaled(const VWords<BITS>& v, int rho) {
+  static_assert(BITS == 2 || BITS == 4, "shift-free fragments need a single plane");
+  if constexpr (BITS == 2) {
+    return pick4(v.lo, rho >> 2) & (0x03030303u << (2 * (rho & 3)));
+  } else {
+    const uint32_t word = (rho >> 1) < 4 ? pick4(v.a, rho >> 1) : pick4(v.b, (rho >> 1) - 4);
+    return word & (0x0F0F0F0Fu << (4 * (rho & 1)));
+  }
+}
+
+// 1 / (factor of v_frag_scaled) for rho.
+template <int BITS>
+__device__ __forceinline__ float v_row_scale(int rho) {
+  if constexpr (BITS == 2) return 1.f / (float)(1 << (2 * (rho & 3)));
+  else return (rho & 1) ? 1.f / 16.f : 1.f;
 }
 
 // Per-token dequantisation parameters: value = scale * code + offset.
