@@ -320,6 +320,7 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
                             int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
                             int32_t quantizer, void* stream) {
   if (!cache || !k_rope_dev || !v_dev || !valid_dtype(in_dtype) || n_tok < 0) return WUSHKV_EINVAL;
+  if (reinterpret_cast<uintptr_t>(T_k_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   const wushkv_config& c = cache->cfg;
   if (bits != c.bits || quantizer != c.quantizer) return WUSHKV_EINVAL;
   if (n_tok == 0) return WUSHKV_OK;
@@ -379,6 +380,7 @@ wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const f
                                      float* q_out_dev, int32_t batch, int32_t n_q_heads,
                                      int32_t n_kv_heads, void* stream) {
   if (!q_dev || !T_k_invT_dev || !q_out_dev || !valid_dtype(q_dtype)) return WUSHKV_EINVAL;
+  if (reinterpret_cast<uintptr_t>(T_k_invT_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads) return WUSHKV_EINVAL;
   if (n_q_heads / n_kv_heads > 16) return WUSHKV_EUNSUPPORTED;
   if ((int64_t)batch * n_kv_heads > 2147483647LL) return WUSHKV_EUNSUPPORTED;

@@ -54,13 +54,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   // Stage T^T of this head once per CTA if any new key needs the product.
   const bool has_new = (4 * q_last > n0) && (4 * q_first < n1);
   const bool transform = (a.T != nullptr) && has_new;
-  if (transform) {
-    const float* T = a.T + (size_t)h * D * D;
-    for (int idx = tid; idx < D * D; idx += 128) {
-      const int i = idx >> 7, j = idx & 127;
-      Tt[j * TT_LD + i] = T[idx];
-    }
-  }
+  if (transform) stage_transpose_128(a.T + (size_t)h * D * D, Tt, TT_LD);
 
   const size_t plane_u0 = (size_t)u * c.plane_unit_stride[0];
   const size_t plane_u1 = (size_t)u * c.plane_unit_stride[1];

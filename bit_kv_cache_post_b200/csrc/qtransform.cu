@@ -26,8 +26,7 @@ __global__ void __launch_bounds__(128) qtransform_kernel(const void* q, int dtyp
   const int G = n_q_heads / n_kv_heads;
   const int b = blockIdx.x / n_kv_heads, h = blockIdx.x % n_kv_heads;
   const int tid = threadIdx.x;
-  const float* M = TinvT + (size_t)h * D * D;
-  for (int idx = tid; idx < D * D; idx += 128) Mt[(idx & 127) * MT_LD + (idx >> 7)] = M[idx];
+  stage_transpose_128(TinvT + (size_t)h * D * D, Mt, MT_LD);
   for (int g = 0; g < G; ++g)
     qs[g * D + tid] = load_q(q, dtype, ((size_t)b * n_q_heads + (size_t)h * G + g) * D + tid);
   __syncthreads();

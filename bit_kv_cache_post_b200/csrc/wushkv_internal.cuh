@@ -82,6 +82,28 @@ __device__ __forceinline__ float warp_sum_f32(float v) {
   return v;
 }
 
+// Stage the transpose of a row-major 128 x 128 fp32 matrix into shared
+// memory (row stride ld, padded against bank conflicts) with a 128-thread
+// block: 16-byte loads, eight in flight per thread.
+__device__ __forceinline__ void stage_transpose_128(const float* __restrict__ M, float* Mt, int ld) {
+  const float4* M4 = reinterpret_cast<const float4*>(M);
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __ldg(M4 + threadIdx.x + 128 * (8 * b + k));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = 4 * (threadIdx.x + 128 * (8 * b + k));   // element index
+      const int i = e >> 7, j = e & 127;
+      Mt[(j + 0) * ld + i] = v[k].x;
+      Mt[(j + 1) * ld + i] = v[k].y;
+      Mt[(j + 2) * ld + i] = v[k].z;
+      Mt[(j + 3) * ld + i] = v[k].w;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Per-token quantisers on one warp.  Lane l holds dims 4l..4l+3 of the token
 // as float values that are exactly fp16 values.

@@ -156,8 +156,9 @@ WUSHKV_API wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t*
  *   k_rope_dev: [batch][n_tok][n_kv_heads][128] post-RoPE keys, dtype in_dtype.
  *   v_dev:      [batch][n_tok][n_kv_heads][128] values (already in the
  *               transformed value space), dtype in_dtype.
- *   T_k_dev:    [n_kv_heads][128][128] fp32 row-major, k'_i = sum_j T[i][j] k_j;
- *               NULL means the keys are already transformed (no product).
+ *   T_k_dev:    [n_kv_heads][128][128] fp32 row-major, k'_i = sum_j T[i][j] k_j,
+ *               16-byte aligned (EINVAL otherwise); NULL means the keys are
+ *               already transformed (no product).
  *   bits, quantizer: must equal the cache's configuration (EINVAL otherwise).
  * Every key and value is rounded once to fp16; tokens landing in the sink or
  * recent window are stored as those fp16 values, tokens that the window
@@ -172,7 +173,8 @@ WUSHKV_API wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_d
  *   Source: same page, 方法关键点 and 工作参考价值 (one d x d product per
  *   query; inverse transpose keeps q'.k' = q.k).
  *   q_dev:        [batch][n_q_heads][128], dtype q_dtype.
- *   T_k_invT_dev: [n_kv_heads][128][128] fp32 row-major, q'_i = sum_j M[i][j] q_j.
+ *   T_k_invT_dev: [n_kv_heads][128][128] fp32 row-major, q'_i = sum_j M[i][j] q_j,
+ *                 16-byte aligned (EINVAL otherwise).
  *   q_out_dev:    [batch][n_q_heads][128] fp32 (kept fp32 for the decode). */
 WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
                                      float* q_out_dev, int32_t batch, int32_t n_q_heads,
