@@ -22,19 +22,16 @@ namespace {
 
 using namespace wushkv;
 
-// Decode work split: the units' bytes (window groups of 32 fp16 tokens,
-// packed blocks of 64 tokens) are shared equally among the CTAs of one wave
-// (stream-K); a CTA gets at least MIN_CTA_BYTES.  A unit is touched by at
-// most ceil(grid / units) + 1 CTAs, each writing one partial, so the
-// workspace holds max(3, MAX_GRID / units + 2) partials per unit and the
-// grid never exceeds (max_splits - 1) * units.
-constexpr int WIN_GROUP = 32;
+// Decode work split: each unit's cache is a sequence of items of about 4 KB
+// (window chunks of 8 fp16 tokens spread among packed blocks of 64 tokens);
+// the units' items are shared equally among the CTAs of one wave
+// (stream-K), at least MIN_CTA_ITEMS each.  A unit is touched by at most
+// ceil(grid / units) + 1 CTAs, each writing one partial, so the workspace
+// holds max(3, MAX_GRID / units + 2) partials per unit and the grid never
+// exceeds (max_splits - 1) * units.
+constexpr int WIN_CHUNK = 8;
 constexpr int PACK_BLOCK = 64;
-constexpr int64_t MIN_CTA_BYTES = 32 * 1024;
-// Window tokens (plain fp16 rows) take fewer instructions per byte than
-// packed tokens; the split weighs their bytes by 1 / WINDOW_COST_DIVISOR so
-// that CTAs and warps receive equal time rather than equal bytes.
-constexpr int64_t WINDOW_COST_DIVISOR = 3;
+constexpr int64_t MIN_CTA_ITEMS = 8;
 constexpr int MAX_GRID = 2048;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -216,12 +213,10 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   a->n_packed = (int)packed_count(n, c);
   a->n_recent = (int)(n - a->n_sink - a->n_packed);
   a->ring_first = (int)(a->n_packed % (c.recent + c.chunk));
-  a->win_groups = (a->n_sink + a->n_recent + WIN_GROUP - 1) / WIN_GROUP;
+  a->win_chunks = (a->n_sink + a->n_recent + WIN_CHUNK - 1) / WIN_CHUNK;
   a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
-  a->cost_w = (int64_t)WIN_GROUP * 2 * 128 * 2 / WINDOW_COST_DIVISOR;
-  a->cost_p = (int64_t)PACK_BLOCK * 2 * (16 * c.bits + (int)h->lay.meta_bytes);
-  const int64_t unit_bytes = a->win_groups * a->cost_w + a->pack_blocks * a->cost_p;
   const int64_t units = a->c.units;
+  const int64_t items = units * (a->win_chunks + a->pack_blocks);
   static int occ[5][9][2] = {};
   int& o = occ[c.bits][a->c.group][c.quantizer];
   if (!o) {
@@ -229,8 +224,7 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
     if (o <= 0) o = 1;
   }
   int64_t grid = (int64_t)device_sms() * o;
-  const int64_t by_size = units * unit_bytes / MIN_CTA_BYTES;
-  if (grid > by_size) grid = by_size;
+  if (grid > items / MIN_CTA_ITEMS) grid = items / MIN_CTA_ITEMS;
   if (grid > (int64_t)(a->c.max_splits - 1) * units) grid = (int64_t)(a->c.max_splits - 1) * units;
   if (grid < 1) grid = 1;
   a->grid = (int)grid;

@@ -9,19 +9,21 @@
 // with (scale, offset) = (delta, delta (1/2 - L/2)) for QuEST INT and
 // (s, lo) for the affine quantiser.
 //
-// Work split (stream-K over bytes): the units' work is laid end to end as
-// window groups (32 fp16 tokens) then packed blocks (64 tokens) per unit,
-// weighted by their bytes, and CTA i of the one-wave grid takes the i-th
-// equal share -- usually part of one unit, sometimes the end of one and the
-// start of the next.  Inside a CTA each unit segment is cut again into four
-// equal byte shares, one per warp.  Window tokens run one token per lane in
-// fp32.  Packed blocks stream through a per-warp ring of shared-memory stages
-// filled by bulk asynchronous copies (the TMA engine) and run on integer
-// tensor cores (mma.sync m16n8k32): codes (u8) x two int8 terms of the query
-// for the scores, codes (u8) x two u8 terms of p * scale for PV.  Each CTA
-// merges its warps per unit segment and writes one (m, l, o) partial; the
-// last CTA of a unit to finish merges that unit's partials (an arrival
-// counter; no CTA ever waits on another).
+// Work items: a unit's cache is a sequence of items -- packed blocks of 64
+// tokens and window chunks of 8 fp16 tokens, each about 4 KB -- with the
+// window chunks spread evenly among the packed blocks.  The units' items are
+// laid end to end and CTA i of the one-wave grid takes the i-th equal share
+// (stream-K): usually part of one unit, sometimes the end of one and the
+// start of the next.  Each unit segment of a CTA is cut into four equal item
+// ranges, one per warp.  A warp streams its items through a ring of
+// shared-memory stages filled by bulk asynchronous copies (the TMA engine)
+// and runs them on tensor cores with mma.sync: packed blocks on the integer
+// pipe (codes u8 x two int8 terms of the query for the scores; codes u8 x
+// two u8 terms of p * scale for PV), window chunks on the fp16 pipe (rows
+// exact, query and p as fp16 hi/lo pairs).  Both kinds update the same
+// online-softmax state.  Each CTA merges its warps per unit segment and
+// writes one (m, l, o) partial; the last CTA of a unit to finish merges that
+// unit's partials (an arrival counter; no CTA ever waits on another).
 #include "async_copy.cuh"
 #include "decode_frag.cuh"
 
@@ -29,11 +31,13 @@ namespace wushkv {
 
 namespace {
 
-constexpr int NW = 4;           // warps per CTA
-constexpr int PB = 64;          // packed tokens per block
-constexpr int WGRP = 32;        // window tokens per group
-constexpr int PS_LD = PB + 16;  // bytes per row of the per-warp P tile
-constexpr int NSTAGE = 2;       // per-warp copy stages
+constexpr int NW = 4;            // warps per CTA
+constexpr int PB = 64;           // packed tokens per block
+constexpr int WC = 8;            // window tokens per chunk
+constexpr int WROW = 256 + 16;   // bytes per window row in a stage (padded: ldmatrix bank spread)
+constexpr int WIN_V = WC * WROW; // offset of the V rows of a window chunk
+constexpr int PS_LD = PB + 16;   // bytes per row of the per-warp P tile
+constexpr int NSTAGE = 2;        // per-warp copy stages
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr unsigned FULL_MASK = 0xffffffffu;
 
@@ -45,7 +49,9 @@ struct StageLayout {
   static constexpr int HI = BITS == 3 ? PB * 16 : 0;      // plane-1 bytes
   static constexpr int K_LO = 0, K_HI = LO, V_LO = LO + HI, V_HI = 2 * LO + HI;
   static constexpr int K_META = 2 * (LO + HI), V_META = K_META + PB * 4;
-  static constexpr int BYTES = V_META + PB * 4;
+  static constexpr int PACKED = V_META + PB * 4;
+  static constexpr int WINDOW = 2 * WIN_V;
+  static constexpr int BYTES = PACKED > WINDOW ? PACKED : WINDOW;
 };
 
 template <int BITS, int G>
@@ -54,22 +60,27 @@ struct Smem {
   alignas(128) unsigned char stage[NW][NSTAGE][StageLayout<BITS>::BYTES];
   float qs[G][D];                          // scaled q' (fp32)
   int8_t qterm[NT * 4][2][D];              // two int8 terms per head (padded heads = 0)
+  __half qh[NT * 4][2][D];                 // fp16 hi/lo terms per head (padded heads = 0)
   float qscale[NT * 4];                    // sigma / 254 per head
   float qsum[NT * 4];                      // sum of the quantised q per head
   uint8_t ps[NW][NT * 8][PS_LD];           // per-warp P terms [col][token]
-  float so_w[NW][G][D];                    // window partial outputs per warp
-  float sm[2 * NW][G], sl[2 * NW][G];      // per-slot softmax max / sum
+  float sm[NW][G], sl[NW][G];              // per-warp softmax max / sum
   alignas(8) uint64_t bar[NW][NSTAGE];
   int is_last;
 };
 
-// Packed partial outputs per warp, placed over the stage buffers once every
-// warp has drained its copy ring.
+// Per-warp partial outputs, placed over the stage buffers once every warp
+// has drained its copy ring.
 template <int BITS, int G>
-__device__ __forceinline__ float (*packed_slots(Smem<BITS, G>& sh))[G][D] {
+__device__ __forceinline__ float (*warp_slots(Smem<BITS, G>& sh))[G][D] {
   static_assert(sizeof(float) * NW * G * D <= sizeof(sh.stage), "stage area too small");
   return reinterpret_cast<float(*)[G][D]>(&sh.stage[0][0][0]);
 }
+
+template <int NT>
+struct SoftmaxState {
+  float m[NT], l[NT], e[NT], o[NT][8][2];   // o: dims 16mt + r (+8) of head 4nt + c
+};
 
 __device__ __forceinline__ float merge_weight(float m, float M) {
   return (m == -INFINITY) ? 0.f : exp2f(m - M);
@@ -77,26 +88,24 @@ __device__ __forceinline__ float merge_weight(float m, float M) {
 
 __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-__device__ __forceinline__ int64_t unit_cost(const DecodeArgs& a) {
-  return (int64_t)a.win_groups * a.cost_w + (int64_t)a.pack_blocks * a.cost_p;
-}
-
-// First item (window group, then packed block) at or after byte offset x of a unit.
-__device__ __forceinline__ int item_at(const DecodeArgs& a, int64_t x) {
-  const int64_t wc = (int64_t)a.win_groups * a.cost_w;
-  if (x <= 0) return 0;
-  if (x < wc) return (int)ceil_div64(x, a.cost_w);
-  const int64_t i = a.win_groups + ceil_div64(x - wc, a.cost_p);
-  return (int)min(i, (int64_t)(a.win_groups + a.pack_blocks));
-}
-
-// CTA whose byte range contains global byte y: CTA i covers
+// CTA whose item range contains global item y: CTA i covers
 // [floor(i T / n), floor((i + 1) T / n)).
 __device__ __forceinline__ int cta_of(int64_t y, int64_t T, int n) {
   return (int)(ceil_div64((y + 1) * n, T) - 1);
 }
 
-// ---- fp16 window tokens: one token per lane -------------------------------------
+// Item i of a unit (0 <= i < win_chunks + pack_blocks): window chunk number
+// floor(i nw / ni) when that count steps up at i, else packed block
+// i - floor(i nw / ni).
+__device__ __forceinline__ bool item_is_window(const DecodeArgs& a, int i, int* idx) {
+  const int64_t ni = a.win_chunks + a.pack_blocks;
+  const int w0 = (int)((int64_t)i * a.win_chunks / ni);
+  const int w1 = (int)((int64_t)(i + 1) * a.win_chunks / ni);
+  if (w1 > w0) { *idx = w0; return true; }
+  *idx = i - w0;
+  return false;
+}
+
 __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const __half* sink,
                                                     const __half* ring, int u, int w) {
   const DevCache& c = a.c;
@@ -105,93 +114,43 @@ __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const _
   return ring + ((size_t)u * c.ring_slots + slot) * D;
 }
 
-template <int BITS, int G>
-__device__ void window_groups(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int g0, int g1,
-                              int warp, int lane) {
+// All lanes: copy item i of unit u into a stage.  Packed blocks: one lane
+// issues the plane and meta copies.  Window chunks: lanes 0-7 copy the K
+// rows, 8-15 the V rows (rows past the window repeat its last row so that
+// the stage holds finite values; their scores are masked).
+template <int BITS, bool AFFINE>
+__device__ __forceinline__ void issue_item(const DecodeArgs& a, int u, int item, unsigned char* st,
+                                           uint64_t* bar, int lane) {
+  using SL = StageLayout<BITS>;
   const DevCache& c = a.c;
-  const int nwin = a.n_sink + a.n_recent;
-  float m[G], l[G], o[G][4];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY; l[g] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[g][i] = 0.f;
-  }
-  for (int grp = g0; grp < g1; ++grp) {
-    const int w = grp * WGRP + lane;
-    const bool valid = w < nwin;
-    float s[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) s[g] = 0.f;
-    const uint4* krow = reinterpret_cast<const uint4*>(window_row(a, c.sink_k, c.ring_k, u, valid ? w : 0));
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint4 raw[D / 16];
-#pragma unroll
-      for (int ch = 0; ch < D / 16; ++ch)
-        raw[ch] = valid ? __ldg(krow + half * (D / 16) + ch) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int ch = 0; ch < D / 16; ++ch) {
-        const __half2* h2 = reinterpret_cast<const __half2*>(&raw[ch]);
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __half22float2(h2[i]);
-          x[2 * i] = f.x; x[2 * i + 1] = f.y;
-        }
-        const int d0 = 8 * (half * (D / 16) + ch);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float4 qa = *reinterpret_cast<const float4*>(&sh.qs[g][d0]);
-          const float4 qb = *reinterpret_cast<const float4*>(&sh.qs[g][d0 + 4]);
-          s[g] = fmaf(qa.x, x[0], s[g]); s[g] = fmaf(qa.y, x[1], s[g]);
-          s[g] = fmaf(qa.z, x[2], s[g]); s[g] = fmaf(qa.w, x[3], s[g]);
-          s[g] = fmaf(qb.x, x[4], s[g]); s[g] = fmaf(qb.y, x[5], s[g]);
-          s[g] = fmaf(qb.z, x[6], s[g]); s[g] = fmaf(qb.w, x[7], s[g]);
-        }
-      }
+  int idx;
+  if (item_is_window(a, item, &idx)) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, 2u * WC * 256u);
+    __syncwarp();
+    if (lane < 2 * WC) {
+      const int nwin = a.n_sink + a.n_recent;
+      const int w = min(idx * WC + (lane & (WC - 1)), nwin - 1);
+      const bool v = lane >= WC;
+      const __half* row = window_row(a, v ? c.sink_v : c.sink_k, v ? c.ring_v : c.ring_k, u, w);
+      bulk_copy_g2s(st + (v ? WIN_V : 0) + (lane & (WC - 1)) * WROW, row, 256u, bar);
     }
-    float p[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float sv = valid ? s[g] : -INFINITY;
-      const float mn = fmaxf(m[g], warp_max_f32(sv));
-      const float al = exp2f(m[g] - mn);
-      p[g] = valid ? exp2f(sv - mn) : 0.f;
-      l[g] = fmaf(l[g], al, p[g]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[g][i] *= al;
-      m[g] = mn;
-    }
-    const int nvalid = min(WGRP, nwin - grp * WGRP);
-    for (int j0 = 0; j0 < nvalid; j0 += 8) {
-      uint2 vr[8];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
-        vr[jj] = (j0 + jj < nvalid)
-                     ? __ldg(reinterpret_cast<const uint2*>(
-                                 window_row(a, c.sink_v, c.ring_v, u, grp * WGRP + j0 + jj)) + lane)
-                     : make_uint2(0u, 0u);
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vr[jj].x));
-        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vr[jj].y));
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pj = __shfl_sync(FULL, p[g], j0 + jj);  // 0 past nvalid
-          o[g][0] = fmaf(pj, v01.x, o[g][0]); o[g][1] = fmaf(pj, v01.y, o[g][1]);
-          o[g][2] = fmaf(pj, v23.x, o[g][2]); o[g][3] = fmaf(pj, v23.y, o[g][3]);
-        }
-      }
-    }
+    return;
   }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float lt = warp_sum_f32(l[g]);
-    if (lane == 0) { sh.sm[warp][g] = m[g]; sh.sl[warp][g] = lt; }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sh.so_w[warp][g][4 * lane + i] = o[g][i];
+  if (lane != 0) return;
+  const int blk = idx;
+  const uint32_t meta = PB * (AFFINE ? 4 : 2);
+  mbar_arrive_expect_tx(bar, 2u * (SL::LO + SL::HI) + 2u * meta);
+  const size_t lo = (size_t)blk * SL::LO;
+  bulk_copy_g2s(st + SL::K_LO, c.k_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
+  bulk_copy_g2s(st + SL::V_LO, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
+  if constexpr (BITS == 3) {
+    const size_t hi = (size_t)blk * SL::HI;
+    bulk_copy_g2s(st + SL::K_HI, c.k_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
+    bulk_copy_g2s(st + SL::V_HI, c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
   }
+  const size_t mo = (size_t)u * c.meta_unit_stride + (size_t)blk * meta;
+  bulk_copy_g2s(st + SL::K_META, c.k_meta + mo, meta, bar);
+  bulk_copy_g2s(st + SL::V_META, c.v_meta + mo, meta, bar);
 }
 
 // ---- packed blocks: copy ring + integer tensor cores ------------------------------
@@ -227,31 +186,6 @@ __device__ __forceinline__ VWords<BITS> stage_v_words(const unsigned char* st, i
   return v;
 }
 
-// One elected lane: copy packed block `blk` of unit u into a stage.
-template <int BITS, bool AFFINE>
-__device__ __forceinline__ void issue_block(const DecodeArgs& a, int u, int blk, unsigned char* st,
-                                            uint64_t* bar) {
-  using SL = StageLayout<BITS>;
-  const DevCache& c = a.c;
-  const uint32_t meta = PB * (AFFINE ? 4 : 2);
-  mbar_arrive_expect_tx(bar, 2u * (SL::LO + SL::HI) + 2u * meta);
-  const size_t lo = (size_t)blk * SL::LO;
-  bulk_copy_g2s(st + SL::K_LO, c.k_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
-  bulk_copy_g2s(st + SL::V_LO, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
-  if constexpr (BITS == 3) {
-    const size_t hi = (size_t)blk * SL::HI;
-    bulk_copy_g2s(st + SL::K_HI, c.k_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
-    bulk_copy_g2s(st + SL::V_HI, c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
-  }
-  const size_t mo = (size_t)u * c.meta_unit_stride + (size_t)blk * meta;
-  bulk_copy_g2s(st + SL::K_META, c.k_meta + mo, meta, bar);
-  bulk_copy_g2s(st + SL::V_META, c.v_meta + mo, meta, bar);
-}
-
-template <int NT>
-struct PackedState {
-  float m[NT], l[NT], e[NT], o[NT][8][2];
-};
 
 // Lane = 4r + c.  Score m-tile rows r, r+8 are tokens; columns are (head,
 // term) pairs, so thread c owns head 4nt + c of n-tile nt.  PV m-tile rows
@@ -261,7 +195,7 @@ template <int BITS, int G, bool AFFINE, bool FULL>
 __device__ __forceinline__ void packed_block_compute(
     const DecodeArgs& a, Smem<BITS, G>& sh, const unsigned char* st, int blk, int warp, int lane,
     const uint32_t (&qb)[(G + 3) / 4][4][2], const float (&qscale)[(G + 3) / 4],
-    const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], PackedState<(G + 3) / 4>& S) {
+    const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   using SL = StageLayout<BITS>;
   const int r = lane >> 2, c4 = lane & 3;
@@ -404,17 +338,101 @@ __device__ __forceinline__ void packed_block_compute(
   }
 }
 
-// The warp's packed blocks [pb0, pb1) of unit u through its copy ring.  `it`
-// counts the blocks this warp has consumed (stage = it % NSTAGE, phase parity
-// = (it / NSTAGE) & 1).
-template <int BITS, int G, bool AFFINE>
-__device__ void packed_blocks(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int pb0, int pb1,
-                              int warp, int lane, uint32_t& it, PackedState<(G + 3) / 4>& S) {
+// Power-of-two factor of a PV dim row in the packed path (shift-free
+// fragments); window contributions are brought to the same units.
+template <int BITS>
+__device__ __forceinline__ float row_factor(int rho) {
+  if constexpr (BITS == 3) return 1.f;
+  else return 1.f / v_row_scale<BITS>(rho);
+}
+
+// One window chunk (8 fp16 tokens) from its stage: scores with fp16 MMA
+// (rows 8-15 of the m16 tile are empty), PV with the transposed rows.
+template <int BITS, int G>
+__device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<BITS, G>& sh,
+                                                     const unsigned char* st, int wc, int lane,
+                                                     SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
+  const bool valid = wc * WC + r < a.n_sink + a.n_recent;
+  // lane supplies row (lane % 8) of matrix (lane / 8): 8 dims at 16-byte steps
+  const uint32_t row_addr = smem_addr(st) + (lane & 7) * WROW + (lane >> 3) * 16;
+
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t kf[4];
+    ldmatrix_x4(kf, row_addr + kk * 64);          // dims 32kk .. 32kk + 31
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int ks = 2 * kk + hf;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const __half* qrow = &sh.qh[nt * 4 + (r >> 1)][r & 1][16 * ks + 2 * c4];
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qrow);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qrow + 8);
+        mma_f16_k16(acc[nt], kf[2 * hf], 0u, kf[2 * hf + 1], 0u, b0, b1);
+      }
+    }
+  }
+
+  float al[NT];
+  uint32_t pb[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float s = valid ? acc[nt][0] + acc[nt][1] : -INFINITY;   // hi + lo query terms
+    float bm = s;
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
+    const float mn = fmaxf(S.m[nt], bm);
+    al[nt] = exp2f(S.m[nt] - mn);
+    S.m[nt] = mn;
+    const float p = valid ? exp2f(s - mn) : 0.f;
+    S.l[nt] = fmaf(S.l[nt], al[nt], p);
+    S.e[nt] *= al[nt];
+    // B fragment of PV: p of tokens 2c, 2c+1 for column r = (head r/2, term r%2)
+    const float pa = __shfl_sync(FULL_MASK, p, 8 * c4 + (r >> 1));
+    const float pc = __shfl_sync(FULL_MASK, p, 8 * c4 + 4 + (r >> 1));
+    __half ha = __float2half_rn(pa), hc = __float2half_rn(pc);
+    if (r & 1) {
+      ha = __float2half_rn(pa - __half2float(ha));
+      hc = __float2half_rn(pc - __half2float(hc));
+    }
+    const __half2 h2 = __halves2half2(ha, hc);
+    pb[nt] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t vf[4];
+    ldmatrix_x4_trans(vf, row_addr + WIN_V + q * 64);   // dims 32q .. 32q + 31
+#pragma unroll
+    for (int hm = 0; hm < 2; ++hm) {
+      const int mt = 2 * q + hm;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_k8(d, vf[2 * hm], vf[2 * hm + 1], pb[nt]);
+        S.o[nt][mt][0] = fmaf(S.o[nt][mt][0], al[nt], row_factor<BITS>(2 * mt) * (d[0] + d[1]));
+        S.o[nt][mt][1] = fmaf(S.o[nt][mt][1], al[nt], row_factor<BITS>(2 * mt + 1) * (d[2] + d[3]));
+      }
+    }
+  }
+}
+
+// The warp's items [i0, i1) of unit u through its copy ring.  `it` counts the
+// items this warp has consumed (stage = it % NSTAGE, phase parity =
+// (it / NSTAGE) & 1).
+template <int BITS, int G, bool AFFINE>
+__device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0, int i1, int warp,
+                           int lane, uint32_t& it, SoftmaxState<(G + 3) / 4>& S) {
+  constexpr int NT = (G + 3) / 4;
+  const int r = lane >> 2, c4 = lane & 3;
+  const float beta = 0.5f - (float)(1 << (BITS - 1));
   uint32_t qb[NT][4][2];
   float qscale[NT], qsum[NT], qoff[NT];
-  const float beta = 0.5f - (float)(1 << (BITS - 1));
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int gcol = nt * 4 + (r >> 1), term = r & 1;
@@ -430,37 +448,38 @@ __device__ void packed_blocks(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) S.o[nt][mt][0] = S.o[nt][mt][1] = 0.f;
   }
-  const int nblk = pb1 - pb0;
-  if (nblk <= 0) return;
-  if (lane == 0) {
-    for (int j = 0; j < NSTAGE && j < nblk; ++j) {
-      const int stg = (it + j) % NSTAGE;
-      issue_block<BITS, AFFINE>(a, u, pb0 + j, sh.stage[warp][stg], &sh.bar[warp][stg]);
-    }
+  const int n = i1 - i0;
+  if (n <= 0) return;
+  for (int j = 0; j < NSTAGE && j < n; ++j) {
+    const int stg = (it + j) % NSTAGE;
+    issue_item<BITS, AFFINE>(a, u, i0 + j, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
   }
-  for (int i = 0; i < nblk; ++i, ++it) {
+  for (int i = 0; i < n; ++i, ++it) {
     const int stg = it % NSTAGE;
     if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
       // A copy never completed: report it, drain what is still in flight
       // (bounded), and contribute nothing.
       if (lane == 0) atomicOr(a.c.status, DEV_ERR_TIMEOUT);
-      for (int j = i; j < nblk && j < i + NSTAGE; ++j)
+      for (int j = i; j < n && j < i + NSTAGE; ++j)
         mbar_wait_bounded(&sh.bar[warp][(it + j - i) % NSTAGE], ((it + j - i) / NSTAGE) & 1, WAIT_POLLS);
-      it += (uint32_t)(nblk - i);
+      it += (uint32_t)(n - i);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
       return;
     }
-    if ((pb0 + i + 1) * PB <= a.n_packed)
-      packed_block_compute<BITS, G, AFFINE, true>(a, sh, sh.stage[warp][stg], pb0 + i, warp, lane, qb,
-                                                  qscale, qoff, qsum, S);
-    else
-      packed_block_compute<BITS, G, AFFINE, false>(a, sh, sh.stage[warp][stg], pb0 + i, warp, lane, qb,
-                                                   qscale, qoff, qsum, S);
+    const unsigned char* st = sh.stage[warp][stg];
+    int idx;
+    if (item_is_window(a, i0 + i, &idx)) {
+      window_chunk_compute<BITS, G>(a, sh, st, idx, lane, S);
+    } else if ((idx + 1) * PB <= a.n_packed) {
+      packed_block_compute<BITS, G, AFFINE, true>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+    } else {
+      packed_block_compute<BITS, G, AFFINE, false>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+    }
     __syncwarp();
-    if (lane == 0 && i + NSTAGE < nblk) {
+    if (i + NSTAGE < n) {
       fence_proxy_async();
-      issue_block<BITS, AFFINE>(a, u, pb0 + i + NSTAGE, sh.stage[warp][stg], &sh.bar[warp][stg]);
+      issue_item<BITS, AFFINE>(a, u, i0 + i + NSTAGE, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
     }
   }
 }
@@ -476,7 +495,8 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
   const int r = lane >> 2, c4 = lane & 3;
   const int Hq = c.n_kv_heads * G;
   const int ncta = (int)gridDim.x, cta = (int)blockIdx.x;
-  const int64_t Cu = unit_cost(a), T = Cu * c.units;
+  const int64_t NI = (int64_t)a.win_chunks + a.pack_blocks;   // items per unit
+  const int64_t T = NI * c.units;
   const int64_t x0 = T * cta / ncta, x1 = T * (cta + 1) / ncta;
 
   if (tid < NW * NSTAGE) mbar_init(&sh.bar[tid / NSTAGE][tid % NSTAGE], 1);
@@ -484,13 +504,13 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
   __syncthreads();
   uint32_t it = 0;
 
-  const int u_first = (int)(x0 / Cu), u_last = (int)((x1 - 1) / Cu);
+  const int u_first = (int)(x0 / NI), u_last = (int)((x1 - 1) / NI);
   for (int u = u_first; u <= u_last; ++u) {
     const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
-    const int64_t ub = (int64_t)u * Cu;
-    const int64_t s0 = max(x0, ub) - ub, s1 = min(x1, ub + Cu) - ub;
+    const int64_t ub = (int64_t)u * NI;
+    const int s0 = (int)(max(x0, ub) - ub), s1 = (int)(min(x1, ub + NI) - ub);
 
-    // ---- scaled query and its two int8 terms per head ----------------------
+    // ---- scaled query: two int8 terms and two fp16 terms per head ---------------
     for (int g = 0; g < G; ++g)
       sh.qs[g][tid] = a.q[((size_t)b * Hq + (size_t)h * G + g) * D + tid] * a.scale_log2;
     __syncthreads();
@@ -511,9 +531,12 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
         sh.qterm[g][0][4 * lane + i] = (int8_t)t0;
         sh.qterm[g][1][4 * lane + i] = (int8_t)t1;
         sum += (int)t0 * 254 + (int)t1;
+        const __half hi = __float2half_rn(x[i]);
+        sh.qh[g][0][4 * lane + i] = hi;
+        sh.qh[g][1][4 * lane + i] = __float2half_rn(x[i] - __half2float(hi));
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
       if (lane == 0) {
         sh.qscale[g] = sigma / 254.f;
         sh.qsum[g] = (sigma / 254.f) * (float)sum;
@@ -521,58 +544,47 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     }
     __syncthreads();
 
-    // ---- this warp's byte share of the segment --------------------------------
-    const int64_t w0 = s0 + (s1 - s0) * warp / NW, w1 = s0 + (s1 - s0) * (warp + 1) / NW;
-    const int i0 = item_at(a, w0), i1 = item_at(a, w1);
-    const int wg0 = min(i0, a.win_groups), wg1 = min(i1, a.win_groups);
-    const int pb0 = max(i0, a.win_groups) - a.win_groups;
-    const int pb1 = max(i1, a.win_groups) - a.win_groups;
-    window_groups<BITS, G>(a, sh, u, wg0, wg1, warp, lane);
-    PackedState<NT> S;
-    packed_blocks<BITS, G, AFFINE>(a, sh, u, pb0, pb1, warp, lane, it, S);
+    // ---- this warp's items ------------------------------------------------------
+    const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
+    const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
+    SoftmaxState<NT> S;
+    warp_items<BITS, G, AFFINE>(a, sh, u, w0, w1, warp, lane, it, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
 
-    float (*so_p)[G][D] = packed_slots(sh);
+    float (*so)[G][D] = warp_slots(sh);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float lt = S.l[nt], et = S.e[nt];
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
-        lt += __shfl_xor_sync(FULL, lt, o);
-        et += __shfl_xor_sync(FULL, et, o);
+        lt += __shfl_xor_sync(FULL_MASK, lt, o);
+        et += __shfl_xor_sync(FULL_MASK, et, o);
       }
       if constexpr (!AFFINE) et *= 0.5f - (float)(1 << (BITS - 1));  // sum p*delta*beta
       const int g = nt * 4 + c4;
       if (g < G) {
-        if (r == 0) { sh.sm[NW + warp][g] = S.m[nt]; sh.sl[NW + warp][g] = lt; }
+        if (r == 0) { sh.sm[warp][g] = S.m[nt]; sh.sl[warp][g] = lt; }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const float s0 = BITS == 3 ? 1.f : v_row_scale<BITS == 3 ? 2 : BITS>(2 * mt);
-          const float s1 = BITS == 3 ? 1.f : v_row_scale<BITS == 3 ? 2 : BITS>(2 * mt + 1);
-          so_p[warp][g][16 * mt + r] = fmaf(S.o[nt][mt][0], s0, et);
-          so_p[warp][g][16 * mt + r + 8] = fmaf(S.o[nt][mt][1], s1, et);
+          so[warp][g][16 * mt + r] = fmaf(S.o[nt][mt][0], 1.f / row_factor<BITS>(2 * mt), et);
+          so[warp][g][16 * mt + r + 8] = fmaf(S.o[nt][mt][1], 1.f / row_factor<BITS>(2 * mt + 1), et);
         }
       }
     }
     __syncthreads();
 
-    // ---- merge the CTA's 2 NW slots, write its partial for this unit -----------
+    // ---- merge the warps, write this CTA's partial for the unit -----------------
     const int k = cta - cta_of(ub, T, ncta);
-    const int nparts = cta_of(ub + Cu - 1, T, ncta) - cta_of(ub, T, ncta) + 1;
+    const int nparts = cta_of(ub + NI - 1, T, ncta) - cta_of(ub, T, ncta) + 1;
     float* part_base = a.partials + ((size_t)u * c.max_splits + k) * G * (D + 2);
     for (int g = 0; g < G; ++g) {
       float M = -INFINITY;
-      for (int s = 0; s < 2 * NW; ++s) M = fmaxf(M, sh.sm[s][g]);
+      for (int s = 0; s < NW; ++s) M = fmaxf(M, sh.sm[s][g]);
       float L = 0.f, O = 0.f;
       for (int s = 0; s < NW; ++s) {
         const float f = merge_weight(sh.sm[s][g], M);
         L = fmaf(sh.sl[s][g], f, L);
-        O = fmaf(sh.so_w[s][g][tid], f, O);
-      }
-      for (int s = 0; s < NW; ++s) {
-        const float f = merge_weight(sh.sm[NW + s][g], M);
-        L = fmaf(sh.sl[NW + s][g], f, L);
-        O = fmaf(so_p[s][g][tid], f, O);
+        O = fmaf(so[s][g][tid], f, O);
       }
       float* part = part_base + (size_t)g * (D + 2);
       part[tid] = O;
@@ -602,7 +614,7 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
       if (tid == 0) a.counters[u] = 0;
     }
     __syncthreads();
-    fence_proxy_async();  // stage area was written as slots; next copies overwrite it
+    fence_proxy_async();  // the stage area was written as slots; next copies overwrite it
   }
 }
 

@@ -254,10 +254,9 @@ struct DecodeArgs {
   float scale_log2;        // scale * log2(e)
   int n_sink, n_packed, n_recent;
   int ring_first;          // ring slot of the oldest recent token
-  int grid;                // CTAs (stream-K shares of the units' bytes)
-  int win_groups;          // ceil((n_sink + n_recent) / 32)
+  int grid;                // CTAs (stream-K shares of the units' items)
+  int win_chunks;          // ceil((n_sink + n_recent) / 8)
   int pack_blocks;         // ceil(n_packed / 64)
-  int64_t cost_w, cost_p;  // bytes of one window group / one packed block
   float* partials;         // split partials [unit][max_splits][G][130]
   int* counters;           // arrival counter per unit
 };
