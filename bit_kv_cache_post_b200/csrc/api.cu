@@ -33,6 +33,9 @@ constexpr int WIN_CHUNK = 8;
 constexpr int PACK_BLOCK = 64;
 constexpr int64_t MIN_CTA_ITEMS = 8;
 constexpr int MAX_GRID = 2048;
+// The unit-merging CTA stages the (m, l) of all partials of a unit in its
+// shared memory; at most this many partials per unit.
+constexpr int MAX_PARTS_PER_UNIT = 256;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -105,7 +108,7 @@ int max_splits_for(const wushkv_config& c, int packed_capacity) {
   (void)packed_capacity;
   const int units = c.batch * c.n_kv_heads;
   const int ms = MAX_GRID / units + 2;
-  return ms > 3 ? ms : 3;
+  return ms < 3 ? 3 : (ms > MAX_PARTS_PER_UNIT ? MAX_PARTS_PER_UNIT : ms);
 }
 
 void make_layout(const wushkv_config& c, wushkv_layout* L) {
@@ -134,7 +137,7 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
   L->ring_v_off = off; off = align_up(off + U * L->ring_unit_stride, 256);
   const int ms = max_splits_for(c, L->packed_capacity);
   L->workspace_off = off;
-  L->workspace_bytes = U * (size_t)ms * G * (128 + 2) * sizeof(float) + U * sizeof(int);
+  L->workspace_bytes = U * (size_t)ms * G * PARTIAL_FLOATS * sizeof(float) + U * sizeof(int);
   off = align_up(off + L->workspace_bytes, 256);
   L->status_off = off; off = align_up(off + 256, 256);
   L->total_bytes = off;
@@ -169,7 +172,7 @@ DevCache dev_view(const wushkv_cache* h) {
   d.partials = reinterpret_cast<float*>(h->base + L.workspace_off);
   d.counters = reinterpret_cast<int*>(h->base + L.workspace_off +
                                       U * (size_t)d.max_splits * (c.n_q_heads / c.n_kv_heads) *
-                                          (128 + 2) * sizeof(float));
+                                          PARTIAL_FLOATS * sizeof(float));
   d.status = reinterpret_cast<int*>(h->base + L.status_off);
   d.units = (int)U;
   d.n_kv_heads = c.n_kv_heads;
@@ -385,6 +388,7 @@ wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const f
 wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream) {
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
+  if (reinterpret_cast<uintptr_t>(out_dev) & 15) return WUSHKV_EINVAL;  // written as float4
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   DecodeArgs a;
   if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
@@ -515,6 +519,7 @@ void* g_noalloc_addr[64] = {nullptr};
 extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const wushkv_cache* cache,
                                                 float* out_dev, float scale, void* stream) {
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
+  if (reinterpret_cast<uintptr_t>(out_dev) & 15) return WUSHKV_EINVAL;  // written as float4
   if (cache->n == 0) return WUSHKV_EINVAL;
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   int dev = 0;
@@ -532,7 +537,7 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   const int total = (a.grid + a.c.units - 1) / a.c.units + 1;
   a.c.max_splits = total;
   const size_t units = (size_t)a.c.units;
-  const size_t partial_bytes = units * (size_t)total * a.c.group * (128 + 2) * sizeof(float);
+  const size_t partial_bytes = units * (size_t)total * a.c.group * PARTIAL_FLOATS * sizeof(float);
   if (units * sizeof(int) > NOALLOC_COUNTER_BYTES ||
       partial_bytes > NOALLOC_SCRATCH_BYTES - NOALLOC_COUNTER_BYTES)
     return WUSHKV_ECAPACITY;

@@ -40,6 +40,7 @@ constexpr int PS_LD = PB + 16;   // bytes per row of the per-warp P tile
 constexpr int NSTAGE = 2;        // per-warp copy stages
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr unsigned FULL_MASK = 0xffffffffu;
+constexpr int PART = PARTIAL_FLOATS;  // floats per partial record (16-byte rows)
 
 // Bytes of one packed block in a stage: K planes, V planes, K meta, V meta.
 template <int BITS>
@@ -422,9 +423,18 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
   }
 }
 
-// The warp's items [i0, i1) of unit u through its copy ring.  `it` counts the
-// items this warp has consumed (stage = it % NSTAGE, phase parity =
-// (it / NSTAGE) & 1).
+// First copies of the warp's items, issued before the query prologue.
+template <int BITS, bool AFFINE, int G>
+__device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, Smem<BITS, G>& sh, int u,
+                                                    int i0, int i1, int warp, int lane, uint32_t it) {
+  for (int j = 0; j < NSTAGE && j < i1 - i0; ++j) {
+    const int stg = (it + j) % NSTAGE;
+    issue_item<BITS, AFFINE>(a, u, i0 + j, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+  }
+}
+
+// The warp's items [i0, i1) of unit u through its copy ring (the first
+// NSTAGE copies were issued by warp_items_prefetch).
 template <int BITS, int G, bool AFFINE>
 __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0, int i1, int warp,
                            int lane, uint32_t& it, SoftmaxState<(G + 3) / 4>& S) {
@@ -450,10 +460,6 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
   }
   const int n = i1 - i0;
   if (n <= 0) return;
-  for (int j = 0; j < NSTAGE && j < n; ++j) {
-    const int stg = (it + j) % NSTAGE;
-    issue_item<BITS, AFFINE>(a, u, i0 + j, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
-  }
   for (int i = 0; i < n; ++i, ++it) {
     const int stg = it % NSTAGE;
     if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
@@ -509,6 +515,10 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
     const int64_t ub = (int64_t)u * NI;
     const int s0 = (int)(max(x0, ub) - ub), s1 = (int)(min(x1, ub + NI) - ub);
+    // this warp's items; their first copies overlap the query prologue
+    const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
+    const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
+    warp_items_prefetch<BITS, AFFINE, G>(a, sh, u, w0, w1, warp, lane, it);
 
     // ---- scaled query: two int8 terms and two fp16 terms per head ---------------
     for (int g = 0; g < G; ++g)
@@ -545,8 +555,6 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     __syncthreads();
 
     // ---- this warp's items ------------------------------------------------------
-    const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
-    const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
     SoftmaxState<NT> S;
     warp_items<BITS, G, AFFINE>(a, sh, u, w0, w1, warp, lane, it, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
@@ -576,7 +584,7 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     // ---- merge the warps, write this CTA's partial for the unit -----------------
     const int k = cta - cta_of(ub, T, ncta);
     const int nparts = cta_of(ub + NI - 1, T, ncta) - cta_of(ub, T, ncta) + 1;
-    float* part_base = a.partials + ((size_t)u * c.max_splits + k) * G * (D + 2);
+    float* part_base = a.partials + ((size_t)u * c.max_splits + k) * G * PART;
     for (int g = 0; g < G; ++g) {
       float M = -INFINITY;
       for (int s = 0; s < NW; ++s) M = fmaxf(M, sh.sm[s][g]);
@@ -586,30 +594,59 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
         L = fmaf(sh.sl[s][g], f, L);
         O = fmaf(so[s][g][tid], f, O);
       }
-      float* part = part_base + (size_t)g * (D + 2);
+      float* part = part_base + (size_t)g * PART;
       part[tid] = O;
       if (tid == 0) { part[D] = M; part[D + 1] = L; }
     }
 
     // ---- arrival: the last CTA of the unit merges its partials ------------------
-    __threadfence();
+    // The barrier orders every thread's partial writes before thread 0's
+    // acq_rel atomic, which publishes them at gpu scope (release) and, for
+    // the last arrival, makes the other CTAs' partials visible (acquire).
     __syncthreads();
-    if (tid == 0) sh.is_last = (atomicAdd(a.counters + u, 1) == nparts - 1);
+    if (tid == 0) {
+      int prev;
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;\n"
+                   : "=r"(prev) : "l"(a.counters + u) : "memory");
+      sh.is_last = (prev == nparts - 1);
+    }
     __syncthreads();
     if (sh.is_last) {
-      __threadfence();
-      for (int g = 0; g < G; ++g) {
+      // M, L of every partial into the (free) stage area, then each warp
+      // merges its heads with 16-byte loads, eight partials in flight.
+      float* cm = reinterpret_cast<float*>(&sh.stage[0][0][0]) + NW * G * D;
+      float* cl = cm + nparts * G;
+      const float* pbase = a.partials + (size_t)u * c.max_splits * G * PART;
+      for (int i = tid; i < nparts * G; i += NW * 32) {
+        const float* part = pbase + (size_t)i * PART;   // i = sp * G + g
+        cm[i] = __ldcg(part + D);
+        cl[i] = __ldcg(part + D + 1);
+      }
+      __syncthreads();
+      for (int g = warp; g < G; g += NW) {
         float M = -INFINITY;
-        for (int sp = 0; sp < nparts; ++sp)
-          M = fmaxf(M, __ldcg(a.partials + (((size_t)u * c.max_splits + sp) * G + g) * (D + 2) + D));
-        float L = 0.f, O = 0.f;
-        for (int sp = 0; sp < nparts; ++sp) {
-          const float* part = a.partials + (((size_t)u * c.max_splits + sp) * G + g) * (D + 2);
-          const float f = merge_weight(__ldcg(part + D), M);
-          L = fmaf(__ldcg(part + D + 1), f, L);
-          O = fmaf(__ldcg(part + tid), f, O);
+        for (int sp = 0; sp < nparts; ++sp) M = fmaxf(M, cm[sp * G + g]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp0 = 0; sp0 < nparts; sp0 += 8) {
+          float4 v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            v[j] = sp0 + j < nparts
+                       ? __ldcg(reinterpret_cast<const float4*>(pbase + ((size_t)(sp0 + j) * G + g) * PART) + lane)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (sp0 + j >= nparts) break;
+            const float f = merge_weight(cm[(sp0 + j) * G + g], M);
+            L = fmaf(cl[(sp0 + j) * G + g], f, L);
+            O.x = fmaf(v[j].x, f, O.x); O.y = fmaf(v[j].y, f, O.y);
+            O.z = fmaf(v[j].z, f, O.z); O.w = fmaf(v[j].w, f, O.w);
+          }
         }
-        a.out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = O / L;
+        const float il = 1.f / L;
+        *reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)h * G + g) * D + 4 * lane) =
+            make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
       }
       if (tid == 0) a.counters[u] = 0;
     }

@@ -11,6 +11,7 @@
 namespace wushkv {
 
 constexpr int D = 128;           // head_dim
+constexpr int PARTIAL_FLOATS = D + 4;   // o[128], m, l, 2 pad: one split partial of one head
 constexpr unsigned FULL = 0xffffffffu;
 
 // Device-visible view of one cache buffer.
@@ -257,7 +258,7 @@ struct DecodeArgs {
   int grid;                // CTAs (stream-K shares of the units' items)
   int win_chunks;          // ceil((n_sink + n_recent) / 8)
   int pack_blocks;         // ceil(n_packed / 64)
-  float* partials;         // split partials [unit][max_splits][G][130]
+  float* partials;         // split partials [unit][max_splits][G][132]
   int* counters;           // arrival counter per unit
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

@@ -185,7 +185,7 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
  *   dequantisation happens inside the score and PV loops.
  *   q_prime_dev: [batch][n_q_heads][128] fp32 transformed queries.
  *   out_dev:     [batch][n_q_heads][128] fp32 = softmax(scale q'.k'^T) v
- *                in the transformed value space.
+ *                in the transformed value space; 16-byte aligned (EINVAL otherwise).
  *   scale: softmax scale; 0 selects 1/sqrt(128).
  * Uses the cache's workspace region for split-K partials; calls on the same
  * cache must therefore be stream-ordered.  EINVAL if the cache is empty. */
@@ -211,7 +211,7 @@ WUSHKV_API wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_ca
  *     overlap on the GPU (other streams, threads or caches) race: issue
  *     them one after another.
  *   - WUSHKV_ECAPACITY, with nothing launched, when this call's partials
- *     (units x splits x G x 520 bytes) exceed 8 MiB minus 256 KiB of
+ *     (units x splits x G x 528 bytes) exceed 8 MiB minus 256 KiB of
  *     counters, or the cache has more than 65536 units.
  * Other errors as wushkv_decode. */
 WUSHKV_API wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const wushkv_cache* cache,

@@ -60,7 +60,7 @@ def test_noalloc_matches_decode_two_calls(wk):
 
 
 def test_noalloc_rejects_oversize_scratch(wk):
-    """2048 units x G 8 need at least one split each: 2048 x 8 x 520 B of
+    """2048 units x G 8 need at least one split each: 2048 x 8 x 528 B of
     partials exceed the fixed array, so the call is refused, not run."""
     import torch
     lib = wk.load()
