@@ -379,7 +379,8 @@ wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const f
   if (!q_dev || !T_k_invT_dev || !q_out_dev || !valid_dtype(q_dtype)) return WUSHKV_EINVAL;
   if (reinterpret_cast<uintptr_t>(T_k_invT_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads) return WUSHKV_EINVAL;
-  if (n_q_heads / n_kv_heads > 16) return WUSHKV_EUNSUPPORTED;
+  const int g = n_q_heads / n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16) return WUSHKV_EUNSUPPORTED;
   if ((int64_t)batch * n_kv_heads > 2147483647LL) return WUSHKV_EUNSUPPORTED;
   return cuda_status(launch_query_transform(q_dev, q_dtype, T_k_invT_dev, q_out_dev, batch,
                                             n_q_heads, n_kv_heads, static_cast<cudaStream_t>(stream)));

@@ -51,10 +51,12 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   const int64_t q_last = min(q_first + a.quads_per_cta, a.quad_begin + a.n_quads);
   if (q_first >= q_last) return;
 
-  // Stage T^T of this head once per CTA if any new key needs the product.
+  // Stage T^T of this head once per CTA if several quads need the product;
+  // a single quad reads T's rows directly instead.
   const bool has_new = (4 * q_last > n0) && (4 * q_first < n1);
   const bool transform = (a.T != nullptr) && has_new;
-  if (transform) stage_transpose_128(a.T + (size_t)h * D * D, Tt, TT_LD);
+  const bool staged = transform && (q_last - q_first > 1);
+  if (staged) stage_transpose_128(a.T + (size_t)h * D * D, Tt, TT_LD);
 
   const size_t plane_u0 = (size_t)u * c.plane_unit_stride[0];
   const size_t plane_u1 = (size_t)u * c.plane_unit_stride[1];
@@ -81,18 +83,25 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     }
     __syncthreads();
     // ---- key transform k' = T k (fp32 FMA), one output dim per thread ------
-    for (int j = 0; j < 4; ++j) {
-      if (kind_s[j] != TOK_NEW) continue;
-      float acc;
-      if (transform) {
-        acc = 0.f;
-        const float* kj = kin + j * D;
+    if (transform && !staged) {
+      float dots[4];
+      row_dots<4>(a.T + (size_t)h * D * D, tid, kin, dots);
+      for (int j = 0; j < 4; ++j)
+        if (kind_s[j] == TOK_NEW) k16[j * D + tid] = round_f16(dots[j]);
+    } else {
+      for (int j = 0; j < 4; ++j) {
+        if (kind_s[j] != TOK_NEW) continue;
+        float acc;
+        if (transform) {
+          acc = 0.f;
+          const float* kj = kin + j * D;
 #pragma unroll 8
-        for (int jj = 0; jj < D; ++jj) acc = fmaf(Tt[jj * TT_LD + tid], kj[jj], acc);
-      } else {
-        acc = kin[j * D + tid];
+          for (int jj = 0; jj < D; ++jj) acc = fmaf(Tt[jj * TT_LD + tid], kj[jj], acc);
+        } else {
+          acc = kin[j * D + tid];
+        }
+        k16[j * D + tid] = round_f16(acc);
       }
-      k16[j * D + tid] = round_f16(acc);
     }
     __syncthreads();
     // ---- destinations --------------------------------------------------------

@@ -61,7 +61,7 @@ struct Smem {
   alignas(128) unsigned char stage[NW][NSTAGE][StageLayout<BITS>::BYTES];
   float qs[G][D];                          // scaled q' (fp32)
   int8_t qterm[NT * 4][2][D];              // two int8 terms per head (padded heads = 0)
-  __half qh[NT * 4][2][D];                 // fp16 hi/lo terms per head (padded heads = 0)
+  __half qh[NT * 4][2][D + 8];             // fp16 hi/lo terms per head (rows padded: banks)
   float qscale[NT * 4];                    // sigma / 254 per head
   float qsum[NT * 4];                      // sum of the quantised q per head
   uint8_t ps[NW][NT * 8][PS_LD];           // per-warp P terms [col][token]
@@ -83,8 +83,15 @@ struct SoftmaxState {
   float m[NT], l[NT], e[NT], o[NT][8][2];   // o: dims 16mt + r (+8) of head 4nt + c
 };
 
+// 2^x with the SFU (approximate, flushes denormal results to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float merge_weight(float m, float M) {
-  return (m == -INFINITY) ? 0.f : exp2f(m - M);
+  return (m == -INFINITY) ? 0.f : ex2(m - M);
 }
 
 __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -257,14 +264,14 @@ __device__ __forceinline__ void packed_block_compute(
     bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
     bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
     const float mn = fmaxf(S.m[nt], bm);
-    al[nt] = exp2f(S.m[nt] - mn);
+    al[nt] = ex2(S.m[nt] - mn);
     S.m[nt] = mn;
     float ls = 0.f, es = 0.f, pm = 0.f;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        const float p = exp2f(sc[mt][th][nt] - mn);   // masked tokens: exp2(-inf) = 0
+        const float p = ex2(sc[mt][th][nt] - mn);   // masked tokens: exp2(-inf) = 0
         float pt = p * vs[mt][th];
         if constexpr (!FULL) pt = (16 * mt + r + 8 * th < nvalid) ? pt : 0.f;
         ls += p;
@@ -389,9 +396,9 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
     bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
     bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
     const float mn = fmaxf(S.m[nt], bm);
-    al[nt] = exp2f(S.m[nt] - mn);
+    al[nt] = ex2(S.m[nt] - mn);
     S.m[nt] = mn;
-    const float p = valid ? exp2f(s - mn) : 0.f;
+    const float p = valid ? ex2(s - mn) : 0.f;
     S.l[nt] = fmaf(S.l[nt], al[nt], p);
     S.e[nt] *= al[nt];
     // B fragment of PV: p of tokens 2c, 2c+1 for column r = (head r/2, term r%2)

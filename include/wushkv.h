@@ -175,7 +175,8 @@ WUSHKV_API wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_d
  *   q_dev:        [batch][n_q_heads][128], dtype q_dtype.
  *   T_k_invT_dev: [n_kv_heads][128][128] fp32 row-major, q'_i = sum_j M[i][j] q_j,
  *                 16-byte aligned (EINVAL otherwise).
- *   q_out_dev:    [batch][n_q_heads][128] fp32 (kept fp32 for the decode). */
+ *   q_out_dev:    [batch][n_q_heads][128] fp32 (kept fp32 for the decode).
+ * G = n_q_heads / n_kv_heads must be 1, 2, 4, 8 or 16 (EUNSUPPORTED otherwise). */
 WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
                                      float* q_out_dev, int32_t batch, int32_t n_q_heads,
                                      int32_t n_kv_heads, void* stream);
