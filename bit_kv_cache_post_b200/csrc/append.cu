@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   const bool transform = (a.T != nullptr) && has_new;
   const bool staged = transform && (q_last - q_first > 1);
   if (staged) stage_transpose_128(a.T + (size_t)h * D * D, Tt, TT_LD);
+  MatRow trow;   // single quad: this thread's row of T, requested before the inputs
+  if (transform && !staged) load_row(a.T + (size_t)h * D * D, tid, trow);
 
   const size_t plane_u0 = (size_t)u * c.plane_unit_stride[0];
   const size_t plane_u1 = (size_t)u * c.plane_unit_stride[1];
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     // ---- key transform k' = T k (fp32 FMA), one output dim per thread ------
     if (transform && !staged) {
       float dots[4];
-      row_dots<4>(a.T + (size_t)h * D * D, tid, kin, dots);
+      row_dots<4>(trow, kin, dots);
       for (int j = 0; j < 4; ++j)
         if (kind_s[j] == TOK_NEW) k16[j * D + tid] = round_f16(dots[j]);
     } else {

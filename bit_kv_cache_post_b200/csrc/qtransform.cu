@@ -24,12 +24,14 @@ __global__ void __launch_bounds__(128) qtransform_kernel(const void* q, int dtyp
   const int Hq = n_kv_heads * G;
   const int b = blockIdx.x / n_kv_heads, h = blockIdx.x % n_kv_heads;
   const int tid = threadIdx.x;
+  MatRow row;
+  load_row(TinvT + (size_t)h * D * D, tid, row);
 #pragma unroll
   for (int g = 0; g < G; ++g)
     qs[g][tid] = load_q(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
   __syncthreads();
   float dots[G];
-  row_dots<G>(TinvT + (size_t)h * D * D, tid, &qs[0][0], dots);
+  row_dots<G>(row, &qs[0][0], dots);
 #pragma unroll
   for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = dots[g];
 }

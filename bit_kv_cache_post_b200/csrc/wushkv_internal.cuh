@@ -105,32 +105,34 @@ __device__ __forceinline__ void stage_transpose_128(const float* __restrict__ M,
   }
 }
 
-// out[j] = dot(row `row` of the row-major 128 x 128 matrix M, x[j][0..127])
-// for j < NV vectors held in shared memory (x: [NV][128] floats).  The row is
-// streamed from global memory in 16-byte loads, sixteen in flight; used when
-// a CTA has too few vectors to amortise staging the whole matrix.
-template <int NV>
-__device__ __forceinline__ void row_dots(const float* __restrict__ M, int row, const float* x,
-                                         float (&out)[NV]) {
+// One row of a row-major 128 x 128 fp32 matrix in registers (32 x 16 bytes),
+// loaded with every request in flight at once.  Used when a CTA has too few
+// vectors to amortise staging the whole matrix: load the row first, then the
+// vectors, so that both latencies overlap.
+struct MatRow {
+  float4 v[32];
+};
+
+__device__ __forceinline__ void load_row(const float* __restrict__ M, int row, MatRow& r) {
   const float4* r4 = reinterpret_cast<const float4*>(M + (size_t)row * 128);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) r.v[k] = __ldg(r4 + k);
+}
+
+// out[j] = dot(row, x[j][0..127]) for NV vectors in shared memory ([NV][128]).
+template <int NV>
+__device__ __forceinline__ void row_dots(const MatRow& r, const float* x, float (&out)[NV]) {
 #pragma unroll
   for (int j = 0; j < NV; ++j) out[j] = 0.f;
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    float4 t[16];
+  for (int k = 0; k < 32; ++k) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) t[k] = __ldg(r4 + 16 * b + k);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int d = 4 * (16 * b + k);
-#pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        const float4 xv = *reinterpret_cast<const float4*>(x + j * 128 + d);
-        out[j] = fmaf(t[k].x, xv.x, out[j]);
-        out[j] = fmaf(t[k].y, xv.y, out[j]);
-        out[j] = fmaf(t[k].z, xv.z, out[j]);
-        out[j] = fmaf(t[k].w, xv.w, out[j]);
-      }
+    for (int j = 0; j < NV; ++j) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + j * 128 + 4 * k);
+      out[j] = fmaf(r.v[k].x, xv.x, out[j]);
+      out[j] = fmaf(r.v[k].y, xv.y, out[j]);
+      out[j] = fmaf(r.v[k].z, xv.z, out[j]);
+      out[j] = fmaf(r.v[k].w, xv.w, out[j]);
     }
   }
 }

@@ -171,3 +171,39 @@ def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "f32":
         return np.asarray(x, np.float32)
     raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# Device-side draws for the workloads too large to generate on the host.
+# Same distributions (outlier channels are the host generator's), drawn with
+# torch's seeded CUDA generator; tests copy back the sampled units so that the
+# oracle reads exactly the values the library received.
+# ---------------------------------------------------------------------------
+
+def device_kv(w: Workload, layer: int, n: int, device="cuda", step: int | None = None,
+              dtype=None):
+    """(k, v) of all sequences: [B, n, Hkv, 128] tensors in the workload's
+    dtype (or `dtype`), drawn on `device`.  `step` selects an independent
+    stream (per decode step)."""
+    import torch
+    tdt = dtype or {"bf16": torch.bfloat16, "f16": torch.float16}[w.dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([w.wid, layer, _KEYS, -1 if step is None else step])
+                      .generate_state(1)[0]))
+    k = torch.randn((w.batch, n, w.n_kv_heads, HEAD_DIM), generator=g, device=device)
+    k *= torch.from_numpy(_key_scale(w, layer)).to(device)[None, None]
+    if w.values == "laplace":
+        u = torch.rand((w.batch, n, w.n_kv_heads, HEAD_DIM), generator=g, device=device) - 0.5
+        v = -torch.sign(u) * torch.log1p(-2.0 * u.abs().clamp_max(0.5 - 2.0 ** -25))
+    else:
+        v = torch.randn((w.batch, n, w.n_kv_heads, HEAD_DIM), generator=g, device=device)
+    return k.to(tdt), v.to(tdt)
+
+
+def device_queries(w: Workload, layer: int, step: int, device="cuda", dtype=None):
+    """[B, Hq, 128] decode queries drawn on `device`."""
+    import torch
+    tdt = dtype or {"bf16": torch.bfloat16, "f16": torch.float16}[w.dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([w.wid, layer, _QUERIES, step]).generate_state(1)[0]))
+    return torch.randn((w.batch, w.n_q_heads, HEAD_DIM), generator=g, device=device).to(tdt)
