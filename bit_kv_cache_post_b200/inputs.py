@@ -188,7 +188,7 @@ def device_kv(w: Workload, layer: int, n: int, device="cuda", step: int | None =
     import torch
     tdt = dtype or {"bf16": torch.bfloat16, "f16": torch.float16}[w.dtype]
     g = torch.Generator(device=device)
-    g.manual_seed(int(np.random.SeedSequence([w.wid, layer, _KEYS, -1 if step is None else step])
+    g.manual_seed(int(np.random.SeedSequence([w.wid, layer, _KEYS, 0 if step is None else step + 1])
                       .generate_state(1)[0]))
     k = torch.randn((w.batch, n, w.n_kv_heads, HEAD_DIM), generator=g, device=device)
     k *= torch.from_numpy(_key_scale(w, layer)).to(device)[None, None]
