@@ -376,6 +376,30 @@ def run_reference(args):
 BASELINE_METRIC = "2-bit KV decode-attention GB/s (% of HBM peak); KV append tokens/s"
 
 
+DECODE_SOURCES = ["bit_kv_cache_post_b200/csrc/decode.cu", "bit_kv_cache_post_b200/csrc/decode_frag.cuh",
+                  "bit_kv_cache_post_b200/csrc/async_copy.cuh",
+                  "bit_kv_cache_post_b200/csrc/wushkv_internal.cuh"]
+
+
+def decode_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, or None
+    when the decode kernel's sources changed since that capture."""
+    import hashlib
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "decode_kernel_qwen3-8b-layer-b16-ctx8192.md")).read()
+        rec = dict(line.split(": ", 1) for line in txt.splitlines()
+                   if line.startswith(("traffic_bytes_per_launch: ", "kernel_sources_sha256: ")))
+        h = hashlib.sha256()
+        for p in DECODE_SOURCES:
+            with open(os.path.join(ROOT, p), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["kernel_sources_sha256"].strip():
+            return None
+        return int(rec["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -430,7 +454,7 @@ def main():
         "decode_gbs": world * r["dec_total"] / (r["ms"] / 1e3) / 1e9,
         "append_tokens_per_s": w.batch * K / (float(np.sum(r["app_ms"])) / 1e3),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "decode",
+                     "frac": achieved / peak, "traffic": decode_traffic(), "kernel": "decode",
                      "peak_source": peak_src, "frac_of_8tbs": achieved / 8000.0,
                      "launch_ms": dec_avg_ms, "bytes_per_launch": r["dec_total"] / K},
         "e2e": {"value": world * e_dec / (e_ms / 1e3) / 1e9 if E else None,
