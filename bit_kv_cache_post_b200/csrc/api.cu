@@ -36,6 +36,10 @@ constexpr int MAX_GRID = 2048;
 // The unit-merging CTA stages the (m, l) of all partials of a unit in its
 // shared memory; at most this many partials per unit.
 constexpr int MAX_PARTS_PER_UNIT = 256;
+// Appends with at least this many tokens per unit going straight to the
+// packed cache take the tensor-core kernel (two 128-token tiles).
+constexpr int64_t TC_MIN_TOKENS = 256;
+constexpr int64_t TC_MIN_CTA_TILES = 6;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -346,7 +350,17 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
   const int64_t q_begin = first / 4, q_end = (n1 + 3) / 4;
   const int units = (int)((int64_t)c.batch * c.n_kv_heads);
 
-  auto launch = [&](int64_t qa, int64_t qb) -> cudaError_t {
+  // New tokens that go straight to the packed cache, whole quads from the
+  // first quad boundary at or after the first new token: on the tensor
+  // cores when the append is a bf16 block with a transform.
+  const int64_t pa = (int64_t)align_up((size_t)((n0 > S ? n0 : S) - S), 4), pb = P1;
+  const uintptr_t kv_addr = reinterpret_cast<uintptr_t>(k_rope_dev) | reinterpret_cast<uintptr_t>(v_dev);
+  const bool tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && pb - pa >= TC_MIN_TOKENS &&
+                  (kv_addr & 15) == 0 && (int64_t)c.batch * n_tok < 2147483647LL &&
+                  (c.quantizer == WUSHKV_QUEST_INT || (c.clip_lo_rank <= 2 && c.clip_hi_rank >= 127));
+  const int64_t tc_qa = tc ? (S + pa) / 4 : 0, tc_qb = tc ? (S + pb) / 4 : 0;
+
+  auto launch_one = [&](int64_t qa, int64_t qb) -> cudaError_t {
     if (qb <= qa) return cudaSuccess;
     a.quad_begin = qa;
     a.n_quads = qb - qa;
@@ -356,6 +370,13 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
     if (per > 64) per = 64;
     a.quads_per_cta = (int)per;
     return launch_append(a, s);
+  };
+  // the FMA kernel takes every quad outside the tensor-core range
+  auto launch = [&](int64_t qa, int64_t qb) -> cudaError_t {
+    if (!tc) return launch_one(qa, qb);
+    cudaError_t e1 = launch_one(qa, qb < tc_qa ? qb : tc_qa);
+    if (e1 != cudaSuccess) return e1;
+    return launch_one(qa > tc_qb ? qa : tc_qb, qb);
   };
 
   cudaError_t e;
@@ -367,6 +388,26 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
     if (e == cudaSuccess) e = launch(q_mid, q_end);
   } else {
     e = launch(q_begin, q_end);
+  }
+  if (e == cudaSuccess && tc) {
+    PrefillArgs pf;
+    std::memset(&pf, 0, sizeof(pf));
+    pf.c = a.c;
+    pf.T = T_k_dev;
+    pf.n_tok = n_tok;
+    pf.n0 = n0;
+    pf.pa = (int)pa;
+    pf.pb = (int)pb;
+    pf.tiles_per_unit = (int)((pb - pa + 127) / 128);
+    const int64_t head_tiles = (int64_t)c.batch * pf.tiles_per_unit;
+    // one CTA per SM shared among the heads, each CTA at least
+    // TC_MIN_CTA_TILES tiles (the T split into smem is paid once per CTA)
+    int64_t per_head = device_sms() / c.n_kv_heads;
+    const int64_t by_work = (head_tiles + TC_MIN_CTA_TILES - 1) / TC_MIN_CTA_TILES;
+    if (per_head > by_work) per_head = by_work;
+    if (per_head < 1) per_head = 1;
+    pf.ctas_per_head = (int)per_head;
+    e = launch_prefill_tc(pf, k_rope_dev, v_dev, device_sms(), s);
   }
   if (e != cudaSuccess) return WUSHKV_ECUDA;
   cache->n = n1;

@@ -277,6 +277,20 @@ struct AppendArgs {
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 
+// Bulk append on the tensor cores: the rows of packed indices [pa, pb) of
+// every unit come straight from the bf16 input (K through T).
+struct PrefillArgs {
+  DevCache c;
+  const float* T;          // [Hkv][128][128] fp32, 16-byte aligned
+  int n_tok;               // tokens per sequence in this append
+  int64_t n0;              // tokens before this append
+  int pa, pb;              // packed index range (multiples of 4)
+  int tiles_per_unit;      // ceil((pb - pa) / 128)
+  int ctas_per_head;       // CTAs sharing one KV head's tiles
+};
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const void* k, const void* v, int sms,
+                              cudaStream_t s);
+
 cudaError_t launch_query_transform(const void* q, int dtype, const float* TinvT, float* out,
                                    int batch, int n_q_heads, int n_kv_heads, cudaStream_t s);
 

@@ -96,3 +96,41 @@ def compare_cache_bitexact(cache, oc: O.OracleCache, units=None):
 def rel_rms_err(got: np.ndarray, want: np.ndarray) -> float:
     """max |got - want| / RMS(want)."""
     return float(np.abs(got - want).max() / math.sqrt(float(np.mean(want ** 2))))
+
+
+def check_unit_transformed(cache, oc: O.OracleCache, ou: int, T_h, k_h, u: int):
+    """Unit u of the GPU cache against unit ou of an oracle cache fed the
+    same rounded inputs, keys through T_h (k_h: that unit's post-RoPE keys).
+
+    Bar: fp16 key windows within 1e-3 relative error of the exact k'; key
+    codes mismatching on at most 1e-4 of elements (k' rounding-boundary
+    flips); key scales within one fp16 ulp (QuEST) or two (affine: two
+    independently rounded order statistics); value windows, codes and
+    scales bit-exact."""
+    ns, P, nr = oc.split()
+    bits = oc.cfg.bits
+    kt = np.asarray(k_h, np.float64) @ np.asarray(T_h, np.float64).T          # exact k'
+    ring = unit_window(cache, u, 0, "ring")[oc.recent_order()].astype(np.float64)
+    want = kt[ns + P:]
+    rel = np.linalg.norm(ring - want, axis=-1) / np.linalg.norm(want, axis=-1)
+    assert rel.max() <= 1e-3
+    sink = unit_window(cache, u, 0, "sink")[:ns].astype(np.float64)
+    rel = np.linalg.norm(sink - kt[:ns], axis=-1) / np.linalg.norm(kt[:ns], axis=-1)
+    assert rel.max() <= 1e-3
+    assert np.array_equal(unit_window(cache, u, 1, "ring")[oc.recent_order()].view(np.uint16),
+                          oc.ring_v[ou, oc.recent_order()].view(np.uint16))
+    assert np.array_equal(unit_window(cache, u, 1, "sink")[:ns].view(np.uint16),
+                          oc.sink_v[ou, :ns].view(np.uint16))
+    kc = O.unpack_k_rows(unit_packed_planes(cache, u, 0, P), bits)
+    mism = float(np.mean(kc != oc.codes_k[ou, :P]))
+    assert mism <= 1e-4, mism
+    for p_, q_ in zip(unit_packed_planes(cache, u, 1, P), oc.packed_v(ou)):
+        assert np.array_equal(p_, q_)
+    gm = unit_meta(cache, u, 0, P).astype(np.float32)
+    om = oc.meta_k[ou, :P, :gm.shape[1]].astype(np.float32)
+    ulp = np.spacing(np.abs(om).astype(np.float16)).astype(np.float32)
+    n_ulp = 1 if oc.cfg.quantizer == O.QUEST_INT else 2
+    assert np.all(np.abs(gm - om) <= n_ulp * ulp)
+    assert np.array_equal(unit_meta(cache, u, 1, P).view(np.uint16),
+                          oc.meta_v[ou, :P, :gm.shape[1]].view(np.uint16))
+    return mism

@@ -26,40 +26,6 @@ def wk():
     return wushkv
 
 
-def _check_unit(cache, oc, T_h, k_h, u):
-    """Compare one unit of the GPU cache with a single-unit oracle cache
-    built from the same rounded inputs (k_h: its post-RoPE keys, float)."""
-    ns, P, nr = oc.split()
-    bits = oc.cfg.bits
-    kt = k_h.astype(np.float64) @ T_h.astype(np.float64).T          # exact k'
-    ring = H.unit_window(cache, u, 0, "ring")[oc.recent_order()].astype(np.float64)
-    want = kt[ns + P:]
-    rel = np.linalg.norm(ring - want, axis=-1) / np.linalg.norm(want, axis=-1)
-    assert rel.max() <= 1e-3
-    sink = H.unit_window(cache, u, 0, "sink")[:ns].astype(np.float64)
-    rel = np.linalg.norm(sink - kt[:ns], axis=-1) / np.linalg.norm(kt[:ns], axis=-1)
-    assert rel.max() <= 1e-3
-    # value windows bit-exact
-    assert np.array_equal(H.unit_window(cache, u, 1, "ring")[oc.recent_order()].view(np.uint16),
-                          oc.ring_v[0, oc.recent_order()].view(np.uint16))
-    # packed codes and scales
-    kc = O.unpack_k_rows(H.unit_packed_planes(cache, u, 0, P), bits)
-    mism = np.mean(kc != oc.codes_k[0, :P])
-    assert mism <= 1e-4, mism
-    vplanes = H.unit_packed_planes(cache, u, 1, P)
-    for p_, q_ in zip(vplanes, oc.packed_v(0)):
-        assert np.array_equal(p_, q_)
-    gm = H.unit_meta(cache, u, 0, P).astype(np.float32)
-    om = oc.meta_k[0, :P, :gm.shape[1]].astype(np.float32)
-    ulp = np.spacing(np.abs(om).astype(np.float16)).astype(np.float32)
-    # QuEST: delta from a float64 RMS, one ulp; affine: (hi - lo) / 3 of two
-    # independently rounded order statistics, two ulps
-    n_ulp = 1 if oc.cfg.quantizer == O.QUEST_INT else 2
-    assert np.all(np.abs(gm - om) <= n_ulp * ulp)
-    assert np.array_equal(H.unit_meta(cache, u, 1, P).view(np.uint16),
-                          oc.meta_v[0, :P, :gm.shape[1]].view(np.uint16))
-
-
 def _oracle_unit(w, bits, quantizer, k_h, v_h, T_h, max_ctx):
     oc = O.OracleCache(O.CacheConfig(1, 1, w.group, max_ctx, bits=bits, quantizer=quantizer,
                                      sink=w.sink, recent=w.recent, chunk=w.chunk,
@@ -105,7 +71,7 @@ def test_qwen3_8b_layer_decode_step(wk, qwen8b_inputs, bits):
         v_h = np.concatenate([v[b, :, h], vs[b, :, h]])
         oc = _oracle_unit(w, bits, O.QUEST_INT, k_h, v_h, T[h], w.context + 8)
         assert oc.split() == cache.tokens()[1:]
-        _check_unit(cache, oc, T[h], k_h, u)
+        H.check_unit_transformed(cache, oc, 0, T[h], k_h, u)
         qprime = O.transform_query(qs[b, h * G:(h + 1) * G], TinvT[h].astype(np.float64))
         want = oc.decode(qprime[None])[0]
         assert H.rel_rms_err(out[b, h * G:(h + 1) * G], want) <= DECODE_TOL
@@ -138,7 +104,7 @@ def _device_workload(wk, w, bits, quantizer, n_prefill, n_step, samples):
         v_h = torch.cat([v[b, :, h], vs[b, :, h]]).float().cpu().numpy()
         oc = _oracle_unit(w, bits, quantizer, k_h, v_h, T[h], max_ctx)
         assert oc.split() == cache.tokens()[1:]
-        _check_unit(cache, oc, T[h], k_h, u)
+        H.check_unit_transformed(cache, oc, 0, T[h], k_h, u)
         qh = q[b, h * G:(h + 1) * G].float().cpu().numpy()
         want = oc.decode(O.transform_query(qh, TinvT[h].astype(np.float64))[None])[0]
         assert H.rel_rms_err(out[b, h * G:(h + 1) * G], want) <= DECODE_TOL
