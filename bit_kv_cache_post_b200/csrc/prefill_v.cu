@@ -1,0 +1,120 @@
+// Bulk (prefill) append of values: the value rows of one append that go
+// straight from the input to the packed cache (the packed index range of
+// the tensor-core key kernel).
+//
+// Method source: summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化"
+// (ai-papers-daily), sections 工作参考价值 and 方法关键点: values need no
+// transform (T_V is folded into W_V / W_O); every token vector leaving the
+// fp16 recent window is quantised per token and bit-packed.
+//
+// A warp takes one quad of 4 tokens x 8 consecutive KV heads of one
+// sequence: lane = 8 * token + head, so the warp's 32 rows are contiguous in
+// the [B][n_tok][Hkv][128] input (8 KB when Hkv = 8) and the four tokens of a
+// quad are lanes 8 apart.  Each lane loads its 256-byte row, rounds it to
+// fp16, takes the per-token quantiser parameters and builds its bytes of the
+// quad words, which byte transposes among the quad's lanes complete.
+#include "wushkv_internal.cuh"
+#include "quant_row.cuh"
+
+namespace wushkv {
+
+namespace {
+
+using namespace rowq;
+
+constexpr int VP_WARPS = 4;
+
+template <int BITS, bool AFFINE>
+__global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const PrefillArgs a,
+                                                                   const __nv_bfloat16* v,
+                                                                   int64_t n_items, int quads) {
+  const DevCache& c = a.c;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * VP_WARPS + warp;
+  if (item >= n_items) return;                       // uniform per warp
+  const int Hkv = c.n_kv_heads;
+  const int n_hg = (Hkv + 7) >> 3;
+  const int hg = (int)(item % n_hg);
+  const int64_t rest = item / n_hg;
+  const int qi = (int)(rest % quads);
+  const int b = (int)(rest / quads);
+  const int beta = lane >> 3, h = hg * 8 + (lane & 7);
+  const bool valid = h < Hkv;
+  const int pk = a.pa + 4 * qi + beta;
+  const int64_t tok = (int64_t)c.sink + pk - a.n0;   // token index within this append
+
+  __half2 xh[64];
+  {
+    uint4 raw[16];
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          v + (((int64_t)b * a.n_tok + tok) * Hkv + h) * D);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) raw[i] = __ldg(src + i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      xh[4 * i] = bf16x2_to_h2(raw[i].x);
+      xh[4 * i + 1] = bf16x2_to_h2(raw[i].y);
+      xh[4 * i + 2] = bf16x2_to_h2(raw[i].z);
+      xh[4 * i + 3] = bf16x2_to_h2(raw[i].w);
+    }
+  }
+  QParams q;
+  if constexpr (AFFINE) {
+    AffineStats st;
+    st.init();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) st.add2(xh[2 * e], xh[2 * e + 1]);
+    affine_finish(st, BITS, c.r_lo == 2, c.r_hi == 127, q);
+  } else {
+    QuestStats st;
+    st.init();
+#pragma unroll
+    for (int e = 0; e < 64; ++e) st.add(xh[e]);
+    quest_finish(st, BITS, c.alpha, q);
+  }
+  constexpr int W0 = BITS == 3 ? 2 : BITS;
+  const int u = b * Hkv + h;
+  const int quad = pk >> 2;
+  emit_v_quad<BITS, AFFINE, 8>(
+      xh, q, beta, quad, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + (size_t)quad * 64 * W0,
+      BITS == 3 ? c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + (size_t)quad * 64 : nullptr,
+      valid);
+  if (valid) {
+    uint8_t* meta = c.v_meta + (size_t)u * c.meta_unit_stride + (size_t)pk * c.meta_bytes;
+    if constexpr (AFFINE) *reinterpret_cast<uint32_t*>(meta) = q.meta;
+    else *reinterpret_cast<uint16_t*>(meta) = (uint16_t)q.meta;
+  }
+}
+
+template <int BITS, bool AFFINE>
+cudaError_t launch_vt(const PrefillArgs& a, const void* v, int64_t n_items, int quads,
+                      cudaStream_t s) {
+  const int64_t blocks = (n_items + VP_WARPS - 1) / VP_WARPS;
+  value_pack_kernel<BITS, AFFINE><<<(unsigned)blocks, VP_WARPS * 32, 0, s>>>(
+      a, static_cast<const __nv_bfloat16*>(v), n_items, quads);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_value_pack(const PrefillArgs& a, const void* v, int sms, cudaStream_t s) {
+  (void)sms;
+  const int B = a.c.units / a.c.n_kv_heads;
+  const int quads = (a.pb - a.pa) / 4;
+  const int64_t n_items = (int64_t)B * quads * ((a.c.n_kv_heads + 7) / 8);
+  if (n_items <= 0) return cudaSuccess;
+  const bool aff = a.c.quantizer == WUSHKV_AFFINE_PCTCLIP;
+  switch (a.c.bits) {
+    case 2: return aff ? launch_vt<2, true>(a, v, n_items, quads, s) : launch_vt<2, false>(a, v, n_items, quads, s);
+    case 3: return aff ? launch_vt<3, true>(a, v, n_items, quads, s) : launch_vt<3, false>(a, v, n_items, quads, s);
+    case 4: return aff ? launch_vt<4, true>(a, v, n_items, quads, s) : launch_vt<4, false>(a, v, n_items, quads, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace wushkv

@@ -290,6 +290,8 @@ struct PrefillArgs {
 };
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const void* k, const void* v, int sms,
                               cudaStream_t s);
+// The value rows of the same packed index range (called by launch_prefill_tc).
+cudaError_t launch_value_pack(const PrefillArgs& a, const void* v, int sms, cudaStream_t s);
 
 cudaError_t launch_query_transform(const void* q, int dtype, const float* TinvT, float* out,
                                    int batch, int n_q_heads, int n_kv_heads, cudaStream_t s);
