@@ -36,8 +36,8 @@ constexpr int MAX_GRID = 2048;
 // The unit-merging CTA stages the (m, l) of all partials of a unit in its
 // shared memory; at most this many partials per unit.
 constexpr int MAX_PARTS_PER_UNIT = 256;
-// Appends with at least this many tokens per unit going straight to the
-// packed cache take the tensor-core kernel (two 128-token tiles).
+// Appends with at least this many new tokens per unit (from the first
+// quad boundary) take the tensor-core kernel (two 128-token tiles).
 constexpr int64_t TC_MIN_TOKENS = 256;
 constexpr int64_t TC_MIN_CTA_TILES = 6;
 
@@ -350,15 +350,15 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
   const int64_t q_begin = first / 4, q_end = (n1 + 3) / 4;
   const int units = (int)((int64_t)c.batch * c.n_kv_heads);
 
-  // New tokens that go straight to the packed cache, whole quads from the
-  // first quad boundary at or after the first new token: on the tensor
-  // cores when the append is a bf16 block with a transform.
-  const int64_t pa = (int64_t)align_up((size_t)((n0 > S ? n0 : S) - S), 4), pb = P1;
+  // A bf16 block with a transform goes to the tensor-core key kernel and the
+  // value kernel from the first quad boundary at or after n0 to the end;
+  // the FMA kernel keeps the flush of old ring rows and the partial quad.
+  const int64_t ta = (n0 + 3) / 4 * 4;
   const uintptr_t kv_addr = reinterpret_cast<uintptr_t>(k_rope_dev) | reinterpret_cast<uintptr_t>(v_dev);
-  const bool tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && pb - pa >= TC_MIN_TOKENS &&
+  const bool tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && n1 - ta >= TC_MIN_TOKENS &&
                   (kv_addr & 15) == 0 && (int64_t)c.batch * n_tok < 2147483647LL &&
                   (c.quantizer == WUSHKV_QUEST_INT || (c.clip_lo_rank <= 2 && c.clip_hi_rank >= 127));
-  const int64_t tc_qa = tc ? (S + pa) / 4 : 0, tc_qb = tc ? (S + pb) / 4 : 0;
+  const int64_t tc_qa = tc ? ta / 4 : 0;
 
   auto launch_one = [&](int64_t qa, int64_t qb) -> cudaError_t {
     if (qb <= qa) return cudaSuccess;
@@ -371,12 +371,9 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
     a.quads_per_cta = (int)per;
     return launch_append(a, s);
   };
-  // the FMA kernel takes every quad outside the tensor-core range
+  // the FMA kernel takes every quad before the tensor-core range
   auto launch = [&](int64_t qa, int64_t qb) -> cudaError_t {
-    if (!tc) return launch_one(qa, qb);
-    cudaError_t e1 = launch_one(qa, qb < tc_qa ? qb : tc_qa);
-    if (e1 != cudaSuccess) return e1;
-    return launch_one(qa > tc_qb ? qa : tc_qb, qb);
+    return launch_one(qa, tc && qb > tc_qa ? tc_qa : qb);
   };
 
   cudaError_t e;
@@ -396,9 +393,10 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
     pf.T = T_k_dev;
     pf.n_tok = n_tok;
     pf.n0 = n0;
-    pf.pa = (int)pa;
-    pf.pb = (int)pb;
-    pf.tiles_per_unit = (int)((pb - pa + 127) / 128);
+    pf.ta = (int)ta;
+    pf.tb = (int)n1;
+    pf.packed1 = (int)P1;
+    pf.tiles_per_unit = (int)((n1 - ta + 127) / 128);
     const int64_t head_tiles = (int64_t)c.batch * pf.tiles_per_unit;
     // one CTA per SM shared among the heads, each CTA at least
     // TC_MIN_CTA_TILES tiles (the T split into smem is paid once per CTA)

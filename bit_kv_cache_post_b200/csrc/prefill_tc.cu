@@ -5,10 +5,10 @@
 // the per-head transform after RoPE (K' = K T^T for a block of tokens), and
 // every token vector that leaves the fp16 recent window is quantised per
 // token (QuEST INT or percentile-clipped affine) and bit-packed.  This file
-// handles the key rows of one append that go straight from the input to the
-// packed cache; their value rows go through the value-pack kernel, and the
-// window rows, the flush of old ring rows and a partial first quad stay with
-// the FMA append kernel.
+// handles the key rows of one append from its first quad boundary on: each
+// goes to the fp16 sink, the packed cache or the fp16 recent ring by its
+// token index.  The value rows go through the value-pack kernel; the flush
+// of old ring rows and a partial first quad stay with the FMA append kernel.
 //
 // Design (one CTA per SM, 18 warps, all tiles of a CTA from one KV head):
 //   warp 0      TMA producer: 128-token bf16 K tiles (128-byte swizzle)
@@ -62,18 +62,18 @@ static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct TileInfo {
   int u;        // unit (sequence, KV head)
-  int pk0;      // packed index of the tile's first row
-  int nv;       // valid rows (multiple of 4)
-  int z;        // input row of the tile's first token: b * n_tok + token - n0
+  int t0;       // absolute token of the tile's first row
+  int nv;       // valid rows
+  int z;        // input row of the tile's first token: b * n_tok + t0 - n0
 };
 
 __device__ __forceinline__ TileInfo tile_info(const PrefillArgs& a, int h, int l) {
   const int b = l / a.tiles_per_unit, i = l - b * a.tiles_per_unit;
   TileInfo t;
   t.u = b * a.c.n_kv_heads + h;
-  t.pk0 = a.pa + TILE * i;
-  t.nv = min(TILE, a.pb - t.pk0);
-  t.z = b * a.n_tok + (int)((int64_t)a.c.sink + t.pk0 - a.n0);
+  t.t0 = a.ta + TILE * i;
+  t.nv = min(TILE, a.tb - t.t0);
+  t.z = b * a.n_tok + (int)(t.t0 - a.n0);
   return t;
 }
 
@@ -91,42 +91,54 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
   atomicOr(status, DEV_ERR_TIMEOUT);
 }
 
-// Key row of one token from its TMEM lane (packed format of wushkv.h): dim
-// d = 32 ks + 4 c + 16 h + beta goes to word c w + rho / (8/w), field
-// rho mod (8/w), byte beta, with rho = 4 h + ks.  Column block cc holds
-// ks = cc; the two codes of a pair (beta, beta + 1) share a word and a field
-// and are placed together with one byte permute.  Every lane must call.
+// Row modes of the epilogue
+enum : int { ROW_NONE = 0, ROW_PACKED = 1, ROW_FP16 = 2 };
+
+// Key row of one token from its TMEM lane.  ROW_FP16: the fp16 rounding of
+// K' goes to `win` (a sink or ring row).  ROW_PACKED (packed format of
+// wushkv.h): dim d = 32 ks + 4 c + 16 h + beta goes to word c w + rho / (8/w),
+// field rho mod (8/w), byte beta, with rho = 4 h + ks.  Column block cc
+// holds ks = cc; the two codes of a pair (beta, beta + 1) share a word and a
+// field and are placed together with one byte permute.  Every lane of the
+// warp must call (the TMEM loads are warp-wide).
 template <int BITS, bool AFFINE>
 __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_second,
-                                        bool hi_second, bool valid, uint8_t* row0, uint8_t* row1,
-                                        uint8_t* meta_p) {
+                                        bool hi_second, int mode, uint8_t* row0, uint8_t* row1,
+                                        uint8_t* meta_p, __half* win) {
   constexpr int L = 1 << BITS;
+  const bool packed = mode == ROW_PACKED;
   QParams q;
-  if constexpr (AFFINE) {
-    AffineStats st;
-    st.init();
+  if (__any_sync(FULL, packed)) {
+    if constexpr (AFFINE) {
+      AffineStats st;
+      st.init();
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(taddr + (uint32_t)(32 * cc), r);
-      tmem_wait_ld();
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(taddr + (uint32_t)(32 * cc), r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        st.add2(f32x2_to_h2(r[4 * e], r[4 * e + 1]), f32x2_to_h2(r[4 * e + 2], r[4 * e + 3]));
+        for (int e = 0; e < 8; ++e)
+          st.add2(f32x2_to_h2(r[4 * e], r[4 * e + 1]), f32x2_to_h2(r[4 * e + 2], r[4 * e + 3]));
+      }
+      affine_finish(st, BITS, lo_second, hi_second, q);
+    } else {
+      QuestStats st;
+      st.init();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(taddr + (uint32_t)(32 * cc), r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) st.add(f32x2_to_h2(r[2 * e], r[2 * e + 1]));
+      }
+      quest_finish(st, BITS, alpha, q);
     }
-    affine_finish(st, BITS, lo_second, hi_second, q);
   } else {
-    QuestStats st;
-    st.init();
-#pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(taddr + (uint32_t)(32 * cc), r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 16; ++e) st.add(f32x2_to_h2(r[2 * e], r[2 * e + 1]));
-    }
-    quest_finish(st, BITS, alpha, q);
+    q.neglo = q.inv = make_float2(0.f, 0.f);
+    q.lo2 = __float2half2_rn(0.f);
+    q.meta = 0u;
   }
 
   uint32_t w0[8], w1[4], t4[8];
@@ -139,6 +151,16 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
     uint32_t r[32];
     tmem_ld32(taddr + (uint32_t)(32 * cc), r);
     tmem_wait_ld();
+    if (mode == ROW_FP16) {
+      uint4* o = reinterpret_cast<uint4*>(win + 32 * cc);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const __half2 h0 = f32x2_to_h2(r[8 * v], r[8 * v + 1]), h1 = f32x2_to_h2(r[8 * v + 2], r[8 * v + 3]);
+        const __half2 h2 = f32x2_to_h2(r[8 * v + 4], r[8 * v + 5]), h3 = f32x2_to_h2(r[8 * v + 6], r[8 * v + 7]);
+        o[v] = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                          *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+      }
+    }
     const uint32_t m2 = 1u << (2 * cc), m4 = 1u << (4 * (cc & 1)), m1 = 1u << cc;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -159,7 +181,7 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
     if constexpr (BITS == 4) {
       // words 4 c + 2 h + cc / 2 are complete after the odd block
       if (cc & 1) {
-        if (valid) {
+        if (packed) {
           uint32_t* o = reinterpret_cast<uint32_t*>(row0);
 #pragma unroll
           for (int x = 0; x < 8; ++x) o[2 * x + (cc >> 1)] = t4[x];
@@ -169,7 +191,7 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
       }
     }
   }
-  if (!valid) return;
+  if (!packed) return;
   if constexpr (BITS != 4) {
     uint4* o0 = reinterpret_cast<uint4*>(row0);
     o0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
@@ -326,8 +348,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int j = g; j < nt; j += NGROUP) {
       const uint32_t use = (uint32_t)(j / NGROUP);
       const TileInfo t = tile_info(a, h, t_begin + j);
-      const bool valid = row < t.nv;
-      const int pk = t.pk0 + row;
+      // destination of this row by its token index
+      const int tok = t.t0 + row;
+      const int pk = tok - c.sink;
+      int mode = ROW_NONE;
+      __half* win = nullptr;
+      if (row < t.nv) {
+        if (tok < c.sink) {
+          mode = ROW_FP16;
+          win = c.sink_k + ((size_t)t.u * c.sink + tok) * D;
+        } else if (pk < a.packed1) {
+          mode = ROW_PACKED;
+        } else {
+          mode = ROW_FP16;
+          win = c.ring_k + ((size_t)t.u * c.ring_slots + (size_t)(pk % c.ring_slots)) * D;
+        }
+      }
+      const size_t pkc = mode == ROW_PACKED ? (size_t)pk : 0;
       const bool ok = wait_or_abort(&t_full[g], use & 1, abort_flag);
       if (!__all_sync(FULL, ok)) {
         raise_abort(abort_flag, c.status);
@@ -335,10 +372,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_after();
       key_row<BITS, AFFINE>(
-          taddr, c.alpha, lo_second, hi_second, valid,
-          c.k_plane[0] + (size_t)t.u * c.plane_unit_stride[0] + (size_t)pk * 16 * W0,
-          BITS == 3 ? c.k_plane[1] + (size_t)t.u * c.plane_unit_stride[1] + (size_t)pk * 16 : nullptr,
-          c.k_meta + (size_t)t.u * c.meta_unit_stride + (size_t)pk * c.meta_bytes);
+          taddr, c.alpha, lo_second, hi_second, mode,
+          c.k_plane[0] + (size_t)t.u * c.plane_unit_stride[0] + pkc * 16 * W0,
+          BITS == 3 ? c.k_plane[1] + (size_t)t.u * c.plane_unit_stride[1] + pkc * 16 : nullptr,
+          c.k_meta + (size_t)t.u * c.meta_unit_stride + pkc * c.meta_bytes, win);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[g]);

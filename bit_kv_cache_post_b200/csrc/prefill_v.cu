@@ -1,6 +1,6 @@
-// Bulk (prefill) append of values: the value rows of one append that go
-// straight from the input to the packed cache (the packed index range of
-// the tensor-core key kernel).
+// Bulk (prefill) append of values: the value rows of one append from its
+// first quad boundary on (the token range of the tensor-core key kernel),
+// each to the fp16 sink, the packed cache or the fp16 recent ring.
 //
 // Method source: summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化"
 // (ai-papers-daily), sections 工作参考价值 and 方法关键点: values need no
@@ -10,9 +10,11 @@
 // A warp takes one quad of 4 tokens x 8 consecutive KV heads of one
 // sequence: lane = 8 * token + head, so the warp's 32 rows are contiguous in
 // the [B][n_tok][Hkv][128] input (8 KB when Hkv = 8) and the four tokens of a
-// quad are lanes 8 apart.  Each lane loads its 256-byte row, rounds it to
-// fp16, takes the per-token quantiser parameters and builds its bytes of the
-// quad words, which byte transposes among the quad's lanes complete.
+// quad are lanes 8 apart.  Each lane loads its 256-byte row and rounds it to
+// fp16.  A quad inside the packed range (its boundaries are multiples of 4)
+// is quantised: per-token parameters, then each lane's bytes of the quad
+// words, completed by byte transposes among the quad's lanes; any other quad
+// stores its fp16 rows to the sink or the ring.
 #include "wushkv_internal.cuh"
 #include "quant_row.cuh"
 
@@ -39,10 +41,13 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
   const int qi = (int)(rest % quads);
   const int b = (int)(rest / quads);
   const int beta = lane >> 3, h = hg * 8 + (lane & 7);
-  const bool valid = h < Hkv;
-  const int pk = a.pa + 4 * qi + beta;
-  const int64_t tok = (int64_t)c.sink + pk - a.n0;   // token index within this append
-
+  const int tq = a.ta + 4 * qi;                      // absolute token of the quad
+  const int tok_abs = tq + beta;
+  const bool valid = h < Hkv && tok_abs < a.tb;
+  const int64_t tok = tok_abs - a.n0;                // token index within this append
+  const int pkq = tq - c.sink;
+  const bool packed_quad = tq >= c.sink && pkq < a.packed1;   // uniform per warp
+  const int pk = pkq + beta;
   __half2 xh[64];
   {
     uint4 raw[16];
@@ -63,6 +68,22 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
       xh[4 * i + 3] = bf16x2_to_h2(raw[i].w);
     }
   }
+  const int u = b * Hkv + h;
+  if (!packed_quad) {
+    if (valid) {
+      __half* dst = tok_abs < c.sink
+                        ? c.sink_v + ((size_t)u * c.sink + tok_abs) * D
+                        : c.ring_v + ((size_t)u * c.ring_slots + (size_t)(pk % c.ring_slots)) * D;
+      uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        o[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&xh[4 * i]),
+                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 1]),
+                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 2]),
+                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 3]));
+    }
+    return;
+  }
   QParams q;
   if constexpr (AFFINE) {
     AffineStats st;
@@ -78,8 +99,7 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
     quest_finish(st, BITS, c.alpha, q);
   }
   constexpr int W0 = BITS == 3 ? 2 : BITS;
-  const int u = b * Hkv + h;
-  const int quad = pk >> 2;
+  const int quad = pkq >> 2;
   emit_v_quad<BITS, AFFINE, 8>(
       xh, q, beta, quad, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + (size_t)quad * 64 * W0,
       BITS == 3 ? c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + (size_t)quad * 64 : nullptr,
@@ -105,7 +125,7 @@ cudaError_t launch_vt(const PrefillArgs& a, const void* v, int64_t n_items, int 
 cudaError_t launch_value_pack(const PrefillArgs& a, const void* v, int sms, cudaStream_t s) {
   (void)sms;
   const int B = a.c.units / a.c.n_kv_heads;
-  const int quads = (a.pb - a.pa) / 4;
+  const int quads = (a.tb - a.ta + 3) / 4;
   const int64_t n_items = (int64_t)B * quads * ((a.c.n_kv_heads + 7) / 8);
   if (n_items <= 0) return cudaSuccess;
   const bool aff = a.c.quantizer == WUSHKV_AFFINE_PCTCLIP;

@@ -277,15 +277,18 @@ struct AppendArgs {
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 
-// Bulk append on the tensor cores: the rows of packed indices [pa, pb) of
-// every unit come straight from the bf16 input (K through T).
+// Bulk append on the tensor cores: every token t in [ta, tb) of every unit
+// comes straight from the bf16 input (keys through T) and goes to the fp16
+// sink (t < sink), the packed cache (sink <= t < sink + packed1) or the
+// fp16 recent ring.
 struct PrefillArgs {
   DevCache c;
   const float* T;          // [Hkv][128][128] fp32, 16-byte aligned
   int n_tok;               // tokens per sequence in this append
   int64_t n0;              // tokens before this append
-  int pa, pb;              // packed index range (multiples of 4)
-  int tiles_per_unit;      // ceil((pb - pa) / 128)
+  int ta, tb;              // absolute token range (ta a multiple of 4, tb = n0 + n_tok)
+  int packed1;             // packed count after this append
+  int tiles_per_unit;      // ceil((tb - ta) / 128)
   int ctas_per_head;       // CTAs sharing one KV head's tiles
 };
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const void* k, const void* v, int sms,
