@@ -10,19 +10,24 @@
 // token index.  The value rows go through the value-pack kernel; the flush
 // of old ring rows and a partial first quad stay with the FMA append kernel.
 //
-// Design (one CTA per SM, 18 warps, all tiles of a CTA from one KV head):
+// Design (one CTA per SM, 20 warps, all tiles of a CTA from one KV head):
 //   warp 0      TMA producer: 128-token bf16 K tiles (128-byte swizzle)
 //               through a four-stage ring;
-//   warp 1      tensor-memory owner and MMA issuer: K' = K T_lo^T + K T_mid^T
-//               + K T_hi^T with T = T_hi + T_mid + T_lo split into three bf16
-//               matrices (T to about 2^-27 relative, so K' is as close to the
-//               exact product as an fp32 FMA loop), fp32 accumulation in four
-//               128-column TMEM accumulators;
-//   warps 2-17  four epilogue warpgroups taking every fourth tile; thread i
-//               owns token row i (TMEM lane i) and reads its 128 columns in
-//               four 32-column blocks twice: once for the per-token
-//               statistics, once for the codes, which are placed two at a
-//               time into the packed row words.
+//   warps 2-3   converters: each landed tile to fp16 in place (bf16 values
+//               inside the fp16 range are exact in fp16; below 2^-17 they
+//               round to the fp16 grid, an error far under the transform's);
+//   warp 1      tensor-memory owner and MMA issuer: K' 2^s = K T_lo^T +
+//               K T_hi^T with T 2^s = T_hi + T_lo split into two fp16
+//               matrices (s a per-head power of two putting max |T| 2^s in
+//               [2^13, 2^14), so T is kept to about 2^-22 relative, as close
+//               to the exact product as an fp32 FMA loop); fp32 accumulation
+//               in four 128-column TMEM accumulators;
+//   warps 4-19  four epilogue warpgroups taking every fourth tile; thread i
+//               owns token row i (TMEM lane i), scales it by 2^-s and reads
+//               its 128 columns twice: in two 64-column loads for the
+//               per-token statistics, in double-buffered 16-column halves
+//               for the codes, which are placed two at a time into the
+//               packed row words.
 // Every wait is bounded; on a timeout the CTA records DEV_ERR_TIMEOUT, stops
 // issuing, waits (bounded) for its own copies and MMAs, frees TMEM and ends.
 #include <cuda.h>
@@ -40,7 +45,8 @@ using namespace rowq;
 constexpr int TILE = 128;                    // tokens per tile (MMA M)
 constexpr int NSTAGE = 4;                    // K tiles in flight
 constexpr int NGROUP = 4;                    // epilogue warpgroups = TMEM accumulators
-constexpr int FIRST_EPI_WARP = 2;
+constexpr int CONV_WARP = 2;                 // two converter warps
+constexpr int FIRST_EPI_WARP = 4;
 constexpr int NTHREADS = (FIRST_EPI_WARP + 4 * NGROUP) * 32;
 constexpr int TMEM_COLS = NGROUP * D;        // 512
 constexpr int TILE_BYTES = TILE * D * 2;     // one bf16 tile, 32 KB
@@ -50,13 +56,12 @@ static_assert(NSTAGE == NGROUP, "tile j uses stage and accumulator j % 4");
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_THI = 0;
-constexpr int OFF_TMID = OFF_THI + TILE_BYTES;
-constexpr int OFF_TLO = OFF_TMID + TILE_BYTES;
+constexpr int OFF_TLO = OFF_THI + TILE_BYTES;
 constexpr int OFF_K = OFF_TLO + TILE_BYTES;
 constexpr int OFF_BAR = OFF_K + NSTAGE * TILE_BYTES;
-constexpr int N_BARS = 4 * NSTAGE + 1;
+constexpr int N_BARS = 5 * NSTAGE + 1;
 constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-constexpr int SMEM_USED = OFF_MISC + 16;
+constexpr int SMEM_USED = OFF_MISC + 16;   // tmem slot, abort flag, max |T|, 2^-s
 constexpr int SMEM_BYTES = SMEM_USED + 1024;          // slack for the alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -94,18 +99,76 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // Row modes of the epilogue
 enum : int { ROW_NONE = 0, ROW_PACKED = 1, ROW_FP16 = 2 };
 
+// fp16 values of two accumulator columns: K' = accumulator * 2^-s (exact).
+__device__ __forceinline__ __half2 kprime_h2(uint32_t a, uint32_t b, float2 unscale) {
+  const float2 v = mul2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), unscale);
+  return __floats2half2_rn(v.x, v.y);
+}
+
+// Codes of the 16-column half HB of column block cc (ks = cc, h = HB) into
+// the row's packed words; ROW_FP16 rows store the half's fp16 values instead.
+template <int BITS, bool AFFINE, int HB>
+__device__ __forceinline__ void key_half(const uint32_t (&r)[16], int cc, float2 unscale,
+                                         const QParams& q, int mode, __half* win,
+                                         uint32_t (&w0)[8], uint32_t (&w1)[4], uint32_t (&t4)[8],
+                                         uint8_t* row0) {
+  constexpr int L = 1 << BITS;
+  __half2 x[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = kprime_h2(r[2 * e], r[2 * e + 1], unscale);
+  if (mode == ROW_FP16) {
+    uint4* o = reinterpret_cast<uint4*>(win + 32 * cc + 16 * HB);
+#pragma unroll
+    for (int v = 0; v < 2; ++v)
+      o[v] = make_uint4(*reinterpret_cast<const uint32_t*>(&x[4 * v]),
+                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 1]),
+                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 2]),
+                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 3]));
+  }
+  const uint32_t m2 = 1u << (2 * cc), m4 = 1u << (4 * (cc & 1)), m1 = (1u << cc) << (4 * HB);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = 2 * e;                            // column in the half: 4 c + beta
+    const int cq = i >> 2, beta = i & 3;            // beta in {0, 2}
+    const uint2 p = code_pat2<AFFINE, L>(x[e], q);
+    // codes to bytes beta, beta + 1; byte 1 of a pattern is zero
+    const uint32_t placed = __byte_perm(p.x, p.y, beta == 0 ? 0x1140u : 0x4011u);
+    if constexpr (BITS == 2) {
+      w0[2 * cq + HB] += placed * m2;
+    } else if constexpr (BITS == 3) {
+      w0[2 * cq + HB] += (placed & 0x03030303u) * m2;
+      w1[cq] += ((placed >> 2) & 0x01010101u) * m1;
+    } else {
+      t4[2 * cq + HB] += placed * m4;
+    }
+  }
+  if constexpr (BITS == 4 && HB == 1) {
+    // words 4 c + 2 h + cc / 2 are complete after the odd block
+    if (cc & 1) {
+      if (mode == ROW_PACKED) {
+        uint32_t* o = reinterpret_cast<uint32_t*>(row0);
+#pragma unroll
+        for (int xw = 0; xw < 8; ++xw) o[2 * xw + (cc >> 1)] = t4[xw];
+      }
+#pragma unroll
+      for (int xw = 0; xw < 8; ++xw) t4[xw] = 0u;
+    }
+  }
+}
+
 // Key row of one token from its TMEM lane.  ROW_FP16: the fp16 rounding of
 // K' goes to `win` (a sink or ring row).  ROW_PACKED (packed format of
 // wushkv.h): dim d = 32 ks + 4 c + 16 h + beta goes to word c w + rho / (8/w),
 // field rho mod (8/w), byte beta, with rho = 4 h + ks.  Column block cc
 // holds ks = cc; the two codes of a pair (beta, beta + 1) share a word and a
-// field and are placed together with one byte permute.  Every lane of the
+// field and are placed together with one byte permute.  The statistics read
+// the lane in two 64-column loads; the codes read it in 16-column halves,
+// each load issued while the previous half is processed.  Every lane of the
 // warp must call (the TMEM loads are warp-wide).
 template <int BITS, bool AFFINE>
-__device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_second,
-                                        bool hi_second, int mode, uint8_t* row0, uint8_t* row1,
-                                        uint8_t* meta_p, __half* win) {
-  constexpr int L = 1 << BITS;
+__device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double alpha,
+                                        bool lo_second, bool hi_second, int mode, uint8_t* row0,
+                                        uint8_t* row1, uint8_t* meta_p, __half* win) {
   const bool packed = mode == ROW_PACKED;
   QParams q;
   if (__any_sync(FULL, packed)) {
@@ -113,25 +176,26 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
       AffineStats st;
       st.init();
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(taddr + (uint32_t)(32 * cc), r);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(taddr + (uint32_t)(64 * hf), r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          st.add2(f32x2_to_h2(r[4 * e], r[4 * e + 1]), f32x2_to_h2(r[4 * e + 2], r[4 * e + 3]));
+        for (int e = 0; e < 16; ++e)
+          st.add2(kprime_h2(r[4 * e], r[4 * e + 1], unscale),
+                  kprime_h2(r[4 * e + 2], r[4 * e + 3], unscale));
       }
       affine_finish(st, BITS, lo_second, hi_second, q);
     } else {
       QuestStats st;
       st.init();
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(taddr + (uint32_t)(32 * cc), r);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r[64];
+        tmem_ld64(taddr + (uint32_t)(64 * hf), r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) st.add(f32x2_to_h2(r[2 * e], r[2 * e + 1]));
+        for (int e = 0; e < 32; ++e) st.add(kprime_h2(r[2 * e], r[2 * e + 1], unscale));
       }
       quest_finish(st, BITS, alpha, q);
     }
@@ -146,50 +210,16 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
   for (int i = 0; i < 8; ++i) w0[i] = t4[i] = 0u;
 #pragma unroll
   for (int i = 0; i < 4; ++i) w1[i] = 0u;
+  uint32_t ra[16], rb[16];
+  tmem_ld16(taddr, ra);
 #pragma unroll 1
   for (int cc = 0; cc < 4; ++cc) {
-    uint32_t r[32];
-    tmem_ld32(taddr + (uint32_t)(32 * cc), r);
-    tmem_wait_ld();
-    if (mode == ROW_FP16) {
-      uint4* o = reinterpret_cast<uint4*>(win + 32 * cc);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const __half2 h0 = f32x2_to_h2(r[8 * v], r[8 * v + 1]), h1 = f32x2_to_h2(r[8 * v + 2], r[8 * v + 3]);
-        const __half2 h2 = f32x2_to_h2(r[8 * v + 4], r[8 * v + 5]), h3 = f32x2_to_h2(r[8 * v + 6], r[8 * v + 7]);
-        o[v] = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
-                          *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
-      }
-    }
-    const uint32_t m2 = 1u << (2 * cc), m4 = 1u << (4 * (cc & 1)), m1 = 1u << cc;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int i = 2 * e;
-      const int hh = i >> 4, cq = (i >> 2) & 3, beta = i & 3;   // beta in {0, 2}
-      const uint2 p = code_pat2<AFFINE, L>(f32x2_to_h2(r[i], r[i + 1]), q);
-      // codes to bytes beta, beta + 1; byte 1 of a pattern is zero
-      const uint32_t placed = __byte_perm(p.x, p.y, beta == 0 ? 0x1140u : 0x4011u);
-      if constexpr (BITS == 2) {
-        w0[2 * cq + hh] += placed * m2;
-      } else if constexpr (BITS == 3) {
-        w0[2 * cq + hh] += (placed & 0x03030303u) * m2;
-        w1[cq] += ((placed >> 2) & 0x01010101u) * (m1 << (4 * hh));
-      } else {
-        t4[2 * cq + hh] += placed * m4;
-      }
-    }
-    if constexpr (BITS == 4) {
-      // words 4 c + 2 h + cc / 2 are complete after the odd block
-      if (cc & 1) {
-        if (packed) {
-          uint32_t* o = reinterpret_cast<uint32_t*>(row0);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) o[2 * x + (cc >> 1)] = t4[x];
-        }
-#pragma unroll
-        for (int x = 0; x < 8; ++x) t4[x] = 0u;
-      }
-    }
+    tmem_wait_ld();                                          // half 0 of block cc in ra
+    tmem_ld16(taddr + (uint32_t)(32 * cc + 16), rb);
+    key_half<BITS, AFFINE, 0>(ra, cc, unscale, q, mode, win, w0, w1, t4, row0);
+    tmem_wait_ld();                                          // half 1 of block cc in rb
+    if (cc < 3) tmem_ld16(taddr + (uint32_t)(32 * cc + 32), ra);
+    key_half<BITS, AFFINE, 1>(rb, cc, unscale, q, mode, win, w0, w1, t4, row0);
   }
   if (!packed) return;
   if constexpr (BITS != 4) {
@@ -202,6 +232,20 @@ __device__ __forceinline__ void key_row(uint32_t taddr, double alpha, bool lo_se
   else *reinterpret_cast<uint16_t*>(meta_p) = (uint16_t)q.meta;
 }
 
+// In-place bf16 -> fp16 of one 16 KB half of a K tile (rows of 64 dims, any
+// swizzle: element-wise) by one warp.
+__device__ __forceinline__ void convert_half_tile(unsigned char* base, int lane) {
+  uint4* p = reinterpret_cast<uint4*>(base);
+#pragma unroll 4
+  for (int i = lane; i < HALF_BYTES / 16; i += 32) {
+    const uint4 w = p[i];
+    const __half2 a = bf16x2_to_h2(w.x), b = bf16x2_to_h2(w.y);
+    const __half2 c2 = bf16x2_to_h2(w.z), d = bf16x2_to_h2(w.w);
+    p[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b),
+                      *reinterpret_cast<const uint32_t*>(&c2), *reinterpret_cast<const uint32_t*>(&d));
+  }
+}
+
 template <int BITS, bool AFFINE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmk) {
@@ -209,13 +253,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* k_full = bars;                    // [NSTAGE] tile landed
-  uint64_t* k_empty = bars + NSTAGE;          // [NSTAGE] tile consumed by the MMAs
-  uint64_t* t_full = bars + 2 * NSTAGE;       // [NGROUP] accumulator ready
-  uint64_t* t_empty = bars + 3 * NSTAGE;      // [NGROUP] accumulator drained
-  uint64_t* drain = bars + 4 * NSTAGE;
+  uint64_t* k_full = bars;                    // [NSTAGE] bf16 tile landed
+  uint64_t* k_conv = bars + NSTAGE;           // [NSTAGE] tile converted to fp16
+  uint64_t* k_empty = bars + 2 * NSTAGE;      // [NSTAGE] tile consumed by the MMAs
+  uint64_t* t_full = bars + 3 * NSTAGE;       // [NGROUP] accumulator ready
+  uint64_t* t_empty = bars + 4 * NSTAGE;      // [NGROUP] accumulator drained
+  uint64_t* drain = bars + 5 * NSTAGE;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  unsigned int* tmax_bits = reinterpret_cast<unsigned int*>(sm + OFF_MISC + 8);
 
   const DevCache& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -226,39 +272,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int nt = t_end - t_begin;
   if (nt <= 0) return;
 
-  // ---- setup: T split into bf16 hi + mid + lo, swizzled K-major ------------
+  // ---- setup: T 2^s = T_hi + T_lo in fp16, swizzled K-major ----------------
+  const float4* T4 = reinterpret_cast<const float4*>(a.T + (size_t)h * D * D);
+  if (tid == 0) *tmax_bits = 0u;
+  __syncthreads();
   {
-    const float4* T4 = reinterpret_cast<const float4*>(a.T + (size_t)h * D * D);
+    float m = 0.f;
     for (int qd = tid; qd < D * D / 4; qd += NTHREADS) {
-      const int i = qd >> 5, j0 = (qd & 31) * 4;
       const float4 v = __ldg(T4 + qd);
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-      uint32_t part[3][2];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // each remainder is exact in fp32 (the difference of a float and
-        // its bf16 rounding)
-        const __nv_bfloat16 b0 = __float2bfloat16_rn(vv[e]);
-        const float r1 = vv[e] - __bfloat162float(b0);
-        const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
-        const __nv_bfloat16 b2 = __float2bfloat16_rn(r1 - __bfloat162float(b1));
-        const uint32_t sh = 16u * (e & 1);
-        if ((e & 1) == 0) part[0][e >> 1] = part[1][e >> 1] = part[2][e >> 1] = 0u;
-        part[0][e >> 1] |= (uint32_t)__bfloat16_as_ushort(b0) << sh;
-        part[1][e >> 1] |= (uint32_t)__bfloat16_as_ushort(b1) << sh;
-        part[2][e >> 1] |= (uint32_t)__bfloat16_as_ushort(b2) << sh;
-      }
-      const int off = (j0 >> 6) * HALF_BYTES + i * 128 + ((((j0 & 63) >> 3) ^ (i & 7)) << 4) +
-                      (j0 & 7) * 2;
-      *reinterpret_cast<uint2*>(sm + OFF_THI + off) = make_uint2(part[0][0], part[0][1]);
-      *reinterpret_cast<uint2*>(sm + OFF_TMID + off) = make_uint2(part[1][0], part[1][1]);
-      *reinterpret_cast<uint2*>(sm + OFF_TLO + off) = make_uint2(part[2][0], part[2][1]);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
-    fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
+    m = warp_max_f32(m);
+    if (lane == 0) atomicMax(tmax_bits, __float_as_uint(m));   // non-negative: bits order as values
   }
+  __syncthreads();
+  // 2^s with max |T| 2^s in [2^13, 2^14)
+  int s_exp = 0;
+  {
+    const float tmax = __uint_as_float(*tmax_bits);
+    if (tmax > 0.f && isfinite(tmax)) {
+      int e;
+      frexpf(tmax, &e);                      // tmax = f 2^e, f in [0.5, 1)
+      s_exp = min(max(14 - e, -100), 100);   // a near-zero T keeps a finite scale
+    }
+  }
+  const float scale = ldexpf(1.f, s_exp);
+  const float2 unscale = make_float2(ldexpf(1.f, -s_exp), ldexpf(1.f, -s_exp));
+  for (int qd = tid; qd < D * D / 4; qd += NTHREADS) {
+    const int i = qd >> 5, j0 = (qd & 31) * 4;
+    const float4 v = __ldg(T4 + qd);
+    const float vv[4] = {v.x * scale, v.y * scale, v.z * scale, v.w * scale};   // exact
+    uint32_t part[2][2];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // the remainder is exact in fp32 (a float minus its fp16 rounding)
+      const __half b0 = __float2half_rn(vv[e]);
+      const __half b1 = __float2half_rn(vv[e] - __half2float(b0));
+      const uint32_t sh = 16u * (e & 1);
+      if ((e & 1) == 0) part[0][e >> 1] = part[1][e >> 1] = 0u;
+      part[0][e >> 1] |= (uint32_t)__half_as_ushort(b0) << sh;
+      part[1][e >> 1] |= (uint32_t)__half_as_ushort(b1) << sh;
+    }
+    const int off = (j0 >> 6) * HALF_BYTES + i * 128 + ((((j0 & 63) >> 3) ^ (i & 7)) << 4) +
+                    (j0 & 7) * 2;
+    *reinterpret_cast<uint2*>(sm + OFF_THI + off) = make_uint2(part[0][0], part[0][1]);
+    *reinterpret_cast<uint2*>(sm + OFF_TLO + off) = make_uint2(part[1][0], part[1][1]);
+  }
+  fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_conv[s], 2);
       mbar_init(&k_empty[s], 1);
       mbar_init(&t_full[s], 1);
       mbar_init(&t_empty[s], 4);
@@ -303,14 +367,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     // ---- MMA issuer -------------------------------------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(true, TILE, D);
-      // smallest terms first
-      const uint32_t tpart[3] = {smem_addr(sm + OFF_TLO), smem_addr(sm + OFF_TMID),
-                                 smem_addr(sm + OFF_THI)};
+      constexpr uint32_t idesc = idesc_f16(false, TILE, D);   // fp16 x fp16 -> fp32
+      const uint32_t tpart[2] = {smem_addr(sm + OFF_TLO), smem_addr(sm + OFF_THI)};  // small first
       for (int j = 0; j < nt; ++j) {
         const int s = j % NSTAGE;
         const uint32_t use = (uint32_t)(j / NSTAGE);
-        if (!wait_or_abort(&k_full[s], use & 1, abort_flag)) {
+        if (!wait_or_abort(&k_conv[s], use & 1, abort_flag)) {
           raise_abort(abort_flag, c.status);
           break;
         }
@@ -322,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t ka = smem_addr(sm + OFF_K + s * TILE_BYTES);
         const uint32_t dt = tmem_base + (uint32_t)(s * D);
 #pragma unroll
-        for (int tp = 0; tp < 3; ++tp)
+        for (int tp = 0; tp < 2; ++tp)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
@@ -337,6 +399,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait_bounded(drain, 0, PF_WAIT_POLLS);
     }
     __syncwarp();
+  } else if (warp < FIRST_EPI_WARP) {
+    // ---- converters: bf16 -> fp16 in place, one 64-dim half each --------------
+    const int half = warp - CONV_WARP;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % NSTAGE;
+      const uint32_t use = (uint32_t)(j / NSTAGE);
+      const bool ok = wait_or_abort(&k_full[s], use & 1, abort_flag);
+      if (!__all_sync(FULL, ok)) {
+        raise_abort(abort_flag, c.status);
+        break;
+      }
+      convert_half_tile(sm + OFF_K + s * TILE_BYTES + half * HALF_BYTES, lane);
+      fence_proxy_async();                   // generic writes -> the tensor core's reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&k_conv[s]);
+    }
   } else {
     // ---- epilogue warpgroups ------------------------------------------------------
     const int g = (warp - FIRST_EPI_WARP) >> 2;
@@ -372,7 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_after();
       key_row<BITS, AFFINE>(
-          taddr, c.alpha, lo_second, hi_second, mode,
+          taddr, unscale, c.alpha, lo_second, hi_second, mode,
           c.k_plane[0] + (size_t)t.u * c.plane_unit_stride[0] + pkc * 16 * W0,
           BITS == 3 ? c.k_plane[1] + (size_t)t.u * c.plane_unit_stride[1] + pkc * 16 : nullptr,
           c.k_meta + (size_t)t.u * c.meta_unit_stride + pkc * c.meta_bytes, win);

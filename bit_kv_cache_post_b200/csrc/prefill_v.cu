@@ -7,14 +7,15 @@
 // transform (T_V is folded into W_V / W_O); every token vector leaving the
 // fp16 recent window is quantised per token and bit-packed.
 //
-// A warp takes one quad of 4 tokens x 8 consecutive KV heads of one
-// sequence: lane = 8 * token + head, so the warp's 32 rows are contiguous in
-// the [B][n_tok][Hkv][128] input (8 KB when Hkv = 8) and the four tokens of a
-// quad are lanes 8 apart.  Each lane loads its 256-byte row and rounds it to
-// fp16.  A quad inside the packed range (its boundaries are multiples of 4)
-// is quantised: per-token parameters, then each lane's bytes of the quad
-// words, completed by byte transposes among the quad's lanes; any other quad
-// stores its fp16 rows to the sink or the ring.
+// A warp takes one quad of 4 tokens x 4 consecutive KV heads of one
+// sequence, two lanes per row: lane = 8 * token + 2 * head + half, each lane
+// holding 64 of the 128 dims (so the four tokens of a quad are lanes 8
+// apart and the warp's rows are 1 KB runs of the [B][n_tok][Hkv][128]
+// input).  Each lane loads its half row and rounds it to fp16.  A quad
+// inside the packed range (its boundaries are multiples of 4) is quantised:
+// per-token parameters merged across the row's two lanes, then each lane's
+// bytes of its half of the quad words, completed by byte transposes among
+// the quad's lanes; any other quad stores its fp16 rows to the sink or ring.
 #include "wushkv_internal.cuh"
 #include "quant_row.cuh"
 
@@ -35,12 +36,12 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
   const int64_t item = (int64_t)blockIdx.x * VP_WARPS + warp;
   if (item >= n_items) return;                       // uniform per warp
   const int Hkv = c.n_kv_heads;
-  const int n_hg = (Hkv + 7) >> 3;
+  const int n_hg = (Hkv + 3) >> 2;
   const int hg = (int)(item % n_hg);
   const int64_t rest = item / n_hg;
   const int qi = (int)(rest % quads);
   const int b = (int)(rest / quads);
-  const int beta = lane >> 3, h = hg * 8 + (lane & 7);
+  const int beta = lane >> 3, hf = lane & 1, h = hg * 4 + ((lane >> 1) & 3);
   const int tq = a.ta + 4 * qi;                      // absolute token of the quad
   const int tok_abs = tq + beta;
   const bool valid = h < Hkv && tok_abs < a.tb;
@@ -48,63 +49,68 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
   const int pkq = tq - c.sink;
   const bool packed_quad = tq >= c.sink && pkq < a.packed1;   // uniform per warp
   const int pk = pkq + beta;
-  __half2 xh[64];
-  {
-    uint4 raw[16];
+  const int u = b * Hkv + h;
+  const uint4* src =
+      reinterpret_cast<const uint4*>(v + (((int64_t)b * a.n_tok + tok) * Hkv + h) * D + 64 * hf);
+  if (!packed_quad) {
+    // fp16 sink or ring row (no quantisation, no lane exchange)
     if (valid) {
-      const uint4* src = reinterpret_cast<const uint4*>(
-          v + (((int64_t)b * a.n_tok + tok) * Hkv + h) * D);
+      __half* dst = tok_abs < c.sink
+                        ? c.sink_v + ((size_t)u * c.sink + tok_abs) * D
+                        : c.ring_v + ((size_t)u * c.ring_slots + (size_t)(pk % c.ring_slots)) * D;
+      uint4* o = reinterpret_cast<uint4*>(dst + 64 * hf);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) raw[i] = __ldg(src + i);
+      for (int i = 0; i < 8; ++i) {
+        const uint4 rw = __ldg(src + i);
+        const __half2 h0 = bf16x2_to_h2(rw.x), h1 = bf16x2_to_h2(rw.y);
+        const __half2 h2 = bf16x2_to_h2(rw.z), h3 = bf16x2_to_h2(rw.w);
+        o[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                          *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+      }
+    }
+    return;
+  }
+  __half2 xh[32];
+  {
+    uint4 raw[8];
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) raw[i] = __ldg(src + i);
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < 8; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < 8; ++i) {
       xh[4 * i] = bf16x2_to_h2(raw[i].x);
       xh[4 * i + 1] = bf16x2_to_h2(raw[i].y);
       xh[4 * i + 2] = bf16x2_to_h2(raw[i].z);
       xh[4 * i + 3] = bf16x2_to_h2(raw[i].w);
     }
   }
-  const int u = b * Hkv + h;
-  if (!packed_quad) {
-    if (valid) {
-      __half* dst = tok_abs < c.sink
-                        ? c.sink_v + ((size_t)u * c.sink + tok_abs) * D
-                        : c.ring_v + ((size_t)u * c.ring_slots + (size_t)(pk % c.ring_slots)) * D;
-      uint4* o = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        o[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&xh[4 * i]),
-                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 1]),
-                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 2]),
-                          *reinterpret_cast<const uint32_t*>(&xh[4 * i + 3]));
-    }
-    return;
-  }
   QParams q;
   if constexpr (AFFINE) {
     AffineStats st;
     st.init();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) st.add2(xh[2 * e], xh[2 * e + 1]);
+    for (int e = 0; e < 16; ++e) st.add2(xh[2 * e], xh[2 * e + 1]);
+    affine_merge_pair(st);
     affine_finish(st, BITS, c.r_lo == 2, c.r_hi == 127, q);
   } else {
     QuestStats st;
     st.init();
 #pragma unroll
-    for (int e = 0; e < 64; ++e) st.add(xh[e]);
+    for (int e = 0; e < 32; ++e) st.add(xh[e]);
+    quest_merge_pair(st);
     quest_finish(st, BITS, c.alpha, q);
   }
   constexpr int W0 = BITS == 3 ? 2 : BITS;
   const int quad = pkq >> 2;
-  emit_v_quad<BITS, AFFINE, 8>(
-      xh, q, beta, quad, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + (size_t)quad * 64 * W0,
+  emit_v_quad_half<BITS, AFFINE, 8>(
+      xh, q, beta, hf, quad, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + (size_t)quad * 64 * W0,
       BITS == 3 ? c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + (size_t)quad * 64 : nullptr,
       valid);
-  if (valid) {
+  if (valid && hf == 0) {
     uint8_t* meta = c.v_meta + (size_t)u * c.meta_unit_stride + (size_t)pk * c.meta_bytes;
     if constexpr (AFFINE) *reinterpret_cast<uint32_t*>(meta) = q.meta;
     else *reinterpret_cast<uint16_t*>(meta) = (uint16_t)q.meta;
@@ -126,7 +132,7 @@ cudaError_t launch_value_pack(const PrefillArgs& a, const void* v, int sms, cuda
   (void)sms;
   const int B = a.c.units / a.c.n_kv_heads;
   const int quads = (a.tb - a.ta + 3) / 4;
-  const int64_t n_items = (int64_t)B * quads * ((a.c.n_kv_heads + 7) / 8);
+  const int64_t n_items = (int64_t)B * quads * ((a.c.n_kv_heads + 3) / 4);
   if (n_items <= 0) return cudaSuccess;
   const bool aff = a.c.quantizer == WUSHKV_AFFINE_PCTCLIP;
   switch (a.c.bits) {

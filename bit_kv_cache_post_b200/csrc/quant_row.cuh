@@ -248,5 +248,90 @@ __device__ __forceinline__ void emit_v_quad(const __half2 (&xh)[64], const QPara
   }
 }
 
+// As emit_v_quad, for a lane holding one half of the token's dims (half hf:
+// dims 64 hf .. 64 hf + 63 in xh[0..31]).  Its dims carry rho in
+// [8 hf, 8 hf + 8), i.e. the words j in [hf 8/(8/w), (hf + 1) 8/(8/w)) of
+// every row unit; the quad transpose runs among the lanes of the same half
+// (STRIDE apart).  Every lane of the warp must call.
+template <int BITS, bool AFFINE, int STRIDE>
+__device__ __forceinline__ void emit_v_quad_half(const __half2 (&xh)[32], const QParams& q, int beta,
+                                                 int hf, int quad, uint8_t* quad0, uint8_t* quad1,
+                                                 bool valid) {
+  constexpr int L = 1 << BITS;
+  constexpr int W0 = BITS == 3 ? 2 : BITS;
+  constexpr int P0 = 8 / W0;
+  constexpr int NJ = 8 / P0;                // words of the half per row unit (= w)
+  uint32_t x0[2][NJ], x1[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) x0[k][j] = 0u;
+    x1[k] = 0u;
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int dl = 2 * e;                   // dim within the half (d = 64 hf + dl)
+    const int r = dl & 7, rh = (dl >> 3) & 1;
+    const int rl = 2 * (dl >> 4) + rh;      // rho - 8 hf
+    const int bb = r >> 1;
+    const uint2 p = code_pat2<AFFINE, L>(xh[e], q);
+    if constexpr (BITS == 3) {
+      x0[0][rl >> 2] += (p.x & 3u) << (8 * bb + 2 * (rl & 3));
+      x0[1][rl >> 2] += (p.y & 3u) << (8 * bb + 2 * (rl & 3));
+      x1[0] += ((p.x >> 2) & 1u) << (8 * bb + rl);
+      x1[1] += ((p.y >> 2) & 1u) << (8 * bb + rl);
+    } else {
+      x0[0][rl / P0] += p.x << (8 * bb + W0 * (rl % P0));
+      x0[1][rl / P0] += p.y << (8 * bb + W0 * (rl % P0));
+    }
+  }
+  if constexpr (BITS != 3) {
+    constexpr uint32_t corr = MAGIC * field_bit_sum(W0);
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) x0[k][j] -= corr;
+  }
+  uint32_t sa, sb;
+  quad_selectors(beta, sa, sb);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) x0[k][j] = quad_transpose<STRIDE>(x0[k][j], sa, sb);
+    if constexpr (BITS == 3) x1[k] = quad_transpose<STRIDE>(x1[k], sa, sb);
+  }
+  if (!valid) return;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int pos = (2 * beta + k + 2 * (quad & 3)) & 7;
+    if constexpr (W0 == 2) {
+      *reinterpret_cast<uint2*>(quad0 + 16 * pos + 8 * hf) = make_uint2(x0[k][0], x0[k][1]);
+    } else {
+      *reinterpret_cast<uint4*>(quad0 + 128 * hf + 16 * pos) =
+          make_uint4(x0[k][0], x0[k][1], x0[k][2], x0[k][3]);
+    }
+    if constexpr (BITS == 3) *reinterpret_cast<uint32_t*>(quad1 + 8 * pos + 4 * hf) = x1[k];
+  }
+}
+
+// Merge the statistics of the two halves of a token (lanes `lane ^ 1`).
+__device__ __forceinline__ void affine_merge_pair(AffineStats& st) {
+  auto xch = [](__half2 v) {
+    const uint32_t u = __shfl_xor_sync(FULL, *reinterpret_cast<const uint32_t*>(&v), 1);
+    return *reinterpret_cast<const __half2*>(&u);
+  };
+  const __half2 a1 = xch(st.a1), a2 = xch(st.a2), b1 = xch(st.b1), b2 = xch(st.b2);
+  st.a2 = __hmin2(__hmax2(st.a1, a1), __hmin2(st.a2, a2));
+  st.a1 = __hmin2(st.a1, a1);
+  st.b2 = __hmax2(__hmin2(st.b1, b1), __hmax2(st.b2, b2));
+  st.b1 = __hmax2(st.b1, b1);
+}
+__device__ __forceinline__ void quest_merge_pair(QuestStats& st) {
+  const double s = st.ss0 + st.ss1;
+  const double o = __shfl_xor_sync(FULL, s, 1);
+  st.ss0 = s;
+  st.ss1 = o;
+}
+
 }  // namespace rowq
 }  // namespace wushkv
