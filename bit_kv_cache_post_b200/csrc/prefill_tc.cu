@@ -12,22 +12,30 @@
 //
 // Design (one CTA per SM, 20 warps, all tiles of a CTA from one KV head):
 //   warp 0      TMA producer: 128-token bf16 K tiles (128-byte swizzle)
-//               through a four-stage ring;
-//   warps 2-3   converters: each landed tile to fp16 in place (bf16 values
-//               inside the fp16 range are exact in fp16; below 2^-17 they
-//               round to the fp16 grid, an error far under the transform's);
+//               through a four-stage shared-memory ring;
+//   warps 4-7   converters, one per TMEM lane quarter: thread i reads token
+//               row i of a landed tile, rounds it to fp16 (bf16 values inside
+//               the fp16 range are exact; below 2^-17 they round to the fp16
+//               grid, an error far under the transform's) and stores it into
+//               one of two TMEM operand buffers (64 columns, row i in lane i),
+//               freeing the shared-memory stage at once;
 //   warp 1      tensor-memory owner and MMA issuer: K' 2^s = K T_lo^T +
-//               K T_hi^T with T 2^s = T_hi + T_lo split into two fp16
-//               matrices (s a per-head power of two putting max |T| 2^s in
-//               [2^13, 2^14), so T is kept to about 2^-22 relative, as close
-//               to the exact product as an fp32 FMA loop); fp32 accumulation
-//               in four 128-column TMEM accumulators;
-//   warps 4-19  four epilogue warpgroups taking every fourth tile; thread i
-//               owns token row i (TMEM lane i), scales it by 2^-s and reads
-//               its 128 columns twice: in two 64-column loads for the
-//               per-token statistics, in double-buffered 16-column halves
-//               for the codes, which are placed two at a time into the
-//               packed row words.
+//               K T_hi^T with A = K from tensor memory and B = T from shared
+//               memory, T 2^s = T_hi + T_lo split into two fp16 matrices (s a
+//               per-head power of two putting max |T| 2^s in [2^13, 2^14), so
+//               T is kept to about 2^-22 relative, as close to the exact
+//               product as an fp32 FMA loop); fp32 accumulation in three
+//               128-column TMEM accumulators.  Two fp16 terms take 16 MMAs a
+//               tile where three bf16 terms would take 24 (a 128x128x16 MMA
+//               runs ~94 cycles here); A in tensor memory keeps the MMAs'
+//               shared-memory reads to T alone;
+//   warps 8-19  three epilogue warpgroups taking every third tile; thread i
+//               owns token row i (TMEM lane i): pass 1 reads its 128 fp32
+//               columns in two 64-column loads, rounds K' = acc 2^-s to fp16,
+//               takes the
+//               per-token statistics and writes the fp16 row back into TMEM;
+//               pass 2 reads the fp16 row in double-buffered 16-column blocks
+//               for the codes, placed two at a time into the packed words.
 // Every wait is bounded; on a timeout the CTA records DEV_ERR_TIMEOUT, stops
 // issuing, waits (bounded) for its own copies and MMAs, frees TMEM and ends.
 #include <cuda.h>
@@ -43,25 +51,28 @@ namespace {
 using namespace rowq;
 
 constexpr int TILE = 128;                    // tokens per tile (MMA M)
-constexpr int NSTAGE = 4;                    // K tiles in flight
-constexpr int NGROUP = 4;                    // epilogue warpgroups = TMEM accumulators
-constexpr int CONV_WARP = 2;                 // two converter warps
-constexpr int FIRST_EPI_WARP = 4;
-constexpr int NTHREADS = (FIRST_EPI_WARP + 4 * NGROUP) * 32;
-constexpr int TMEM_COLS = NGROUP * D;        // 512
+constexpr int NSTAGE = 4;                    // bf16 K tiles in shared memory
+constexpr int NACC = 3;                      // TMEM accumulators = epilogue warpgroups
+constexpr int NABUF = 2;                     // TMEM fp16 operand buffers
+constexpr int CONV_WARP = 4;                 // converters: warps 4-7 (lane quarters 0-3)
+constexpr int FIRST_EPI_WARP = 8;
+constexpr int NTHREADS = (FIRST_EPI_WARP + 4 * NACC) * 32;
+constexpr int TMEM_COLS = 512;
+constexpr int ABUF_COL = NACC * D;           // operand buffers after the accumulators
+constexpr int ABUF_COLS = D / 2;             // 128 fp16 per lane = 64 columns
+static_assert(ABUF_COL + NABUF * ABUF_COLS <= TMEM_COLS, "tensor memory columns");
 constexpr int TILE_BYTES = TILE * D * 2;     // one bf16 tile, 32 KB
 constexpr int HALF_BYTES = TILE_BYTES / 2;   // 64 dims (one 128-byte swizzle span)
 constexpr uint32_t PF_WAIT_POLLS = 1u << 22;
-static_assert(NSTAGE == NGROUP, "tile j uses stage and accumulator j % 4");
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_THI = 0;
 constexpr int OFF_TLO = OFF_THI + TILE_BYTES;
 constexpr int OFF_K = OFF_TLO + TILE_BYTES;
 constexpr int OFF_BAR = OFF_K + NSTAGE * TILE_BYTES;
-constexpr int N_BARS = 5 * NSTAGE + 1;
+constexpr int N_BARS = 2 * NSTAGE + 2 * NABUF + 2 * NACC + 1;
 constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-constexpr int SMEM_USED = OFF_MISC + 16;   // tmem slot, abort flag, max |T|, 2^-s
+constexpr int SMEM_USED = OFF_MISC + 16;   // tmem slot, abort flag, max |T|
 constexpr int SMEM_BYTES = SMEM_USED + 1024;          // slack for the alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -99,53 +110,43 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
 // Row modes of the epilogue
 enum : int { ROW_NONE = 0, ROW_PACKED = 1, ROW_FP16 = 2 };
 
-// fp16 values of two accumulator columns: K' = accumulator * 2^-s (exact).
-__device__ __forceinline__ __half2 kprime_h2(uint32_t a, uint32_t b, float2 unscale) {
+// fp16 values of two accumulator columns: K' = accumulator * 2^-s (exact),
+// rounded once to fp16.
+__device__ __forceinline__ uint32_t kprime_h2(uint32_t a, uint32_t b, float2 unscale) {
   const float2 v = mul2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), unscale);
-  return __floats2half2_rn(v.x, v.y);
+  const __half2 h = __floats2half2_rn(v.x, v.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Codes of the 16-column half HB of column block cc (ks = cc, h = HB) into
-// the row's packed words; ROW_FP16 rows store the half's fp16 values instead.
-template <int BITS, bool AFFINE, int HB>
-__device__ __forceinline__ void key_half(const uint32_t (&r)[16], int cc, float2 unscale,
-                                         const QParams& q, int mode, __half* win,
-                                         uint32_t (&w0)[8], uint32_t (&w1)[4], uint32_t (&t4)[8],
-                                         uint8_t* row0) {
+// Codes of column block cc (dims 32 cc .. 32 cc + 31, ks = cc) from its 16
+// fp16 pairs into the row's packed words.
+template <int BITS, bool AFFINE>
+__device__ __forceinline__ void key_block(const uint32_t (&hb)[16], int cc, const QParams& q,
+                                          uint32_t (&w0)[8], uint32_t (&w1)[4], uint32_t (&t4)[8],
+                                          bool packed, uint8_t* row0) {
   constexpr int L = 1 << BITS;
-  __half2 x[8];
+  const uint32_t m2 = 1u << (2 * cc), m4 = 1u << (4 * (cc & 1)), m1 = 1u << cc;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) x[e] = kprime_h2(r[2 * e], r[2 * e + 1], unscale);
-  if (mode == ROW_FP16) {
-    uint4* o = reinterpret_cast<uint4*>(win + 32 * cc + 16 * HB);
-#pragma unroll
-    for (int v = 0; v < 2; ++v)
-      o[v] = make_uint4(*reinterpret_cast<const uint32_t*>(&x[4 * v]),
-                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 1]),
-                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 2]),
-                        *reinterpret_cast<const uint32_t*>(&x[4 * v + 3]));
-  }
-  const uint32_t m2 = 1u << (2 * cc), m4 = 1u << (4 * (cc & 1)), m1 = (1u << cc) << (4 * HB);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = 2 * e;                            // column in the half: 4 c + beta
-    const int cq = i >> 2, beta = i & 3;            // beta in {0, 2}
-    const uint2 p = code_pat2<AFFINE, L>(x[e], q);
+  for (int e = 0; e < 16; ++e) {
+    const int i = 2 * e;                                 // dim within the block: 16 h + 4 c + beta
+    const int hh = i >> 4, cq = (i >> 2) & 3, beta = i & 3;   // beta in {0, 2}
+    const __half2 x2 = *reinterpret_cast<const __half2*>(&hb[e]);
+    const uint2 p = code_pat2<AFFINE, L>(x2, q);
     // codes to bytes beta, beta + 1; byte 1 of a pattern is zero
     const uint32_t placed = __byte_perm(p.x, p.y, beta == 0 ? 0x1140u : 0x4011u);
     if constexpr (BITS == 2) {
-      w0[2 * cq + HB] += placed * m2;
+      w0[2 * cq + hh] += placed * m2;
     } else if constexpr (BITS == 3) {
-      w0[2 * cq + HB] += (placed & 0x03030303u) * m2;
-      w1[cq] += ((placed >> 2) & 0x01010101u) * m1;
+      w0[2 * cq + hh] += (placed & 0x03030303u) * m2;
+      w1[cq] += ((placed >> 2) & 0x01010101u) * (m1 << (4 * hh));
     } else {
-      t4[2 * cq + HB] += placed * m4;
+      t4[2 * cq + hh] += placed * m4;
     }
   }
-  if constexpr (BITS == 4 && HB == 1) {
+  if constexpr (BITS == 4) {
     // words 4 c + 2 h + cc / 2 are complete after the odd block
     if (cc & 1) {
-      if (mode == ROW_PACKED) {
+      if (packed) {
         uint32_t* o = reinterpret_cast<uint32_t*>(row0);
 #pragma unroll
         for (int xw = 0; xw < 8; ++xw) o[2 * xw + (cc >> 1)] = t4[xw];
@@ -156,71 +157,83 @@ __device__ __forceinline__ void key_half(const uint32_t (&r)[16], int cc, float2
   }
 }
 
-// Key row of one token from its TMEM lane.  ROW_FP16: the fp16 rounding of
-// K' goes to `win` (a sink or ring row).  ROW_PACKED (packed format of
-// wushkv.h): dim d = 32 ks + 4 c + 16 h + beta goes to word c w + rho / (8/w),
-// field rho mod (8/w), byte beta, with rho = 4 h + ks.  Column block cc
-// holds ks = cc; the two codes of a pair (beta, beta + 1) share a word and a
-// field and are placed together with one byte permute.  The statistics read
-// the lane in two 64-column loads; the codes read it in 16-column halves,
-// each load issued while the previous half is processed.  Every lane of the
-// warp must call (the TMEM loads are warp-wide).
+// Packed words of the row from its fp16 K' (TMEM columns 0-63, two dims per
+// column): four blocks of 16 columns, each load issued while the previous
+// block is processed.
+template <int BITS, bool AFFINE>
+__device__ __forceinline__ void key_codes(uint32_t taddr, const QParams& q, bool packed,
+                                          uint32_t (&w0)[8], uint32_t (&w1)[4], uint8_t* row0) {
+  uint32_t t4[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t4[i] = 0u;
+  uint32_t ra[16], rb[16];
+  tmem_ld16(taddr, ra);
+#pragma unroll 1
+  for (int cp = 0; cp < 2; ++cp) {
+    tmem_wait_ld();                                          // block 2 cp in ra
+    tmem_ld16(taddr + (uint32_t)(32 * cp + 16), rb);
+    key_block<BITS, AFFINE>(ra, 2 * cp, q, w0, w1, t4, packed, row0);
+    tmem_wait_ld();                                          // block 2 cp + 1 in rb
+    if (cp == 0) tmem_ld16(taddr + 32u, ra);
+    key_block<BITS, AFFINE>(rb, 2 * cp + 1, q, w0, w1, t4, packed, row0);
+  }
+}
+
+// Key row of one token from its TMEM lane.  Pass 1 reads the fp32
+// accumulator in two 64-column loads, rounds K' = acc 2^-s to fp16, takes the
+// per-token statistics, stores fp16 windows rows (ROW_FP16) to `win` and
+// writes the fp16 row back into the (already read) columns 0-63.  Pass 2
+// (warps with a ROW_PACKED lane) turns the fp16 row into codes (packed
+// format of wushkv.h): dim d = 32 ks + 4 c + 16 h + beta goes to word
+// c w + rho / (8/w), field rho mod (8/w), byte beta, with rho = 4 h + ks; the
+// two codes of a pair (beta, beta + 1) share a word and a field and are
+// placed together with one byte permute.  Every lane of the warp must call
+// (the TMEM accesses are warp-wide).
 template <int BITS, bool AFFINE>
 __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double alpha,
                                         bool lo_second, bool hi_second, int mode, uint8_t* row0,
                                         uint8_t* row1, uint8_t* meta_p, __half* win) {
   const bool packed = mode == ROW_PACKED;
-  QParams q;
-  if (__any_sync(FULL, packed)) {
+  AffineStats ast;
+  QuestStats qst;
+  ast.init();
+  qst.init();
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {
+    uint32_t r[64];
+    tmem_ld64(taddr + (uint32_t)(64 * hf), r);
+    tmem_wait_ld();
+    uint32_t hb[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) hb[e] = kprime_h2(r[2 * e], r[2 * e + 1], unscale);
     if constexpr (AFFINE) {
-      AffineStats st;
-      st.init();
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(taddr + (uint32_t)(64 * hf), r);
-        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          st.add2(kprime_h2(r[4 * e], r[4 * e + 1], unscale),
-                  kprime_h2(r[4 * e + 2], r[4 * e + 3], unscale));
-      }
-      affine_finish(st, BITS, lo_second, hi_second, q);
+      for (int e = 0; e < 16; ++e)
+        ast.add2(*reinterpret_cast<const __half2*>(&hb[2 * e]),
+                 *reinterpret_cast<const __half2*>(&hb[2 * e + 1]));
     } else {
-      QuestStats st;
-      st.init();
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r[64];
-        tmem_ld64(taddr + (uint32_t)(64 * hf), r);
-        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) st.add(kprime_h2(r[2 * e], r[2 * e + 1], unscale));
-      }
-      quest_finish(st, BITS, alpha, q);
+      for (int e = 0; e < 32; ++e) qst.add(*reinterpret_cast<const __half2*>(&hb[e]));
     }
-  } else {
-    q.neglo = q.inv = make_float2(0.f, 0.f);
-    q.lo2 = __float2half2_rn(0.f);
-    q.meta = 0u;
-  }
-
-  uint32_t w0[8], w1[4], t4[8];
+    if (mode == ROW_FP16) {
+      uint4* o = reinterpret_cast<uint4*>(win + 64 * hf);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) w0[i] = t4[i] = 0u;
+      for (int v = 0; v < 8; ++v) o[v] = make_uint4(hb[4 * v], hb[4 * v + 1], hb[4 * v + 2], hb[4 * v + 3]);
+    }
+    tmem_st32(taddr + (uint32_t)(32 * hf), hb);
+  }
+  tmem_wait_st();
+  if (!__any_sync(FULL, packed)) return;
+
+  QParams q;
+  if constexpr (AFFINE) affine_finish(ast, BITS, lo_second, hi_second, q);
+  else quest_finish(qst, BITS, alpha, q);
+  uint32_t w0[8], w1[4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w0[i] = 0u;
 #pragma unroll
   for (int i = 0; i < 4; ++i) w1[i] = 0u;
-  uint32_t ra[16], rb[16];
-  tmem_ld16(taddr, ra);
-#pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {
-    tmem_wait_ld();                                          // half 0 of block cc in ra
-    tmem_ld16(taddr + (uint32_t)(32 * cc + 16), rb);
-    key_half<BITS, AFFINE, 0>(ra, cc, unscale, q, mode, win, w0, w1, t4, row0);
-    tmem_wait_ld();                                          // half 1 of block cc in rb
-    if (cc < 3) tmem_ld16(taddr + (uint32_t)(32 * cc + 32), ra);
-    key_half<BITS, AFFINE, 1>(rb, cc, unscale, q, mode, win, w0, w1, t4, row0);
-  }
+  key_codes<BITS, AFFINE>(taddr, q, packed, w0, w1, row0);
   if (!packed) return;
   if constexpr (BITS != 4) {
     uint4* o0 = reinterpret_cast<uint4*>(row0);
@@ -232,20 +245,6 @@ __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double a
   else *reinterpret_cast<uint16_t*>(meta_p) = (uint16_t)q.meta;
 }
 
-// In-place bf16 -> fp16 of one 16 KB half of a K tile (rows of 64 dims, any
-// swizzle: element-wise) by one warp.
-__device__ __forceinline__ void convert_half_tile(unsigned char* base, int lane) {
-  uint4* p = reinterpret_cast<uint4*>(base);
-#pragma unroll 4
-  for (int i = lane; i < HALF_BYTES / 16; i += 32) {
-    const uint4 w = p[i];
-    const __half2 a = bf16x2_to_h2(w.x), b = bf16x2_to_h2(w.y);
-    const __half2 c2 = bf16x2_to_h2(w.z), d = bf16x2_to_h2(w.w);
-    p[i] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b),
-                      *reinterpret_cast<const uint32_t*>(&c2), *reinterpret_cast<const uint32_t*>(&d));
-  }
-}
-
 template <int BITS, bool AFFINE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmk) {
@@ -253,12 +252,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* k_full = bars;                    // [NSTAGE] bf16 tile landed
-  uint64_t* k_conv = bars + NSTAGE;           // [NSTAGE] tile converted to fp16
-  uint64_t* k_empty = bars + 2 * NSTAGE;      // [NSTAGE] tile consumed by the MMAs
-  uint64_t* t_full = bars + 3 * NSTAGE;       // [NGROUP] accumulator ready
-  uint64_t* t_empty = bars + 4 * NSTAGE;      // [NGROUP] accumulator drained
-  uint64_t* drain = bars + 5 * NSTAGE;
+  uint64_t* k_full = bars;                                // [NSTAGE] bf16 tile landed
+  uint64_t* k_empty = bars + NSTAGE;                      // [NSTAGE] tile read by the converters
+  uint64_t* a_full = bars + 2 * NSTAGE;                   // [NABUF] fp16 operand in TMEM
+  uint64_t* a_empty = bars + 2 * NSTAGE + NABUF;          // [NABUF] operand consumed by the MMAs
+  uint64_t* t_full = bars + 2 * NSTAGE + 2 * NABUF;       // [NACC] accumulator ready
+  uint64_t* t_empty = t_full + NACC;                      // [NACC] accumulator drained
+  uint64_t* drain = t_empty + NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
   unsigned int* tmax_bits = reinterpret_cast<unsigned int*>(sm + OFF_MISC + 8);
@@ -322,10 +322,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_conv[s], 2);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&t_full[s], 1);
-      mbar_init(&t_empty[s], 4);
+      mbar_init(&k_empty[s], 4);
+    }
+    for (int b = 0; b < NABUF; ++b) {
+      mbar_init(&a_full[b], 4);
+      mbar_init(&a_empty[b], 1);
+    }
+    for (int g = 0; g < NACC; ++g) {
+      mbar_init(&t_full[g], 1);
+      mbar_init(&t_empty[g], 4);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -370,61 +375,85 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idesc = idesc_f16(false, TILE, D);   // fp16 x fp16 -> fp32
       const uint32_t tpart[2] = {smem_addr(sm + OFF_TLO), smem_addr(sm + OFF_THI)};  // small first
       for (int j = 0; j < nt; ++j) {
-        const int s = j % NSTAGE;
-        const uint32_t use = (uint32_t)(j / NSTAGE);
-        if (!wait_or_abort(&k_conv[s], use & 1, abort_flag)) {
+        const int ab = j % NABUF, acc = j % NACC;
+        const uint32_t use_a = (uint32_t)(j / NABUF), use_t = (uint32_t)(j / NACC);
+        if (!wait_or_abort(&a_full[ab], use_a & 1, abort_flag)) {
           raise_abort(abort_flag, c.status);
           break;
         }
-        if (use > 0 && !wait_or_abort(&t_empty[s], (use - 1) & 1, abort_flag)) {
+        if (use_t > 0 && !wait_or_abort(&t_empty[acc], (use_t - 1) & 1, abort_flag)) {
           raise_abort(abort_flag, c.status);
           break;
         }
         tc_fence_after();
-        const uint32_t ka = smem_addr(sm + OFF_K + s * TILE_BYTES);
-        const uint32_t dt = tmem_base + (uint32_t)(s * D);
+        const uint32_t at = tmem_base + (uint32_t)(ABUF_COL + ab * ABUF_COLS);
+        const uint32_t dt = tmem_base + (uint32_t)(acc * D);
 #pragma unroll
         for (int tp = 0; tp < 2; ++tp)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
-            umma_f16_ss(dt, sdesc_kmajor_sw128(ka + koff, 1024),
-                        sdesc_kmajor_sw128(tpart[tp] + koff, 1024), idesc,
-                        (tp | kk) ? 1u : 0u);
+            umma_f16_ts(dt, at + (uint32_t)(8 * kk), sdesc_kmajor_sw128(tpart[tp] + koff, 1024),
+                        idesc, (tp | kk) ? 1u : 0u);
           }
-        umma_commit(&k_empty[s]);
-        umma_commit(&t_full[s]);
+        umma_commit(&a_empty[ab]);
+        umma_commit(&t_full[acc]);
       }
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, PF_WAIT_POLLS);
     }
     __syncwarp();
+  } else if (warp < CONV_WARP) {
+    // warps 2 and 3 have no role after the setup
   } else if (warp < FIRST_EPI_WARP) {
-    // ---- converters: bf16 -> fp16 in place, one 64-dim half each --------------
-    const int half = warp - CONV_WARP;
+    // ---- converters: bf16 row -> fp16 row in a TMEM operand buffer ------------
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     for (int j = 0; j < nt; ++j) {
-      const int s = j % NSTAGE;
-      const uint32_t use = (uint32_t)(j / NSTAGE);
-      const bool ok = wait_or_abort(&k_full[s], use & 1, abort_flag);
+      const int s = j % NSTAGE, ab = j % NABUF;
+      const uint32_t use_s = (uint32_t)(j / NSTAGE), use_a = (uint32_t)(j / NABUF);
+      bool ok = wait_or_abort(&k_full[s], use_s & 1, abort_flag);
+      if (ok && use_a > 0) ok = wait_or_abort(&a_empty[ab], (use_a - 1) & 1, abort_flag);
       if (!__all_sync(FULL, ok)) {
         raise_abort(abort_flag, c.status);
         break;
       }
-      convert_half_tile(sm + OFF_K + s * TILE_BYTES + half * HALF_BYTES, lane);
-      fence_proxy_async();                   // generic writes -> the tensor core's reads
+      tc_fence_after();
+      uint32_t r[64];
+      const unsigned char* src = sm + OFF_K + s * TILE_BYTES + row * 128;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(src + hf * HALF_BYTES + ((ch ^ (row & 7)) << 4));
+          const __half2 h0 = bf16x2_to_h2(q4.x), h1 = bf16x2_to_h2(q4.y);
+          const __half2 h2 = bf16x2_to_h2(q4.z), h3 = bf16x2_to_h2(q4.w);
+          const int e = hf * 32 + ch * 4;
+          r[e] = *reinterpret_cast<const uint32_t*>(&h0);
+          r[e + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+          r[e + 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          r[e + 3] = *reinterpret_cast<const uint32_t*>(&h3);
+        }
+      tmem_st64(tmem_base + (uint32_t)(ABUF_COL + ab * ABUF_COLS) + lane_off, r);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&k_conv[s]);
+      if (lane == 0) {
+        mbar_arrive(&a_full[ab]);
+        mbar_arrive(&k_empty[s]);
+      }
     }
   } else {
     // ---- epilogue warpgroups ------------------------------------------------------
-    const int g = (warp - FIRST_EPI_WARP) >> 2;
+    const int g = (warp - FIRST_EPI_WARP) >> 2;   // accumulator of this group
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;          // token row of the tile
     constexpr int W0 = BITS == 3 ? 2 : BITS;
     const bool lo_second = c.r_lo == 2, hi_second = c.r_hi == 127;
     const uint32_t taddr = tmem_base + (uint32_t)(g * D) + ((uint32_t)(wq * 32) << 16);
-    for (int j = g; j < nt; j += NGROUP) {
-      const uint32_t use = (uint32_t)(j / NGROUP);
+    for (int j = g; j < nt; j += NACC) {
+      const uint32_t use = (uint32_t)(j / NACC);
       const TileInfo t = tile_info(a, h, t_begin + j);
       // destination of this row by its token index
       const int tok = t.t0 + row;

@@ -113,9 +113,9 @@ __device__ __forceinline__ void quest_finish(const QuestStats& st, int bits, dou
 // Packed fp32 arithmetic (two lanes per instruction) with an explicit
 // rounding mode.  Only for steps that cannot be contracted into a fused
 // multiply-add: on sm_100 a packed multiply feeding a packed add was
-// observed to fuse even with explicit .rn (the QuEST step x * inv + L/2
-// then rounded once), so that step uses the scalar intrinsics, which never
-// contract.
+// observed to fuse even with explicit .rn (rounding the product only once),
+// so a packed multiply is always followed by a clamp before any add, and the
+// QuEST step x * inv + L/2 uses the scalar intrinsics, which never contract.
 __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
   float2 r;
   asm("{\n .reg .b64 a, b, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n"
