@@ -102,17 +102,32 @@ __device__ __forceinline__ int cta_of(int64_t y, int64_t T, int n) {
   return (int)(ceil_div64((y + 1) * n, T) - 1);
 }
 
-// Item i of a unit (0 <= i < win_chunks + pack_blocks): window chunk number
-// floor(i nw / ni) when that count steps up at i, else packed block
-// i - floor(i nw / ni).
-__device__ __forceinline__ bool item_is_window(const DecodeArgs& a, int i, int* idx) {
-  const int64_t ni = a.win_chunks + a.pack_blocks;
-  const int w0 = (int)((int64_t)i * a.win_chunks / ni);
-  const int w1 = (int)((int64_t)(i + 1) * a.win_chunks / ni);
-  if (w1 > w0) { *idx = w0; return true; }
-  *idx = i - w0;
-  return false;
-}
+// Item i of a unit (0 <= i < ni = win_chunks + pack_blocks) is window chunk
+// number W(i) = floor(i nw / ni) when W steps up at i, else packed block
+// i - W(i).  A cursor walks a warp's items in order, keeping W(i) as a
+// quotient and remainder: one division when it starts, then an add and a
+// compare per item.
+struct ItemCursor {
+  int i, w, rem;   // current item, W(i), i nw - W(i) ni
+  __device__ __forceinline__ void start(const DecodeArgs& a, int i0) {
+    const int ni = a.win_chunks + a.pack_blocks;
+    const int64_t x = (int64_t)i0 * a.win_chunks;
+    i = i0;
+    w = (int)(x / ni);
+    rem = (int)(x - (int64_t)w * ni);
+  }
+  // Classify the current item (window chunk or packed block, and its
+  // number), then step to the next.
+  __device__ __forceinline__ bool take(const DecodeArgs& a, int* idx) {
+    const int ni = a.win_chunks + a.pack_blocks;
+    rem += a.win_chunks;
+    const bool win = rem >= ni;
+    *idx = win ? w : i - w;
+    if (win) { rem -= ni; ++w; }
+    ++i;
+    return win;
+  }
+};
 
 __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const __half* sink,
                                                     const __half* ring, int u, int w) {
@@ -122,17 +137,16 @@ __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const _
   return ring + ((size_t)u * c.ring_slots + slot) * D;
 }
 
-// All lanes: copy item i of unit u into a stage.  Packed blocks: one lane
-// issues the plane and meta copies.  Window chunks: lanes 0-7 copy the K
+// All lanes: copy an item of unit u (window chunk or packed block number idx)
+// into a stage.  Packed blocks: one lane issues the plane and meta copies.  Window chunks: lanes 0-7 copy the K
 // rows, 8-15 the V rows (rows past the window repeat its last row so that
 // the stage holds finite values; their scores are masked).
 template <int BITS, bool AFFINE>
-__device__ __forceinline__ void issue_item(const DecodeArgs& a, int u, int item, unsigned char* st,
-                                           uint64_t* bar, int lane) {
+__device__ __forceinline__ void issue_item(const DecodeArgs& a, int u, bool win, int idx,
+                                           unsigned char* st, uint64_t* bar, int lane) {
   using SL = StageLayout<BITS>;
   const DevCache& c = a.c;
-  int idx;
-  if (item_is_window(a, item, &idx)) {
+  if (win) {
     if (lane == 0) mbar_arrive_expect_tx(bar, 2u * WC * 256u);
     __syncwarp();
     if (lane < 2 * WC) {
@@ -433,18 +447,23 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
 // First copies of the warp's items, issued before the query prologue.
 template <int BITS, bool AFFINE, int G>
 __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, Smem<BITS, G>& sh, int u,
-                                                    int i0, int i1, int warp, int lane, uint32_t it) {
+                                                    int i0, int i1, int warp, int lane, uint32_t it,
+                                                    ItemCursor& ic) {
+  ic.start(a, i0);
   for (int j = 0; j < NSTAGE && j < i1 - i0; ++j) {
     const int stg = (it + j) % NSTAGE;
-    issue_item<BITS, AFFINE>(a, u, i0 + j, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+    int idx;
+    const bool win = ic.take(a, &idx);
+    issue_item<BITS, AFFINE>(a, u, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
   }
 }
 
 // The warp's items [i0, i1) of unit u through its copy ring (the first
-// NSTAGE copies were issued by warp_items_prefetch).
+// NSTAGE copies were issued by warp_items_prefetch, whose cursor ic stands
+// at the next item to copy).
 template <int BITS, int G, bool AFFINE>
 __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0, int i1, int warp,
-                           int lane, uint32_t& it, SoftmaxState<(G + 3) / 4>& S) {
+                           int lane, uint32_t& it, ItemCursor& ic, SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
   const float beta = 0.5f - (float)(1 << (BITS - 1));
@@ -467,6 +486,8 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
   }
   const int n = i1 - i0;
   if (n <= 0) return;
+  ItemCursor cc;
+  cc.start(a, i0);
   for (int i = 0; i < n; ++i, ++it) {
     const int stg = it % NSTAGE;
     if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
@@ -482,7 +503,7 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
     }
     const unsigned char* st = sh.stage[warp][stg];
     int idx;
-    if (item_is_window(a, i0 + i, &idx)) {
+    if (cc.take(a, &idx)) {
       window_chunk_compute<BITS, G>(a, sh, st, idx, lane, S);
     } else if ((idx + 1) * PB <= a.n_packed) {
       packed_block_compute<BITS, G, AFFINE, true>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
@@ -492,7 +513,9 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
     __syncwarp();
     if (i + NSTAGE < n) {
       fence_proxy_async();
-      issue_item<BITS, AFFINE>(a, u, i0 + i + NSTAGE, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+      int nidx;
+      const bool nwin = ic.take(a, &nidx);
+      issue_item<BITS, AFFINE>(a, u, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
     }
   }
 }
@@ -525,7 +548,8 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     // this warp's items; their first copies overlap the query prologue
     const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
     const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
-    warp_items_prefetch<BITS, AFFINE, G>(a, sh, u, w0, w1, warp, lane, it);
+    ItemCursor ic;
+    warp_items_prefetch<BITS, AFFINE, G>(a, sh, u, w0, w1, warp, lane, it, ic);
 
     // ---- scaled query: two int8 terms and two fp16 terms per head ---------------
     for (int g = 0; g < G; ++g)
@@ -563,7 +587,7 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
 
     // ---- this warp's items ------------------------------------------------------
     SoftmaxState<NT> S;
-    warp_items<BITS, G, AFFINE>(a, sh, u, w0, w1, warp, lane, it, S);
+    warp_items<BITS, G, AFFINE>(a, sh, u, w0, w1, warp, lane, it, ic, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
 
     float (*so)[G][D] = warp_slots(sh);
