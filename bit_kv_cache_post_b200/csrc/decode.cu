@@ -78,16 +78,73 @@ __device__ __forceinline__ float (*warp_slots(Smem<BITS, G>& sh))[G][D] {
   return reinterpret_cast<float(*)[G][D]>(&sh.stage[0][0][0]);
 }
 
-template <int NT>
-struct SoftmaxState {
-  float m[NT], l[NT], e[NT], o[NT][8][2];   // o: dims 16mt + r (+8) of head 4nt + c
-};
-
 // 2^x with the SFU (approximate, flushes denormal results to zero; 2^-inf = 0).
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Online-softmax state of a warp.  m is a reference maximum raised lazily:
+// only when a score exceeds it by more than TAU (log2 units), so weights
+// p = 2^(s - m) stay below 2^TAU and most items need no rescale.  In KEEP
+// mode the packed blocks' PV products stay in int32 accumulators across
+// items, all at the P scale F (a power of two bounding every p * scale
+// quantised since the last flush); they are converted and added into o only
+// when F or m changes, every FLUSH_BLOCKS blocks, and at the end.  Otherwise
+// each block is quantised at its own maximum F and flushed at once.
+constexpr float TAU = 8.f;
+constexpr int FLUSH_BLOCKS = 256;  // int32 headroom: 256 blocks x 64 tokens x 255 x 240 < 2^31
+
+template <int NT>
+struct SoftmaxState {
+  float m[NT], l[NT], e[NT], o[NT][8][2];   // o: dims 16mt + r (+8) of head 4nt + c
+  float F[NT];                              // P scale of the pending int32 products (0: none)
+  int pacc[8][NT][4];                       // pending PV products (KEEP only)
+  int nacc;                                 // packed blocks since the last flush
+};
+
+// Smallest power of two >= x (x > 0, finite).
+__device__ __forceinline__ float pow2_ceil(float x) {
+  return __int_as_float((__float_as_int(x) + 0x007FFFFF) & 0x7F800000);
+}
+
+// Add the pending int32 PV products of n-tile nt (two byte terms, units of
+// F / 65535) into o and clear them.
+template <int NT>
+__device__ __forceinline__ void flush_pv(SoftmaxState<NT>& S, int nt) {
+  const float f = S.F[nt] * (1.f / 65535.f);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    S.o[nt][mt][0] = fmaf(f, fmaf((float)S.pacc[mt][nt][0], 256.f, (float)S.pacc[mt][nt][1]), S.o[nt][mt][0]);
+    S.o[nt][mt][1] = fmaf(f, fmaf((float)S.pacc[mt][nt][2], 256.f, (float)S.pacc[mt][nt][3]), S.o[nt][mt][1]);
+    S.pacc[mt][nt][0] = S.pacc[mt][nt][1] = S.pacc[mt][nt][2] = S.pacc[mt][nt][3] = 0;
+  }
+}
+
+// Raise the reference maximum of every n-tile to at least its score maximum
+// over the warp (lm: this lane's), rescaling what was accumulated under the
+// old one.  Called only when some lane's score exceeds m + TAU.
+template <int NT, bool KEEP>
+__device__ __forceinline__ void raise_max(SoftmaxState<NT>& S, const float (&lm)[NT]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float bm = lm[nt];
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+    const float mn = fmaxf(S.m[nt], bm);
+    if constexpr (KEEP) {
+      if (S.F[nt] > 0.f) flush_pv(S, nt);
+      S.F[nt] = 0.f;
+    }
+    const float al = S.m[nt] == mn ? 1.f : ex2(S.m[nt] - mn);   // 0 while m is still -inf
+    S.l[nt] *= al;
+    S.e[nt] *= al;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) { S.o[nt][mt][0] *= al; S.o[nt][mt][1] *= al; }
+    S.m[nt] = mn;
+  }
 }
 
 __device__ __forceinline__ float merge_weight(float m, float M) {
@@ -213,7 +270,7 @@ __device__ __forceinline__ VWords<BITS> stage_v_words(const unsigned char* st, i
 // term) pairs, so thread c owns head 4nt + c of n-tile nt.  PV m-tile rows
 // are dims 16mt + r (+8); the PV B operand comes back through the warp's P
 // tile in shared memory.  FULL: all 64 tokens of the block are cached.
-template <int BITS, int G, bool AFFINE, bool FULL>
+template <int BITS, int G, bool AFFINE, bool FULL, bool KEEP>
 __device__ __forceinline__ void packed_block_compute(
     const DecodeArgs& a, Smem<BITS, G>& sh, const unsigned char* st, int blk, int warp, int lane,
     const uint32_t (&qb)[(G + 3) / 4][4][2], const float (&qscale)[(G + 3) / 4],
@@ -267,25 +324,33 @@ __device__ __forceinline__ void packed_block_compute(
   }
 
   // ---- online softmax; P as 16-bit fixed point in two byte terms ---------------
+  // Votes keep the common item free of cross-lane reductions: the maximum
+  // is reduced only when some score passes m + TAU, the P scale only when
+  // some p * scale passes F.
+  {
+    float lm[NT];
+    bool up = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float x = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) x = fmaxf(x, fmaxf(sc[mt][0][nt], sc[mt][1][nt]));
+      lm[nt] = x;
+      up |= x > S.m[nt] + TAU;
+    }
+    if (__any_sync(FULL_MASK, up)) raise_max<NT, KEEP>(S, lm);
+  }
   uint8_t* ps = &sh.ps[warp][0][0];
-  float al[NT], sp[NT];
+  float pmx[NT];
+  bool grow = false;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    float bm = -INFINITY;
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) bm = fmaxf(bm, fmaxf(sc[mt][0][nt], sc[mt][1][nt]));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 4));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
-    const float mn = fmaxf(S.m[nt], bm);
-    al[nt] = ex2(S.m[nt] - mn);
-    S.m[nt] = mn;
     float ls = 0.f, es = 0.f, pm = 0.f;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        const float p = ex2(sc[mt][th][nt] - mn);   // masked tokens: exp2(-inf) = 0
+        const float p = ex2(sc[mt][th][nt] - S.m[nt]);   // masked tokens: exp2(-inf) = 0
         float pt = p * vs[mt][th];
         if constexpr (!FULL) pt = (16 * mt + r + 8 * th < nvalid) ? pt : 0.f;
         ls += p;
@@ -294,19 +359,37 @@ __device__ __forceinline__ void packed_block_compute(
         pm = fmaxf(pm, pt);
         sc[mt][th][nt] = pt;
       }
-    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 4));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 8));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 16));
-    sp[nt] = pm;
-    S.l[nt] = fmaf(S.l[nt], al[nt], ls);
-    S.e[nt] = fmaf(S.e[nt], al[nt], es);
-    const float inv = pm > 0.f ? 65535.f / pm : 0.f;
+    S.l[nt] += ls;
+    S.e[nt] += es;
+    pmx[nt] = pm;
+    grow |= pm > S.F[nt];
+  }
+  if (KEEP ? __any_sync(FULL_MASK, grow) : true) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pm = pmx[nt];
+      pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 4));
+      pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 8));
+      pm = fmaxf(pm, __shfl_xor_sync(FULL_MASK, pm, 16));
+      if constexpr (KEEP) {
+        if (pm > S.F[nt]) {
+          if (S.F[nt] > 0.f) flush_pv(S, nt);
+          S.F[nt] = pow2_ceil(pm);
+        }
+      } else {
+        S.F[nt] = pm;
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float inv = S.F[nt] > 0.f ? 65535.f / S.F[nt] : 0.f;
     const int col = nt * 8 + 2 * c4;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        // 1.5 * 2^23 + rint(pt * 65535 / pm): the low 16 mantissa bits are the
+        // 1.5 * 2^23 + rint(pt * 65535 / F): the low 16 mantissa bits are the
         // rounded value; its high byte is term 0, its low byte term 1.
         const uint32_t bits = __float_as_uint(fmaf(sc[mt][th][nt], inv, 12582912.f));
         const int t = 16 * mt + r + 8 * th;
@@ -317,11 +400,13 @@ __device__ __forceinline__ void packed_block_compute(
   __syncwarp();
 
   // ---- PV: dims x (head, term) over the 64 tokens ------------------------------
-  int pacc[8][NT][4];
+  if constexpr (!KEEP) {
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt)
+    for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) pacc[mt][nt][0] = pacc[mt][nt][1] = pacc[mt][nt][2] = pacc[mt][nt][3] = 0;
+      for (int nt = 0; nt < NT; ++nt)
+        S.pacc[mt][nt][0] = S.pacc[mt][nt][1] = S.pacc[mt][nt][2] = S.pacc[mt][nt][3] = 0;
+  }
   const int pos = (r + 2 * c4) & 7;  // rotated row unit (quads 8k2 + c4 + 4q all have quad & 3 == c4)
 #pragma unroll
   for (int k2 = 0; k2 < 2; ++k2) {
@@ -345,18 +430,19 @@ __device__ __forceinline__ void packed_block_compute(
         a2 = v_frag_scaled<BITS>(v1, 2 * mt); a3 = v_frag_scaled<BITS>(v1, 2 * mt + 1);
       }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_u8u8(pacc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      for (int nt = 0; nt < NT; ++nt) mma_u8u8(S.pacc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }
   }
   __syncwarp();
+  if constexpr (KEEP) {
+    if (++S.nacc == FLUSH_BLOCKS) {
+      S.nacc = 0;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const float f = sp[nt] * (1.f / 65535.f);
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      S.o[nt][mt][0] = fmaf(S.o[nt][mt][0], al[nt], f * (float)(pacc[mt][nt][0] * 256 + pacc[mt][nt][1]));
-      S.o[nt][mt][1] = fmaf(S.o[nt][mt][1], al[nt], f * (float)(pacc[mt][nt][2] * 256 + pacc[mt][nt][3]));
+      for (int nt = 0; nt < NT; ++nt) flush_pv(S, nt);
     }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) flush_pv(S, nt);
   }
 }
 
@@ -370,7 +456,7 @@ __device__ __forceinline__ float row_factor(int rho) {
 
 // One window chunk (8 fp16 tokens) from its stage: scores with fp16 MMA
 // (rows 8-15 of the m16 tile are empty), PV with the transposed rows.
-template <int BITS, int G>
+template <int BITS, int G, bool KEEP>
 __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<BITS, G>& sh,
                                                      const unsigned char* st, int wc, int lane,
                                                      SoftmaxState<(G + 3) / 4>& S) {
@@ -400,21 +486,21 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
     }
   }
 
-  float al[NT];
+  float sv[NT];
+  {
+    bool up = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      sv[nt] = valid ? acc[nt][0] + acc[nt][1] : -INFINITY;   // hi + lo query terms
+      up |= sv[nt] > S.m[nt] + TAU;
+    }
+    if (__any_sync(FULL_MASK, up)) raise_max<NT, KEEP>(S, sv);
+  }
   uint32_t pb[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float s = valid ? acc[nt][0] + acc[nt][1] : -INFINITY;   // hi + lo query terms
-    float bm = s;
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 4));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 8));
-    bm = fmaxf(bm, __shfl_xor_sync(FULL_MASK, bm, 16));
-    const float mn = fmaxf(S.m[nt], bm);
-    al[nt] = ex2(S.m[nt] - mn);
-    S.m[nt] = mn;
-    const float p = valid ? ex2(s - mn) : 0.f;
-    S.l[nt] = fmaf(S.l[nt], al[nt], p);
-    S.e[nt] *= al[nt];
+    const float p = valid ? ex2(sv[nt] - S.m[nt]) : 0.f;
+    S.l[nt] += p;
     // B fragment of PV: p of tokens 2c, 2c+1 for column r = (head r/2, term r%2)
     const float pa = __shfl_sync(FULL_MASK, p, 8 * c4 + (r >> 1));
     const float pc = __shfl_sync(FULL_MASK, p, 8 * c4 + 4 + (r >> 1));
@@ -437,8 +523,8 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
       for (int nt = 0; nt < NT; ++nt) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
         mma_f16_k8(d, vf[2 * hm], vf[2 * hm + 1], pb[nt]);
-        S.o[nt][mt][0] = fmaf(S.o[nt][mt][0], al[nt], row_factor<BITS>(2 * mt) * (d[0] + d[1]));
-        S.o[nt][mt][1] = fmaf(S.o[nt][mt][1], al[nt], row_factor<BITS>(2 * mt + 1) * (d[2] + d[3]));
+        S.o[nt][mt][0] = fmaf(row_factor<BITS>(2 * mt), d[0] + d[1], S.o[nt][mt][0]);
+        S.o[nt][mt][1] = fmaf(row_factor<BITS>(2 * mt + 1), d[2] + d[3], S.o[nt][mt][1]);
       }
     }
   }
@@ -465,6 +551,10 @@ template <int BITS, int G, bool AFFINE>
 __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0, int i1, int warp,
                            int lane, uint32_t& it, ItemCursor& ic, SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
+  // int32 PV accumulators kept across items: one n-tile (registers) and 2 or
+  // 3 bits (with 4-bit codes the coarser shared P scale shows next to the
+  // finer code grid, so those flush every block at its own exact scale)
+  constexpr bool KEEP = NT == 1 && BITS <= 3;
   const int r = lane >> 2, c4 = lane & 3;
   const float beta = 0.5f - (float)(1 << (BITS - 1));
   uint32_t qb[NT][4][2];
@@ -480,10 +570,14 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
     qscale[nt] = sh.qscale[nt * 4 + c4];
     qsum[nt] = sh.qsum[nt * 4 + c4];
     qoff[nt] = beta * qsum[nt];
-    S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f;
+    S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; S.F[nt] = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) S.o[nt][mt][0] = S.o[nt][mt][1] = 0.f;
+    for (int mt = 0; mt < 8; ++mt) {
+      S.o[nt][mt][0] = S.o[nt][mt][1] = 0.f;
+      S.pacc[mt][nt][0] = S.pacc[mt][nt][1] = S.pacc[mt][nt][2] = S.pacc[mt][nt][3] = 0;
+    }
   }
+  S.nacc = 0;
   const int n = i1 - i0;
   if (n <= 0) return;
   ItemCursor cc;
@@ -504,11 +598,11 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
     const unsigned char* st = sh.stage[warp][stg];
     int idx;
     if (cc.take(a, &idx)) {
-      window_chunk_compute<BITS, G>(a, sh, st, idx, lane, S);
+      window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, lane, S);
     } else if ((idx + 1) * PB <= a.n_packed) {
-      packed_block_compute<BITS, G, AFFINE, true>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+      packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
     } else {
-      packed_block_compute<BITS, G, AFFINE, false>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+      packed_block_compute<BITS, G, AFFINE, false, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
     }
     __syncwarp();
     if (i + NSTAGE < n) {
@@ -517,6 +611,11 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
       const bool nwin = ic.take(a, &nidx);
       issue_item<BITS, AFFINE>(a, u, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
     }
+  }
+  if constexpr (KEEP) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      if (S.F[nt] > 0.f) flush_pv(S, nt);
   }
 }
 
