@@ -16,6 +16,7 @@ struct wushkv_cache {
   size_t bytes;
   int64_t n;        // tokens per sequence
   double alpha;     // QuEST clip ratio in use
+  wushkv::WindowMaps wmaps;   // tensor maps over the fp16 windows (decode)
 };
 
 namespace {
@@ -122,16 +123,16 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
   if (c.bits == 3) { L->n_planes = 2; L->plane_bits[0] = 2; L->plane_bits[1] = 1; }
   else { L->n_planes = 1; L->plane_bits[0] = c.bits; }
   L->packed_capacity = (int)align_up((size_t)c.max_ctx, 128);
-  size_t off = 0;
-  for (int p = 0; p < L->n_planes; ++p) {
-    L->plane_unit_stride[p] = (size_t)L->packed_capacity * 16 * L->plane_bits[p];
-    L->k_plane_off[p] = off; off = align_up(off + U * L->plane_unit_stride[p], 256);
-    L->v_plane_off[p] = off; off = align_up(off + U * L->plane_unit_stride[p], 256);
-  }
   L->meta_bytes = c.quantizer == WUSHKV_QUEST_INT ? 2 : 4;
-  L->meta_unit_stride = align_up((size_t)L->packed_capacity * L->meta_bytes, 16);
-  L->k_meta_off = off; off = align_up(off + U * L->meta_unit_stride, 256);
-  L->v_meta_off = off; off = align_up(off + U * L->meta_unit_stride, 256);
+  // block record of 64 packed tokens: K planes, V planes, K meta, V meta
+  size_t in_block = 0;
+  for (int p = 0; p < L->n_planes; ++p) { L->k_plane_off[p] = in_block; in_block += 64 * 16 * L->plane_bits[p]; }
+  for (int p = 0; p < L->n_planes; ++p) { L->v_plane_off[p] = in_block; in_block += 64 * 16 * L->plane_bits[p]; }
+  L->k_meta_off = in_block; in_block += 64 * L->meta_bytes;
+  L->v_meta_off = in_block; in_block += 64 * L->meta_bytes;
+  L->block_stride = in_block;                                   // a multiple of 128
+  L->unit_stride = (size_t)(L->packed_capacity / 64) * L->block_stride;
+  size_t off = align_up(U * L->unit_stride, 256);               // packed region at offset 0
   L->sink_unit_stride = (size_t)c.sink * 128 * 2;
   L->sink_k_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
   L->sink_v_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
@@ -155,7 +156,6 @@ DevCache dev_view(const wushkv_cache* h) {
   for (int p = 0; p < L.n_planes; ++p) {
     d.k_plane[p] = h->base + L.k_plane_off[p];
     d.v_plane[p] = h->base + L.v_plane_off[p];
-    d.plane_unit_stride[p] = L.plane_unit_stride[p];
     d.plane_bits[p] = L.plane_bits[p];
   }
   d.n_planes = L.n_planes;
@@ -164,7 +164,8 @@ DevCache dev_view(const wushkv_cache* h) {
   d.k_meta = h->base + L.k_meta_off;
   d.v_meta = h->base + L.v_meta_off;
   d.meta_bytes = (int)L.meta_bytes;
-  d.meta_unit_stride = L.meta_unit_stride;
+  d.unit_stride = L.unit_stride;
+  d.block_stride = L.block_stride;
   d.sink_k = reinterpret_cast<__half*>(h->base + L.sink_k_off);
   d.sink_v = reinterpret_cast<__half*>(h->base + L.sink_v_off);
   d.ring_k = reinterpret_cast<__half*>(h->base + L.ring_k_off);
@@ -287,6 +288,7 @@ wushkv_status wushkv_cache_create(const wushkv_config* cfg, void* dev_mem, size_
   h->bytes = bytes;
   h->n = 0;
   h->alpha = cfg->quest_alpha > 0 ? cfg->quest_alpha : wushkv_default_quest_alpha(cfg->bits);
+  make_window_maps(dev_view(h), &h->wmaps);
   const cudaError_t e = cudaMemsetAsync(dev_mem, 0, L.total_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { delete h; return WUSHKV_ECUDA; }
   *out = h;
@@ -432,7 +434,7 @@ wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache,
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   DecodeArgs a;
   if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
-  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode(a, cache->wmaps, static_cast<cudaStream_t>(stream)));
 }
 
 wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head, int32_t kv,
@@ -449,18 +451,15 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
   const int64_t ns = n < c.sink ? n : c.sink;
   const int64_t P = packed_count(n, c);
   const int W = L.ring_slots;
-  // copy the unit's regions to host
-  std::vector<std::vector<uint32_t>> planes(L.n_planes);
-  for (int p = 0; p < L.n_planes; ++p) {
-    planes[p].resize(L.plane_unit_stride[p] / 4);
-    const uint64_t off = (kv == 0 ? L.k_plane_off[p] : L.v_plane_off[p]) + u * L.plane_unit_stride[p];
-    if (cudaMemcpy(planes[p].data(), cache->base + off, L.plane_unit_stride[p], cudaMemcpyDeviceToHost))
-      return WUSHKV_ECUDA;
-  }
-  std::vector<uint16_t> meta(L.meta_unit_stride / 2);
-  if (cudaMemcpy(meta.data(), cache->base + (kv == 0 ? L.k_meta_off : L.v_meta_off) + u * L.meta_unit_stride,
-                 L.meta_unit_stride, cudaMemcpyDeviceToHost))
+  // copy the unit's regions to host (its block records hold K and V)
+  std::vector<uint8_t> packed(L.unit_stride);
+  if (cudaMemcpy(packed.data(), cache->base + u * L.unit_stride, L.unit_stride, cudaMemcpyDeviceToHost))
     return WUSHKV_ECUDA;
+  auto word_at = [&](uint64_t part_off, int64_t blk, size_t byte) {
+    uint32_t wd;
+    std::memcpy(&wd, packed.data() + (size_t)blk * L.block_stride + part_off + byte, 4);
+    return wd;
+  };
   std::vector<uint16_t> sink((size_t)c.sink * 128), ring((size_t)W * 128);
   if (c.sink > 0 &&
       cudaMemcpy(sink.data(), cache->base + (kv == 0 ? L.sink_k_off : L.sink_v_off) + u * L.sink_unit_stride,
@@ -490,13 +489,14 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
           if (kv == 0) {
             const int ks = d / 32, rem = d % 32, h2 = rem / 16, c4 = (rem % 16) / 4, beta = d % 4;
             const int rho = 4 * h2 + ks;
-            wd = planes[p][(size_t)pk * 4 * w + c4 * w + rho / F];
+            wd = word_at(L.k_plane_off[p], pk / 64, (size_t)(pk % 64) * 16 * w + 4 * (c4 * w + rho / F));
             bit = 8 * beta + w * (rho % F);
           } else {
             const int mt = d / 16, rem = d % 16, rh = rem / 8, r = rem % 8;
             const int rho = 2 * mt + rh, beta = (int)(pk % 4);
             const int quad = (int)(pk / 4);
-            wd = planes[p][(size_t)quad * 16 * w + v_word_index(quad, r, rho / F, w)];
+            wd = word_at(L.v_plane_off[p], quad / 16,
+                         (size_t)(quad % 16) * 64 * w + 4 * v_word_index(quad, r, rho / F, w));
             bit = 8 * beta + w * (rho % F);
           }
           code[d] |= (uint8_t)(((wd >> bit) & mask) << shift);
@@ -505,8 +505,11 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
       }
       if (codes_host) std::memcpy(codes_host + (size_t)i * 128, code, 128);
       if (meta_host) {
-        meta_host[2 * i] = meta[(size_t)pk * mb];
-        meta_host[2 * i + 1] = mb == 2 ? meta[(size_t)pk * mb + 1] : 0;
+        const uint8_t* m = packed.data() + (size_t)(pk / 64) * L.block_stride +
+                           (kv == 0 ? L.k_meta_off : L.v_meta_off) + (size_t)(pk % 64) * L.meta_bytes;
+        std::memcpy(&meta_host[2 * i], m, 2);
+        if (mb == 2) std::memcpy(&meta_host[2 * i + 1], m + 2, 2);
+        else meta_host[2 * i + 1] = 0;
       }
       if (fp16_host) std::memset(fp16_host + (size_t)i * 128, 0, 256);
     } else {
@@ -590,5 +593,5 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   // The array keeps the previous call's contents: arrival counters must
   // start at zero.
   if (cudaMemsetAsync(a.counters, 0, units * sizeof(int), s) != cudaSuccess) return WUSHKV_ECUDA;
-  return cuda_status(launch_decode(a, s));
+  return cuda_status(launch_decode(a, cache->wmaps, s));
 }

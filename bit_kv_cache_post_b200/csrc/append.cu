@@ -60,9 +60,6 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   MatRow trow;   // single quad: this thread's row of T, requested before the inputs
   if (transform && !staged) load_row(a.T + (size_t)h * D * D, tid, trow);
 
-  const size_t plane_u0 = (size_t)u * c.plane_unit_stride[0];
-  const size_t plane_u1 = (size_t)u * c.plane_unit_stride[1];
-
   for (int64_t Q = q_first; Q < q_last; ++Q) {
     __syncthreads();  // previous quad's smem consumers are done
     // ---- gather the quad's four tokens -------------------------------------
@@ -135,8 +132,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) x[i] = src[4 * lane + i];
       uint8_t cd[4];
-      uint8_t* meta = (kv == 0 ? c.k_meta : c.v_meta) + (size_t)u * c.meta_unit_stride +
-                      (size_t)(pk + warp) * c.meta_bytes;
+      uint8_t* meta = kv == 0 ? k_meta_at(c, u, pk + warp) : v_meta_at(c, u, pk + warp);
       if (c.quantizer == WUSHKV_QUEST_INT) {
         __half dl;
         quest_warp(x, c.bits, c.alpha, cd, dl);
@@ -151,7 +147,6 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
       __syncthreads();
       for (int p = 0; p < c.n_planes; ++p) {
         const int w = c.plane_bits[p], P = 8 / w;
-        uint8_t* base = (kv == 0 ? c.k_plane[p] : c.v_plane[p]) + (p == 0 ? plane_u0 : plane_u1);
         if (kv == 0) {
           // four K rows, 4w words each: warp = token, lane = word
           if (lane < 4 * w) {
@@ -161,7 +156,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
                 const int dim = k_field_dim(lane, w, s, beta);
                 word |= plane_value(codes[warp * D + dim], c.bits, p) << (8 * beta + w * s);
               }
-            reinterpret_cast<uint32_t*>(base + (size_t)(pk + warp) * 16 * w)[lane] = word;
+            reinterpret_cast<uint32_t*>(k_row_at(c, p, u, pk + warp))[lane] = word;
           }
         } else {
           // one V quad, 16w words: thread tid builds unit word (r, j)
@@ -174,7 +169,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
                 word |= plane_value(codes[beta * D + dim], c.bits, p) << (8 * beta + w * s);
             }
             const int quad = (int)(pk / 4);
-            reinterpret_cast<uint32_t*>(base + (size_t)quad * 64 * w)[v_word_index(quad, r, j, w)] = word;
+            reinterpret_cast<uint32_t*>(v_quad_at(c, p, u, quad))[v_word_index(quad, r, j, w)] = word;
           }
         }
       }

@@ -33,32 +33,42 @@ namespace {
 
 constexpr int NW = 4;            // warps per CTA
 constexpr int PB = 64;           // packed tokens per block
-constexpr int WC = 8;            // window tokens per chunk
-constexpr int WROW = 256 + 16;   // bytes per window row in a stage (padded: ldmatrix bank spread)
-constexpr int WIN_V = WC * WROW; // offset of the V rows of a window chunk
+constexpr int WC = WIN_BOX_ROWS; // window tokens per chunk
+// A window chunk in a stage: K then V, each two 1 KB tiles (dims 0-63 and
+// 64-127) of WC rows x 128 bytes in the 128-byte swizzle (16-byte chunk j of
+// row i at chunk j ^ i), as the tensor-map copies write them.
+constexpr int WIN_V = 2048;      // offset of the V tiles of a window chunk
 constexpr int PS_LD = PB + 16;   // bytes per row of the per-warp P tile
 constexpr int NSTAGE = 2;        // per-warp copy stages
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr int PART = PARTIAL_FLOATS;  // floats per partial record (16-byte rows)
 
-// Bytes of one packed block in a stage: K planes, V planes, K meta, V meta.
-template <int BITS>
+// One packed block in a stage, byte for byte the cache's block record: K
+// planes, V planes, K meta, V meta (MB bytes per token).
+template <int BITS, bool AFFINE = false>
 struct StageLayout {
   static constexpr int W0 = BITS == 4 ? 4 : 2;           // width of plane 0
   static constexpr int LO = PB * 16 * W0;                 // plane-0 bytes (K or V)
   static constexpr int HI = BITS == 3 ? PB * 16 : 0;      // plane-1 bytes
+  static constexpr int MB = AFFINE ? 4 : 2;
   static constexpr int K_LO = 0, K_HI = LO, V_LO = LO + HI, V_HI = 2 * LO + HI;
-  static constexpr int K_META = 2 * (LO + HI), V_META = K_META + PB * 4;
-  static constexpr int PACKED = V_META + PB * 4;
-  static constexpr int WINDOW = 2 * WIN_V;
-  static constexpr int BYTES = PACKED > WINDOW ? PACKED : WINDOW;
+  static constexpr int K_META = 2 * (LO + HI), V_META = K_META + PB * MB;
+  static constexpr int PACKED = V_META + PB * MB;
+};
+// Stage size: the larger packed record or a window chunk, in whole 1 KB
+// swizzle atoms (stages start on 1 KB boundaries).
+template <int BITS>
+struct StageBytes {
+  static constexpr int RAW = StageLayout<BITS, true>::PACKED > 2 * WIN_V ? StageLayout<BITS, true>::PACKED
+                                                                         : 2 * WIN_V;
+  static constexpr int BYTES = (RAW + 1023) / 1024 * 1024;
 };
 
 template <int BITS, int G>
 struct Smem {
   static constexpr int NT = (G + 3) / 4;   // n-tiles of 8 columns (4 heads x 2 terms)
-  alignas(128) unsigned char stage[NW][NSTAGE][StageLayout<BITS>::BYTES];
+  alignas(1024) unsigned char stage[NW][NSTAGE][StageBytes<BITS>::BYTES];
   float qs[G][D];                          // scaled q' (fp32)
   int8_t qterm[NT * 4][2][D];              // two int8 terms per head (padded heads = 0)
   __half qh[NT * 4][2][D + 8];             // fp16 hi/lo terms per head (rows padded: banks)
@@ -195,41 +205,57 @@ __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const _
 }
 
 // All lanes: copy an item of unit u (window chunk or packed block number idx)
-// into a stage.  Packed blocks: one lane issues the plane and meta copies.  Window chunks: lanes 0-7 copy the K
-// rows, 8-15 the V rows (rows past the window repeat its last row so that
-// the stage holds finite values; their scores are masked).
+// into a stage.  A packed block is one bulk copy of its block record.  A
+// window chunk whose valid rows are consecutive in the sink or the ring
+// (the usual case) is four tensor-map copies; any other chunk (it straddles
+// the sink and the ring, or the ring's wrap) is gathered by the warp with
+// plain loads into the same swizzled tiles.  Rows past the window are
+// whatever the box covers there (zeros outside the array, else stale but
+// finite rows, the buffer being zeroed at creation) or, when gathered, the
+// window's last row; their scores are masked.
 template <int BITS, bool AFFINE>
-__device__ __forceinline__ void issue_item(const DecodeArgs& a, int u, bool win, int idx,
-                                           unsigned char* st, uint64_t* bar, int lane) {
-  using SL = StageLayout<BITS>;
+__device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps& wm, int u, bool win,
+                                           int idx, unsigned char* st, uint64_t* bar, int lane) {
+  using SL = StageLayout<BITS, AFFINE>;
   const DevCache& c = a.c;
   if (win) {
-    if (lane == 0) mbar_arrive_expect_tx(bar, 2u * WC * 256u);
-    __syncwarp();
-    if (lane < 2 * WC) {
-      const int nwin = a.n_sink + a.n_recent;
-      const int w = min(idx * WC + (lane & (WC - 1)), nwin - 1);
-      const bool v = lane >= WC;
-      const __half* row = window_row(a, v ? c.sink_v : c.sink_k, v ? c.ring_v : c.ring_k, u, w);
-      bulk_copy_g2s(st + (v ? WIN_V : 0) + (lane & (WC - 1)) * WROW, row, 256u, bar);
+    const int nwin = a.n_sink + a.n_recent;
+    const int w0 = idx * WC, w1 = min(w0 + WC, nwin) - 1;
+    const CUtensorMap* mk = nullptr;
+    const CUtensorMap* mv = nullptr;
+    int y = 0;
+    if (w1 < a.n_sink) {
+      if (wm.has_sink) { mk = &wm.sink_k; mv = &wm.sink_v; y = u * c.sink + w0; }
+    } else if (w0 >= a.n_sink) {
+      const int s0 = (a.ring_first + (w0 - a.n_sink)) % c.ring_slots;
+      if (wm.has_ring && s0 + (w1 - w0) < c.ring_slots) {
+        mk = &wm.ring_k; mv = &wm.ring_v; y = u * c.ring_slots + s0;
+      }
     }
+    if (mk != nullptr) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar, 2u * WIN_V);
+        tma_load_2d(st, mk, 0, y, bar);
+        tma_load_2d(st + 1024, mk, 64, y, bar);
+        tma_load_2d(st + WIN_V, mv, 0, y, bar);
+        tma_load_2d(st + WIN_V + 1024, mv, 64, y, bar);
+      }
+      return;
+    }
+    for (int e = lane; e < 2 * WC * 16; e += 32) {
+      const int kv = e / (WC * 16), j = (e / 16) % WC, q = e % 16;
+      const int w = min(w0 + j, nwin - 1);
+      const __half* row = window_row(a, kv ? c.sink_v : c.sink_k, kv ? c.ring_v : c.ring_k, u, w);
+      const uint4 val = *reinterpret_cast<const uint4*>(row + 8 * q);
+      *reinterpret_cast<uint4*>(st + kv * WIN_V + (q / 8) * 1024 + j * 128 + (((q % 8) ^ j) * 16)) = val;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_once(bar);
     return;
   }
   if (lane != 0) return;
-  const int blk = idx;
-  const uint32_t meta = PB * (AFFINE ? 4 : 2);
-  mbar_arrive_expect_tx(bar, 2u * (SL::LO + SL::HI) + 2u * meta);
-  const size_t lo = (size_t)blk * SL::LO;
-  bulk_copy_g2s(st + SL::K_LO, c.k_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
-  bulk_copy_g2s(st + SL::V_LO, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + lo, SL::LO, bar);
-  if constexpr (BITS == 3) {
-    const size_t hi = (size_t)blk * SL::HI;
-    bulk_copy_g2s(st + SL::K_HI, c.k_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
-    bulk_copy_g2s(st + SL::V_HI, c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + hi, SL::HI, bar);
-  }
-  const size_t mo = (size_t)u * c.meta_unit_stride + (size_t)blk * meta;
-  bulk_copy_g2s(st + SL::K_META, c.k_meta + mo, meta, bar);
-  bulk_copy_g2s(st + SL::V_META, c.v_meta + mo, meta, bar);
+  mbar_arrive_expect_tx(bar, (uint32_t)SL::PACKED);
+  bulk_copy_g2s(st, k_row_at(c, 0, u, (int64_t)idx * PB), (uint32_t)SL::PACKED, bar);
 }
 
 // ---- packed blocks: copy ring + integer tensor cores ------------------------------
@@ -276,7 +302,7 @@ __device__ __forceinline__ void packed_block_compute(
     const uint32_t (&qb)[(G + 3) / 4][4][2], const float (&qscale)[(G + 3) / 4],
     const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
-  using SL = StageLayout<BITS>;
+  using SL = StageLayout<BITS, AFFINE>;
   const int r = lane >> 2, c4 = lane & 3;
   const int nvalid = a.n_packed - blk * PB;  // used when !FULL
 
@@ -463,8 +489,11 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
   const bool valid = wc * WC + r < a.n_sink + a.n_recent;
-  // lane supplies row (lane % 8) of matrix (lane / 8): 8 dims at 16-byte steps
-  const uint32_t row_addr = smem_addr(st) + (lane & 7) * WROW + (lane >> 3) * 16;
+  // lane supplies row j = lane % 8 of matrix lane / 8 (dims 32kk + 8 (lane / 8)
+  // .. +7: 16-byte chunk 4 (kk % 2) + lane / 8 of tile kk / 2, swizzled with j;
+  // odd kk flips bit 2 of the chunk, i.e. bit 6 of the 1 KB-aligned address)
+  const int j8 = lane & 7;
+  const uint32_t row_addr = smem_addr(st) + j8 * 128 + (((lane >> 3) ^ j8) << 4);
 
   float acc[NT][4];
 #pragma unroll
@@ -472,7 +501,7 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     uint32_t kf[4];
-    ldmatrix_x4(kf, row_addr + kk * 64);          // dims 32kk .. 32kk + 31
+    ldmatrix_x4(kf, (row_addr ^ ((kk & 1) << 6)) + (kk >> 1) * 1024);   // dims 32kk .. 32kk + 31
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int ks = 2 * kk + hf;
@@ -515,7 +544,7 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t vf[4];
-    ldmatrix_x4_trans(vf, row_addr + WIN_V + q * 64);   // dims 32q .. 32q + 31
+    ldmatrix_x4_trans(vf, (row_addr ^ ((q & 1) << 6)) + WIN_V + (q >> 1) * 1024);   // dims 32q .. 32q + 31
 #pragma unroll
     for (int hm = 0; hm < 2; ++hm) {
       const int mt = 2 * q + hm;
@@ -532,7 +561,8 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
 
 // First copies of the warp's items, issued before the query prologue.
 template <int BITS, bool AFFINE, int G>
-__device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, Smem<BITS, G>& sh, int u,
+__device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const WindowMaps& wm,
+                                                    Smem<BITS, G>& sh, int u,
                                                     int i0, int i1, int warp, int lane, uint32_t it,
                                                     ItemCursor& ic) {
   ic.start(a, i0);
@@ -540,7 +570,7 @@ __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, Smem<BI
     const int stg = (it + j) % NSTAGE;
     int idx;
     const bool win = ic.take(a, &idx);
-    issue_item<BITS, AFFINE>(a, u, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+    issue_item<BITS, AFFINE>(a, wm, u, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
   }
 }
 
@@ -548,7 +578,8 @@ __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, Smem<BI
 // NSTAGE copies were issued by warp_items_prefetch, whose cursor ic stands
 // at the next item to copy).
 template <int BITS, int G, bool AFFINE>
-__device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0, int i1, int warp,
+__device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u, int i0,
+                           int i1, int warp,
                            int lane, uint32_t& it, ItemCursor& ic, SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   // int32 PV accumulators kept across items: one n-tile (registers) and 2 or
@@ -609,7 +640,7 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
       fence_proxy_async();
       int nidx;
       const bool nwin = ic.take(a, &nidx);
-      issue_item<BITS, AFFINE>(a, u, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+      issue_item<BITS, AFFINE>(a, wm, u, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
     }
   }
   if constexpr (KEEP) {
@@ -621,9 +652,11 @@ __device__ void warp_items(const DecodeArgs& a, Smem<BITS, G>& sh, int u, int i0
 
 // ---- the kernel --------------------------------------------------------------------
 template <int BITS, int G, bool AFFINE>
-__global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem<BITS, G>& sh = *reinterpret_cast<Smem<BITS, G>*>(smem_raw);
+__global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4)
+    decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // stages on 1 KB boundaries (swizzle atoms): the launch adds 1 KB of slack
+  Smem<BITS, G>& sh = *reinterpret_cast<Smem<BITS, G>*>(smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u));
   constexpr int NT = (G + 3) / 4;
   const DevCache& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -648,7 +681,7 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
     const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
     const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
     ItemCursor ic;
-    warp_items_prefetch<BITS, AFFINE, G>(a, sh, u, w0, w1, warp, lane, it, ic);
+    warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, u, w0, w1, warp, lane, it, ic);
 
     // ---- scaled query: two int8 terms and two fp16 terms per head ---------------
     for (int g = 0; g < G; ++g)
@@ -686,7 +719,7 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
 
     // ---- this warp's items ------------------------------------------------------
     SoftmaxState<NT> S;
-    warp_items<BITS, G, AFFINE>(a, sh, u, w0, w1, warp, lane, it, ic, S);
+    warp_items<BITS, G, AFFINE>(a, wm, sh, u, w0, w1, warp, lane, it, ic, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
 
     float (*so)[G][D] = warp_slots(sh);
@@ -786,9 +819,9 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4) decode_kernel(DecodeA
 }
 
 template <int BITS, int G, bool AFFINE>
-cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
   auto k = decode_kernel<BITS, G, AFFINE>;
-  const int smem = (int)sizeof(Smem<BITS, G>);
+  const int smem = (int)sizeof(Smem<BITS, G>) + 1024;
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -797,17 +830,17 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  k<<<(unsigned)a.grid, NW * 32, smem, s>>>(a);
+  k<<<(unsigned)a.grid, NW * 32, smem, s>>>(a, wm);
   return cudaGetLastError();
 }
 
 template <int BITS, bool AFFINE>
-cudaError_t launch_g(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_g(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
   switch (a.c.group) {
-    case 1: return launch_t<BITS, 1, AFFINE>(a, s);
-    case 2: return launch_t<BITS, 2, AFFINE>(a, s);
-    case 4: return launch_t<BITS, 4, AFFINE>(a, s);
-    case 8: return launch_t<BITS, 8, AFFINE>(a, s);
+    case 1: return launch_t<BITS, 1, AFFINE>(a, wm, s);
+    case 2: return launch_t<BITS, 2, AFFINE>(a, wm, s);
+    case 4: return launch_t<BITS, 4, AFFINE>(a, wm, s);
+    case 8: return launch_t<BITS, 8, AFFINE>(a, wm, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -815,7 +848,7 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t s) {
 template <int BITS, int G, bool AFFINE>
 int occupancy_t() {
   auto k = decode_kernel<BITS, G, AFFINE>;
-  const int smem = (int)sizeof(Smem<BITS, G>);
+  const int smem = (int)sizeof(Smem<BITS, G>) + 1024;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
   int n = 0;
@@ -825,12 +858,12 @@ int occupancy_t() {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
   const bool affine = a.c.quantizer == WUSHKV_AFFINE_PCTCLIP;
   switch (a.c.bits) {
-    case 2: return affine ? launch_g<2, true>(a, s) : launch_g<2, false>(a, s);
-    case 3: return affine ? launch_g<3, true>(a, s) : launch_g<3, false>(a, s);
-    case 4: return affine ? launch_g<4, true>(a, s) : launch_g<4, false>(a, s);
+    case 2: return affine ? launch_g<2, true>(a, wm, s) : launch_g<2, false>(a, wm, s);
+    case 3: return affine ? launch_g<3, true>(a, wm, s) : launch_g<3, false>(a, wm, s);
+    case 4: return affine ? launch_g<4, true>(a, wm, s) : launch_g<4, false>(a, wm, s);
     default: return cudaErrorInvalidValue;
   }
 }

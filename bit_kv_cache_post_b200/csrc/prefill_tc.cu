@@ -449,7 +449,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int g = (warp - FIRST_EPI_WARP) >> 2;   // accumulator of this group
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;          // token row of the tile
-    constexpr int W0 = BITS == 3 ? 2 : BITS;
     const bool lo_second = c.r_lo == 2, hi_second = c.r_hi == 127;
     const uint32_t taddr = tmem_base + (uint32_t)(g * D) + ((uint32_t)(wq * 32) << 16);
     for (int j = g; j < nt; j += NACC) {
@@ -480,9 +479,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       key_row<BITS, AFFINE>(
           taddr, unscale, c.alpha, lo_second, hi_second, mode,
-          c.k_plane[0] + (size_t)t.u * c.plane_unit_stride[0] + pkc * 16 * W0,
-          BITS == 3 ? c.k_plane[1] + (size_t)t.u * c.plane_unit_stride[1] + pkc * 16 : nullptr,
-          c.k_meta + (size_t)t.u * c.meta_unit_stride + pkc * c.meta_bytes, win);
+          k_row_at(c, 0, t.u, (int64_t)pkc), BITS == 3 ? k_row_at(c, 1, t.u, (int64_t)pkc) : nullptr,
+          k_meta_at(c, t.u, (int64_t)pkc), win);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[g]);
@@ -504,24 +502,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // ---------------------------------------------------------------------------
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn lookup_encode() {
-  void* p = nullptr;
-  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-      q != cudaDriverEntryPointSuccess)
-    return nullptr;
-  return reinterpret_cast<EncodeTiledFn>(p);
-}
-
 // [rows][Hkv][128] bf16 rows, box = 128 rows x 64 dims of one head,
 // 128-byte swizzle (the K-major operand layout of the MMA).
 bool make_row_map(CUtensorMap* m, const void* base, int n_kv_heads, int64_t rows) {
-  static const EncodeTiledFn encode = lookup_encode();
+  const EncodeTiledFn encode = tensor_map_encoder();
   if (!encode) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_kv_heads, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)n_kv_heads * D * 2};

@@ -104,14 +104,12 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
     quest_merge_pair(st);
     quest_finish(st, BITS, c.alpha, q);
   }
-  constexpr int W0 = BITS == 3 ? 2 : BITS;
   const int quad = pkq >> 2;
   emit_v_quad_half<BITS, AFFINE, 8>(
-      xh, q, beta, hf, quad, c.v_plane[0] + (size_t)u * c.plane_unit_stride[0] + (size_t)quad * 64 * W0,
-      BITS == 3 ? c.v_plane[1] + (size_t)u * c.plane_unit_stride[1] + (size_t)quad * 64 : nullptr,
+      xh, q, beta, hf, quad, v_quad_at(c, 0, u, quad), BITS == 3 ? v_quad_at(c, 1, u, quad) : nullptr,
       valid);
   if (valid && hf == 0) {
-    uint8_t* meta = c.v_meta + (size_t)u * c.meta_unit_stride + (size_t)pk * c.meta_bytes;
+    uint8_t* meta = v_meta_at(c, u, pk);
     if constexpr (AFFINE) *reinterpret_cast<uint32_t*>(meta) = q.meta;
     else *reinterpret_cast<uint16_t*>(meta) = (uint16_t)q.meta;
   }

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libwushkv kernels and host code.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -14,11 +15,14 @@ constexpr int D = 128;           // head_dim
 constexpr int PARTIAL_FLOATS = D + 4;   // o[128], m, l, 2 pad: one split partial of one head
 constexpr unsigned FULL = 0xffffffffu;
 
-// Device-visible view of one cache buffer.
+// Device-visible view of one cache buffer.  The packed region is a run of
+// block records (64 packed tokens each: K planes, V planes, K meta, V meta);
+// k_plane[p] etc. point at those parts of unit 0's block 0.
 struct DevCache {
   uint8_t* k_plane[2];
   uint8_t* v_plane[2];
-  uint64_t plane_unit_stride[2];     // bytes per unit (K and V alike)
+  uint64_t unit_stride;              // bytes per unit of the packed region
+  uint64_t block_stride;             // bytes per block record
   int n_planes;
   int plane_bits[2];
   int bits;
@@ -26,7 +30,6 @@ struct DevCache {
   uint8_t* k_meta;
   uint8_t* v_meta;
   int meta_bytes;                    // 2 (QuEST delta) or 4 (affine scale, lo)
-  uint64_t meta_unit_stride;         // bytes per unit
   __half* sink_k;
   __half* sink_v;
   __half* ring_k;
@@ -41,6 +44,29 @@ struct DevCache {
   double alpha;                      // QuEST clip ratio
   int r_lo, r_hi;                    // affine ranks (1-indexed)
 };
+
+// Packed tokens per block record.
+constexpr int PACK_BLOCK_TOKENS = 64;
+
+// Address of the K row (16 w bytes, plane p) of packed token pk of unit u.
+__host__ __device__ __forceinline__ uint8_t* k_row_at(const DevCache& c, int p, int64_t u, int64_t pk) {
+  return c.k_plane[p] + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
+         (uint64_t)(pk & 63) * 16 * c.plane_bits[p];
+}
+// Address of V quad `quad` (tokens 4 quad .. 4 quad + 3; 64 w bytes, plane p) of unit u.
+__host__ __device__ __forceinline__ uint8_t* v_quad_at(const DevCache& c, int p, int64_t u, int64_t quad) {
+  return c.v_plane[p] + (uint64_t)u * c.unit_stride + (uint64_t)(quad >> 4) * c.block_stride +
+         (uint64_t)(quad & 15) * 64 * c.plane_bits[p];
+}
+// Addresses of the per-token meta of packed token pk of unit u.
+__host__ __device__ __forceinline__ uint8_t* k_meta_at(const DevCache& c, int64_t u, int64_t pk) {
+  return c.k_meta + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
+         (uint64_t)(pk & 63) * c.meta_bytes;
+}
+__host__ __device__ __forceinline__ uint8_t* v_meta_at(const DevCache& c, int64_t u, int64_t pk) {
+  return c.v_meta + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
+         (uint64_t)(pk & 63) * c.meta_bytes;
+}
 
 // Status bits a kernel may set in the sticky word.
 enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2, DEV_ERR_TIMEOUT = 4 };
@@ -299,6 +325,24 @@ cudaError_t launch_value_pack(const PrefillArgs& a, const void* v, int sms, cuda
 cudaError_t launch_query_transform(const void* q, int dtype, const float* TinvT, float* out,
                                    int batch, int n_q_heads, int n_kv_heads, cudaStream_t s);
 
+// Tensor maps over the fp16 windows (sink and recent ring, K and V), each a
+// [units * slots][128] array read in boxes of WIN_BOX_ROWS rows x 64 dims
+// with the 128-byte swizzle.  Built once per cache; a region whose map
+// could not be built (no sink, or more than 2^31 rows) is read without one.
+constexpr int WIN_BOX_ROWS = 8;
+struct WindowMaps {
+  CUtensorMap sink_k, sink_v, ring_k, ring_v;
+  int has_sink, has_ring;
+};
+void make_window_maps(const DevCache& c, WindowMaps* m);
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+// cuTensorMapEncodeTiled through the runtime's entry-point query (null if absent).
+EncodeTiledFn tensor_map_encoder();
+
 struct DecodeArgs {
   DevCache c;
   const float* q;          // [B][Hq][128] fp32
@@ -312,7 +356,7 @@ struct DecodeArgs {
   float* partials;         // split partials [unit][max_splits][G][132]
   int* counters;           // arrival counter per unit
 };
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& m, cudaStream_t s);
 int decode_ctas_per_sm(int bits, int group, int quantizer);
 
 }  // namespace wushkv

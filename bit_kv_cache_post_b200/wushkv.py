@@ -37,9 +37,9 @@ class Layout(ctypes.Structure):
         ("n_planes", ctypes.c_int32), ("plane_bits", ctypes.c_int32 * 2),
         ("packed_capacity", ctypes.c_int32),
         ("k_plane_off", ctypes.c_uint64 * 2), ("v_plane_off", ctypes.c_uint64 * 2),
-        ("plane_unit_stride", ctypes.c_uint64 * 2),
         ("k_meta_off", ctypes.c_uint64), ("v_meta_off", ctypes.c_uint64),
-        ("meta_bytes", ctypes.c_uint32), ("meta_unit_stride", ctypes.c_uint64),
+        ("meta_bytes", ctypes.c_uint32), ("unit_stride", ctypes.c_uint64),
+        ("block_stride", ctypes.c_uint64),
         ("sink_k_off", ctypes.c_uint64), ("sink_v_off", ctypes.c_uint64),
         ("sink_unit_stride", ctypes.c_uint64),
         ("ring_k_off", ctypes.c_uint64), ("ring_v_off", ctypes.c_uint64),

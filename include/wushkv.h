@@ -91,7 +91,18 @@ typedef struct {
 typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
 
 /* Byte layout of a cache buffer (offsets from the buffer base).  Exposed so
- * that callers can checkpoint, inspect or move the cache.  Packed format:
+ * that callers can checkpoint, inspect or move the cache.
+ *   Packed region (at offset 0): per unit, packed_capacity / 64 block
+ *     records of block_stride bytes, unit u's at u * unit_stride.  A record
+ *     holds 64 consecutive packed tokens as [K plane 0][K plane 1][V plane 0]
+ *     [V plane 1][K meta][V meta] (plane 1 only for 3-bit), so that one bulk
+ *     copy fetches everything the decode needs for those tokens.
+ *     k_plane_off[p], v_plane_off[p], k_meta_off and v_meta_off are the
+ *     offsets of these parts in unit 0's block 0; block b of unit u adds
+ *     u * unit_stride + b * block_stride.  Within a record, K rows of packed
+ *     token b * 64 + i sit at 16 * w * i, V quads b * 16 + q at 64 * w * q,
+ *     meta entries at meta_bytes * i.
+ * Formats:
  *   planes: 2-bit codes -> one 2-bit plane, 4-bit -> one 4-bit plane, 3-bit
  *     -> a 2-bit plane of (code & 3) and a 1-bit plane of (code >> 2).  A
  *     plane of width w packs 8/w fields per byte; field s of byte beta of a
@@ -114,11 +125,11 @@ typedef struct {
   int32_t n_planes;
   int32_t plane_bits[2];
   int32_t packed_capacity;          /* token slots per unit in the packed region */
-  uint64_t k_plane_off[2], v_plane_off[2];
-  uint64_t plane_unit_stride[2];    /* bytes per unit, K and V alike */
+  uint64_t k_plane_off[2], v_plane_off[2];   /* parts of unit 0's block 0 */
   uint64_t k_meta_off, v_meta_off;
   uint32_t meta_bytes;              /* per token: 2 (QuEST) or 4 (affine) */
-  uint64_t meta_unit_stride;
+  uint64_t unit_stride;             /* bytes per unit of the packed region */
+  uint64_t block_stride;            /* bytes per block record */
   uint64_t sink_k_off, sink_v_off, sink_unit_stride;
   uint64_t ring_k_off, ring_v_off, ring_unit_stride;
   int32_t ring_slots;               /* recent + chunk */

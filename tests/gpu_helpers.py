@@ -31,24 +31,36 @@ def region(cache, off: int, nbytes: int) -> np.ndarray:
     return cache.buffer[start:start + nbytes].cpu().numpy()
 
 
-def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
-    """The packed plane bytes of unit u for its first n_packed tokens, as
-    uint32 arrays shaped like the oracle's pack_* output."""
+def _unit_blocks(cache, u: int, n_packed: int) -> np.ndarray:
+    """Unit u's block records covering its first n_packed tokens, as
+    [blocks][block_stride] uint8 (64 packed tokens per record)."""
     L = cache.layout()
+    nb = (n_packed + 63) // 64
+    return region(cache, u * L.unit_stride, nb * L.block_stride).reshape(nb, L.block_stride)
+
+
+def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
+    """The packed plane bytes of unit u for its first n_packed tokens,
+    gathered from the block records into uint32 arrays shaped like the
+    oracle's pack_* output (token rows for K, quads for V)."""
+    L = cache.layout()
+    blocks = _unit_blocks(cache, u, n_packed)
     out = []
     for p in range(L.n_planes):
         w = L.plane_bits[p]
-        base = (L.k_plane_off[p] if kv == 0 else L.v_plane_off[p]) + u * L.plane_unit_stride[p]
-        raw = region(cache, base, n_packed * 16 * w).view(np.uint32)
+        off = L.k_plane_off[p] if kv == 0 else L.v_plane_off[p]
+        part = blocks[:, off:off + 64 * 16 * w].reshape(-1)[:n_packed * 16 * w]
+        raw = np.ascontiguousarray(part).view(np.uint32)
         out.append(raw.reshape(n_packed, 4 * w) if kv == 0 else raw.reshape(n_packed // 4, 16 * w))
     return out
 
 
 def unit_meta(cache, u: int, kv: int, n_packed: int) -> np.ndarray:
     L = cache.layout()
-    base = (L.k_meta_off if kv == 0 else L.v_meta_off) + u * L.meta_unit_stride
-    raw = region(cache, base, n_packed * L.meta_bytes).view(np.float16)
-    return raw.reshape(n_packed, L.meta_bytes // 2)
+    blocks = _unit_blocks(cache, u, n_packed)
+    off = L.k_meta_off if kv == 0 else L.v_meta_off
+    part = blocks[:, off:off + 64 * L.meta_bytes].reshape(-1)[:n_packed * L.meta_bytes]
+    return np.ascontiguousarray(part).view(np.float16).reshape(n_packed, L.meta_bytes // 2)
 
 
 def unit_window(cache, u: int, kv: int, which: str) -> np.ndarray:
