@@ -26,10 +26,9 @@ using namespace wushkv;
 // Decode work split: each unit's cache is a sequence of items of about 4 KB
 // (window chunks of 8 fp16 tokens spread among packed blocks of 64 tokens);
 // the units' items are shared equally among the CTAs of one wave
-// (stream-K), at least MIN_CTA_ITEMS each.  A unit is touched by at most
-// ceil(grid / units) + 1 CTAs, each writing one partial, so the workspace
-// holds max(3, MAX_GRID / units + 2) partials per unit and the grid never
-// exceeds (max_splits - 1) * units.
+// (stream-K), at least MIN_CTA_ITEMS each.  Each CTA touching a unit writes
+// one partial; the workspace holds max(3, MAX_GRID / units + 2) partials
+// per unit and the grid shrinks until no unit can meet more CTAs than that.
 constexpr int WIN_CHUNK = 8;
 constexpr int PACK_BLOCK = 64;
 constexpr int64_t MIN_CTA_ITEMS = 8;
@@ -207,7 +206,18 @@ int device_sms() {
   return sms[dev];
 }
 
-bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale, DecodeArgs* a) {
+// Most CTAs of a stream-K split that touch one unit: every CTA takes at
+// least items / grid items, so a unit of ni items meets at most
+// ceil((ni - 1) / q) + 1 of them.
+int64_t parts_per_unit_bound(int64_t items, int64_t grid, int64_t ni) {
+  const int64_t q = items / grid;
+  return (ni - 1 + q - 1) / q + 1;
+}
+
+// Fill the decode arguments of the cache's current state: window/packed
+// counts and the split plan.  EINVAL if the cache is empty, EUNSUPPORTED if
+// the item indices would not fit the kernel's 32-bit arithmetic.
+wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, float scale, DecodeArgs* a) {
   const wushkv_config& c = h->cfg;
   std::memset(a, 0, sizeof(*a));
   a->c = dev_view(h);
@@ -216,7 +226,7 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
   a->scale_log2 = sc * 1.4426950408889634f;
   const int64_t n = h->n;
-  if (n == 0) return false;
+  if (n == 0) return WUSHKV_EINVAL;
   a->n_sink = (int)(n < c.sink ? n : c.sink);
   a->n_packed = (int)packed_count(n, c);
   a->n_recent = (int)(n - a->n_sink - a->n_packed);
@@ -224,7 +234,9 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   a->win_chunks = (a->n_sink + a->n_recent + WIN_CHUNK - 1) / WIN_CHUNK;
   a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
   const int64_t units = a->c.units;
-  const int64_t items = units * (a->win_chunks + a->pack_blocks);
+  const int64_t ni = (int64_t)a->win_chunks + a->pack_blocks;
+  const int64_t items = units * ni;
+  if (items >= (int64_t(1) << 31) || ni * a->win_chunks >= (int64_t(1) << 32)) return WUSHKV_EUNSUPPORTED;
   static int occ[5][9][2] = {};
   int& o = occ[c.bits][a->c.group][c.quantizer];
   if (!o) {
@@ -235,10 +247,14 @@ bool plan_decode(const wushkv_cache* h, const float* q, float* out, float scale,
   if (grid > items / MIN_CTA_ITEMS) grid = items / MIN_CTA_ITEMS;
   if (grid > (int64_t)(a->c.max_splits - 1) * units) grid = (int64_t)(a->c.max_splits - 1) * units;
   if (grid < 1) grid = 1;
+  while (grid > 1 && parts_per_unit_bound(items, grid, ni) > a->c.max_splits) --grid;
   a->grid = (int)grid;
+  a->items_per_unit = (int)ni;
+  a->cta_q = (uint32_t)(items / grid);
+  a->cta_r = (uint32_t)(items % grid);
   a->partials = a->c.partials;
   a->counters = a->c.counters;
-  return true;
+  return WUSHKV_OK;
 }
 
 }  // namespace
@@ -430,10 +446,12 @@ wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const f
 wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream) {
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
-  if (reinterpret_cast<uintptr_t>(out_dev) & 15) return WUSHKV_EINVAL;  // written as float4
+  if ((reinterpret_cast<uintptr_t>(out_dev) | reinterpret_cast<uintptr_t>(q_prime_dev)) & 15)
+    return WUSHKV_EINVAL;  // read and written as float4
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   DecodeArgs a;
-  if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
+  const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  if (st != WUSHKV_OK) return st;
   return cuda_status(launch_decode(a, cache->wmaps, static_cast<cudaStream_t>(stream)));
 }
 
@@ -562,7 +580,8 @@ void* g_noalloc_addr[64] = {nullptr};
 extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const wushkv_cache* cache,
                                                 float* out_dev, float scale, void* stream) {
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
-  if (reinterpret_cast<uintptr_t>(out_dev) & 15) return WUSHKV_EINVAL;  // written as float4
+  if ((reinterpret_cast<uintptr_t>(out_dev) | reinterpret_cast<uintptr_t>(q_prime_dev)) & 15)
+    return WUSHKV_EINVAL;  // read and written as float4
   if (cache->n == 0) return WUSHKV_EINVAL;
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   int dev = 0;
@@ -574,10 +593,12 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
     g_noalloc_addr[dev] = p;
   }
   DecodeArgs a;
-  if (!plan_decode(cache, q_prime_dev, out_dev, scale, &a)) return WUSHKV_EINVAL;
-  // Partials are packed densely: a unit is touched by at most
-  // ceil(grid / units) + 1 CTAs of this call.
-  const int total = (a.grid + a.c.units - 1) / a.c.units + 1;
+  const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  if (st != WUSHKV_OK) return st;
+  // Partials are packed densely, as many per unit as CTAs of this call can
+  // touch one unit.
+  const int total = (int)parts_per_unit_bound((int64_t)a.items_per_unit * a.c.units, a.grid,
+                                              a.items_per_unit);
   a.c.max_splits = total;
   const size_t units = (size_t)a.c.units;
   const size_t partial_bytes = units * (size_t)total * a.c.group * PARTIAL_FLOATS * sizeof(float);

@@ -31,7 +31,10 @@ namespace wushkv {
 
 namespace {
 
-constexpr int NW = 4;            // warps per CTA
+// Warps per CTA (one CTA per SM): as many two-stage copy rings as shared
+// memory holds for the code width.
+template <int BITS> struct Warps { static constexpr int N = BITS == 2 ? 16 : BITS == 3 ? 12 : 10; };
+constexpr int UMAX = 4;          // unit segments prepared per batch
 constexpr int PB = 64;           // packed tokens per block
 constexpr int WC = WIN_BOX_ROWS; // window tokens per chunk
 // A window chunk in a stage: K then V, each two 1 KB tiles (dims 0-63 and
@@ -67,24 +70,24 @@ struct StageBytes {
 
 template <int BITS, int G>
 struct Smem {
+  static constexpr int NW = Warps<BITS>::N;
   static constexpr int NT = (G + 3) / 4;   // n-tiles of 8 columns (4 heads x 2 terms)
   alignas(1024) unsigned char stage[NW][NSTAGE][StageBytes<BITS>::BYTES];
-  float qs[G][D];                          // scaled q' (fp32)
-  int8_t qterm[NT * 4][2][D];              // two int8 terms per head (padded heads = 0)
-  __half qh[NT * 4][2][D + 8];             // fp16 hi/lo terms per head (rows padded: banks)
-  float qscale[NT * 4];                    // sigma / 254 per head
-  float qsum[NT * 4];                      // sum of the quantised q per head
+  int8_t qterm[UMAX][NT * 4][2][D];        // two int8 terms per head (padded heads = 0)
+  __half qh[UMAX][NT * 4][2][D + 8];       // fp16 hi/lo terms per head (rows padded: banks)
+  float qscale[UMAX][NT * 4];              // sigma / 254 per head
+  float qsum[UMAX][NT * 4];                // sum of the quantised q per head
   uint8_t ps[NW][NT * 8][PS_LD];           // per-warp P terms [col][token]
   float sm[NW][G], sl[NW][G];              // per-warp softmax max / sum
   alignas(8) uint64_t bar[NW][NSTAGE];
-  int is_last;
+  int is_last[UMAX];
 };
 
 // Per-warp partial outputs, placed over the stage buffers once every warp
 // has drained its copy ring.
 template <int BITS, int G>
 __device__ __forceinline__ float (*warp_slots(Smem<BITS, G>& sh))[G][D] {
-  static_assert(sizeof(float) * NW * G * D <= sizeof(sh.stage), "stage area too small");
+  static_assert(sizeof(float) * Smem<BITS, G>::NW * G * D <= sizeof(sh.stage), "stage area too small");
   return reinterpret_cast<float(*)[G][D]>(&sh.stage[0][0][0]);
 }
 
@@ -161,12 +164,16 @@ __device__ __forceinline__ float merge_weight(float m, float M) {
   return (m == -INFINITY) ? 0.f : ex2(m - M);
 }
 
-__device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-// CTA whose item range contains global item y: CTA i covers
-// [floor(i T / n), floor((i + 1) T / n)).
-__device__ __forceinline__ int cta_of(int64_t y, int64_t T, int n) {
-  return (int)(ceil_div64((y + 1) * n, T) - 1);
+// Stream-K split of the items laid end to end: the first cta_r CTAs take
+// cta_q + 1 items, the others cta_q (cta_q >= 1).  All indices fit in 32
+// bits (the host refuses larger problems).
+__device__ __forceinline__ uint32_t cta_begin(const DecodeArgs& a, uint32_t cta) {
+  return cta * a.cta_q + min(cta, a.cta_r);
+}
+// CTA whose item range contains global item y.
+__device__ __forceinline__ uint32_t cta_of(const DecodeArgs& a, uint32_t y) {
+  const uint32_t big = a.cta_r * (a.cta_q + 1);
+  return y < big ? y / (a.cta_q + 1) : a.cta_r + (y - big) / a.cta_q;
 }
 
 // Item i of a unit (0 <= i < ni = win_chunks + pack_blocks) is window chunk
@@ -177,16 +184,16 @@ __device__ __forceinline__ int cta_of(int64_t y, int64_t T, int n) {
 struct ItemCursor {
   int i, w, rem;   // current item, W(i), i nw - W(i) ni
   __device__ __forceinline__ void start(const DecodeArgs& a, int i0) {
-    const int ni = a.win_chunks + a.pack_blocks;
-    const int64_t x = (int64_t)i0 * a.win_chunks;
+    const uint32_t ni = a.items_per_unit;
+    const uint32_t x = (uint32_t)i0 * (uint32_t)a.win_chunks;   // < 2^32 (host check)
     i = i0;
     w = (int)(x / ni);
-    rem = (int)(x - (int64_t)w * ni);
+    rem = (int)(x - (uint32_t)w * ni);
   }
   // Classify the current item (window chunk or packed block, and its
   // number), then step to the next.
   __device__ __forceinline__ bool take(const DecodeArgs& a, int* idx) {
-    const int ni = a.win_chunks + a.pack_blocks;
+    const int ni = a.items_per_unit;
     rem += a.win_chunks;
     const bool win = rem >= ni;
     *idx = win ? w : i - w;
@@ -200,7 +207,8 @@ __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const _
                                                     const __half* ring, int u, int w) {
   const DevCache& c = a.c;
   if (w < a.n_sink) return sink + ((size_t)u * c.sink + w) * D;
-  const int slot = (a.ring_first + (w - a.n_sink)) % c.ring_slots;
+  int slot = a.ring_first + (w - a.n_sink);   // < 2 ring_slots
+  if (slot >= c.ring_slots) slot -= c.ring_slots;
   return ring + ((size_t)u * c.ring_slots + slot) * D;
 }
 
@@ -227,7 +235,8 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps
     if (w1 < a.n_sink) {
       if (wm.has_sink) { mk = &wm.sink_k; mv = &wm.sink_v; y = u * c.sink + w0; }
     } else if (w0 >= a.n_sink) {
-      const int s0 = (a.ring_first + (w0 - a.n_sink)) % c.ring_slots;
+      int s0 = a.ring_first + (w0 - a.n_sink);
+      if (s0 >= c.ring_slots) s0 -= c.ring_slots;
       if (wm.has_ring && s0 + (w1 - w0) < c.ring_slots) {
         mk = &wm.ring_k; mv = &wm.ring_v; y = u * c.ring_slots + s0;
       }
@@ -484,7 +493,7 @@ __device__ __forceinline__ float row_factor(int rho) {
 // (rows 8-15 of the m16 tile are empty), PV with the transposed rows.
 template <int BITS, int G, bool KEEP>
 __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<BITS, G>& sh,
-                                                     const unsigned char* st, int wc, int lane,
+                                                     const unsigned char* st, int wc, int j, int lane,
                                                      SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
@@ -507,7 +516,7 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
       const int ks = 2 * kk + hf;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const __half* qrow = &sh.qh[nt * 4 + (r >> 1)][r & 1][16 * ks + 2 * c4];
+        const __half* qrow = &sh.qh[j][nt * 4 + (r >> 1)][r & 1][16 * ks + 2 * c4];
         const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qrow);
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qrow + 8);
         mma_f16_k16(acc[nt], kf[2 * hf], 0u, kf[2 * hf + 1], 0u, b0, b1);
@@ -578,8 +587,8 @@ __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const W
 // NSTAGE copies were issued by warp_items_prefetch, whose cursor ic stands
 // at the next item to copy).
 template <int BITS, int G, bool AFFINE>
-__device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u, int i0,
-                           int i1, int warp,
+__device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u, int j,
+                           int i0, int i1, int warp,
                            int lane, uint32_t& it, ItemCursor& ic, SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
   // int32 PV accumulators kept across items: one n-tile (registers) and 2 or
@@ -597,9 +606,9 @@ __device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS,
     for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        qb[nt][ks][h] = *reinterpret_cast<const uint32_t*>(&sh.qterm[gcol][term][32 * ks + 16 * h + 4 * c4]);
-    qscale[nt] = sh.qscale[nt * 4 + c4];
-    qsum[nt] = sh.qsum[nt * 4 + c4];
+        qb[nt][ks][h] = *reinterpret_cast<const uint32_t*>(&sh.qterm[j][gcol][term][32 * ks + 16 * h + 4 * c4]);
+    qscale[nt] = sh.qscale[j][nt * 4 + c4];
+    qsum[nt] = sh.qsum[j][nt * 4 + c4];
     qoff[nt] = beta * qsum[nt];
     S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; S.F[nt] = 0.f;
 #pragma unroll
@@ -629,7 +638,7 @@ __device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS,
     const unsigned char* st = sh.stage[warp][stg];
     int idx;
     if (cc.take(a, &idx)) {
-      window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, lane, S);
+      window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, j, lane, S);
     } else if ((idx + 1) * PB <= a.n_packed) {
       packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
     } else {
@@ -651,75 +660,132 @@ __device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS,
 }
 
 // ---- the kernel --------------------------------------------------------------------
+// Warps of a CTA whose items cover nseg unit segments: segment j (cumulative
+// start cum_j items into the range of len items) owns warps [b_j, b_{j+1})
+// with b_j = clamp(round(NW cum_j / len), b_{j-1} + 1, NW - (nseg - j)), so
+// every segment has a warp and each warp stays inside one unit.
+template <int NW>
+__device__ __forceinline__ int seg_warp_bound(int j, int nseg, uint32_t cum, uint32_t len, int prev) {
+  if (j == 0) return 0;
+  if (j >= nseg) return NW;
+  int b = (int)((2u * NW * cum + len) / (2u * len));
+  b = max(b, prev + 1);
+  return min(b, NW - (nseg - j));
+}
+
+// One CTA per SM.  The CTA's stream-K item range is handled in batches of at
+// most UMAX unit segments (one batch unless the units are short): the
+// queries of the batch's units are prepared once, every warp streams the
+// items of one segment, then the warps of each segment are merged into the
+// CTA's partial for that unit, and the last CTA to finish a unit merges its
+// partials into the output.
 template <int BITS, int G, bool AFFINE>
-__global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4)
+__global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm) {
+  constexpr int NW = Warps<BITS>::N;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // stages on 1 KB boundaries (swizzle atoms): the launch adds 1 KB of slack
   Smem<BITS, G>& sh = *reinterpret_cast<Smem<BITS, G>*>(smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u));
   constexpr int NT = (G + 3) / 4;
+  constexpr int NG = NT * 4;                 // heads incl. zero padding
   const DevCache& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = lane >> 2, c4 = lane & 3;
   const int Hq = c.n_kv_heads * G;
-  const int ncta = (int)gridDim.x, cta = (int)blockIdx.x;
-  const int64_t NI = (int64_t)a.win_chunks + a.pack_blocks;   // items per unit
-  const int64_t T = NI * c.units;
-  const int64_t x0 = T * cta / ncta, x1 = T * (cta + 1) / ncta;
+  const uint32_t cta = blockIdx.x;
+  const uint32_t NI = (uint32_t)a.items_per_unit;
+  const uint32_t X0 = cta_begin(a, cta), X1 = X0 + a.cta_q + (cta < a.cta_r ? 1u : 0u);
+  const int U0 = (int)(X0 / NI), U1 = (int)((X1 - 1) / NI);
 
   if (tid < NW * NSTAGE) mbar_init(&sh.bar[tid / NSTAGE][tid % NSTAGE], 1);
   fence_barrier_init();
-  __syncthreads();
   uint32_t it = 0;
 
-  const int u_first = (int)(x0 / NI), u_last = (int)((x1 - 1) / NI);
-  for (int u = u_first; u <= u_last; ++u) {
-    const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
-    const int64_t ub = (int64_t)u * NI;
+  for (int u_first = U0; u_first <= U1; u_first += UMAX) {
+    const int nseg = min(UMAX, U1 - u_first + 1);
+    const uint32_t x0 = max(X0, (uint32_t)u_first * NI);
+    const uint32_t x1 = min(X1, (uint32_t)(u_first + nseg) * NI);
+    const uint32_t len = x1 - x0;
+
+    // ---- this warp's segment and item range ------------------------------------
+    int j = 0, bj = 0, bn = NW;
+    {
+      int prev = 0;
+      bool found = false;
+      for (int jj = 1; jj <= nseg; ++jj) {
+        const uint32_t cum = min((uint32_t)(u_first + jj) * NI, x1) - x0;
+        const int b = seg_warp_bound<NW>(jj, nseg, cum, len, prev);
+        prev = b;
+        if (!found) {
+          if (warp < b) { bn = b; found = true; }
+          else { j = jj; bj = b; }
+        }
+      }
+    }
+    const int u = u_first + j;
+    const uint32_t ub = (uint32_t)u * NI;
     const int s0 = (int)(max(x0, ub) - ub), s1 = (int)(min(x1, ub + NI) - ub);
-    // this warp's items; their first copies overlap the query prologue
-    const int w0 = s0 + (int)((int64_t)(s1 - s0) * warp / NW);
-    const int w1 = s0 + (int)((int64_t)(s1 - s0) * (warp + 1) / NW);
+    const uint32_t nw_seg = (uint32_t)(bn - bj), kw = (uint32_t)(warp - bj);
+    const int w0 = s0 + (int)((uint32_t)(s1 - s0) * kw / nw_seg);
+    const int w1 = s0 + (int)((uint32_t)(s1 - s0) * (kw + 1) / nw_seg);
+
+    // ---- query loads first (ahead of the copy flood), then the first copies ------
+    // pair p = (segment p / NG, head p % NG); warp w takes pairs w, w + NW, ...
+    constexpr int PMAX = (UMAX * NG + NW - 1) / NW;
+    float4 qv[PMAX];
+#pragma unroll
+    for (int i = 0; i < PMAX; ++i) {
+      const int p = warp + i * NW, pj = p / NG, g = p % NG;
+      qv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pj < nseg && g < G) {
+        const int pu = u_first + pj;
+        const int pb = pu / c.n_kv_heads, ph = pu % c.n_kv_heads;
+        qv[i] = __ldg(reinterpret_cast<const float4*>(a.q + ((size_t)pb * Hq + (size_t)ph * G + g) * D) + lane);
+      }
+    }
+    // barrier initialisation (first batch) or the previous batch's slot
+    // reads are complete before any copy lands
+    __syncthreads();
     ItemCursor ic;
     warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, u, w0, w1, warp, lane, it, ic);
 
-    // ---- scaled query: two int8 terms and two fp16 terms per head ---------------
-    for (int g = 0; g < G; ++g)
-      sh.qs[g][tid] = a.q[((size_t)b * Hq + (size_t)h * G + g) * D + tid] * a.scale_log2;
-    __syncthreads();
-    for (int g = warp; g < NT * 4; g += NW) {
-      float x[4];
+    // ---- scaled query: two int8 terms and two fp16 terms per head ----------------
 #pragma unroll
-      for (int i = 0; i < 4; ++i) x[i] = g < G ? sh.qs[g][4 * lane + i] : 0.f;
-      float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-      mx = warp_max_f32(mx);
-      const float sigma = mx / 127.f;
-      const float inv = mx > 0.f ? 127.f / mx : 0.f;
-      int sum = 0;
+    for (int i = 0; i < PMAX; ++i) {
+      const int p = warp + i * NW, pj = p / NG, g = p % NG;
+      if (pj < nseg) {
+        float x[4] = {qv[i].x * a.scale_log2, qv[i].y * a.scale_log2, qv[i].z * a.scale_log2,
+                      qv[i].w * a.scale_log2};
+        float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+        mx = warp_max_f32(mx);
+        const float sigma = mx / 127.f;
+        const float inv = mx > 0.f ? 127.f / mx : 0.f;
+        int sum = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float y = x[i] * inv;
-        const float t0 = fminf(fmaxf(rintf(y), -127.f), 127.f);
-        const float t1 = fminf(fmaxf(rintf((y - t0) * 254.f), -127.f), 127.f);
-        sh.qterm[g][0][4 * lane + i] = (int8_t)t0;
-        sh.qterm[g][1][4 * lane + i] = (int8_t)t1;
-        sum += (int)t0 * 254 + (int)t1;
-        const __half hi = __float2half_rn(x[i]);
-        sh.qh[g][0][4 * lane + i] = hi;
-        sh.qh[g][1][4 * lane + i] = __float2half_rn(x[i] - __half2float(hi));
-      }
+        for (int e = 0; e < 4; ++e) {
+          const float y = x[e] * inv;
+          const float t0 = fminf(fmaxf(rintf(y), -127.f), 127.f);
+          const float t1 = fminf(fmaxf(rintf((y - t0) * 254.f), -127.f), 127.f);
+          sh.qterm[pj][g][0][4 * lane + e] = (int8_t)t0;
+          sh.qterm[pj][g][1][4 * lane + e] = (int8_t)t1;
+          sum += (int)t0 * 254 + (int)t1;
+          const __half hi = __float2half_rn(x[e]);
+          sh.qh[pj][g][0][4 * lane + e] = hi;
+          sh.qh[pj][g][1][4 * lane + e] = __float2half_rn(x[e] - __half2float(hi));
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
-      if (lane == 0) {
-        sh.qscale[g] = sigma / 254.f;
-        sh.qsum[g] = (sigma / 254.f) * (float)sum;
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+        if (lane == 0) {
+          sh.qscale[pj][g] = sigma / 254.f;
+          sh.qsum[pj][g] = (sigma / 254.f) * (float)sum;
+        }
       }
     }
     __syncthreads();
 
-    // ---- this warp's items ------------------------------------------------------
+    // ---- this warp's items ---------------------------------------------------------
     SoftmaxState<NT> S;
-    warp_items<BITS, G, AFFINE>(a, wm, sh, u, w0, w1, warp, lane, it, ic, S);
+    warp_items<BITS, G, AFFINE>(a, wm, sh, u, j, w0, w1, warp, lane, it, ic, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
 
     float (*so)[G][D] = warp_slots(sh);
@@ -744,83 +810,95 @@ __global__ void __launch_bounds__(NW * 32, G >= 8 ? 3 : 4)
     }
     __syncthreads();
 
-    // ---- merge the warps, write this CTA's partial for the unit -----------------
-    const int k = cta - cta_of(ub, T, ncta);
-    const int nparts = cta_of(ub + NI - 1, T, ncta) - cta_of(ub, T, ncta) + 1;
-    float* part_base = a.partials + ((size_t)u * c.max_splits + k) * G * PART;
-    for (int g = 0; g < G; ++g) {
-      float M = -INFINITY;
-      for (int s = 0; s < NW; ++s) M = fmaxf(M, sh.sm[s][g]);
-      float L = 0.f, O = 0.f;
-      for (int s = 0; s < NW; ++s) {
-        const float f = merge_weight(sh.sm[s][g], M);
-        L = fmaf(sh.sl[s][g], f, L);
-        O = fmaf(so[s][g][tid], f, O);
+    // ---- merge the warps of each segment into this CTA's partial for the unit ----
+    {
+      int b0 = 0;
+      for (int jj = 0; jj < nseg; ++jj) {
+        const uint32_t cum = min((uint32_t)(u_first + jj + 1) * NI, x1) - x0;
+        const int b1 = seg_warp_bound<NW>(jj + 1, nseg, cum, len, b0);
+        const int uu = u_first + jj;
+        const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
+        float* part_base = a.partials + ((size_t)uu * c.max_splits + (cta - cta_u0)) * G * PART;
+        for (int e = tid; e < G * D; e += NW * 32) {
+          const int g = e / D, d = e % D;
+          float M = -INFINITY;
+          for (int w = b0; w < b1; ++w) M = fmaxf(M, sh.sm[w][g]);
+          float L = 0.f, O = 0.f;
+          for (int w = b0; w < b1; ++w) {
+            const float f = merge_weight(sh.sm[w][g], M);
+            L = fmaf(sh.sl[w][g], f, L);
+            O = fmaf(so[w][g][d], f, O);
+          }
+          float* part = part_base + (size_t)g * PART;
+          part[d] = O;
+          if (d == 0) { part[D] = M; part[D + 1] = L; }
+        }
+        b0 = b1;
       }
-      float* part = part_base + (size_t)g * PART;
-      part[tid] = O;
-      if (tid == 0) { part[D] = M; part[D + 1] = L; }
     }
 
-    // ---- arrival: the last CTA of the unit merges its partials ------------------
-    // The barrier orders every thread's partial writes before thread 0's
-    // acq_rel atomic, which publishes them at gpu scope (release) and, for
-    // the last arrival, makes the other CTAs' partials visible (acquire).
+    // ---- arrival: the last CTA of a unit merges its partials -----------------------
+    // The barrier orders every thread's partial writes before the acq_rel
+    // atomics, which publish them at gpu scope (release) and, for the last
+    // arrival, make the other CTAs' partials visible (acquire).
     __syncthreads();
-    if (tid == 0) {
-      int prev;
+    if (tid < nseg) {
+      const int uu = u_first + tid;
+      const uint32_t ubj = (uint32_t)uu * NI;
+      const int nparts = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj)) + 1;
+      int prevc;
       asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;\n"
-                   : "=r"(prev) : "l"(a.counters + u) : "memory");
-      sh.is_last = (prev == nparts - 1);
+                   : "=r"(prevc) : "l"(a.counters + uu) : "memory");
+      sh.is_last[tid] = (prevc == nparts - 1);
     }
     __syncthreads();
-    if (sh.is_last) {
-      // M, L of every partial into the (free) stage area, then each warp
-      // merges its heads with 16-byte loads, eight partials in flight.
-      float* cm = reinterpret_cast<float*>(&sh.stage[0][0][0]) + NW * G * D;
-      float* cl = cm + nparts * G;
-      const float* pbase = a.partials + (size_t)u * c.max_splits * G * PART;
-      for (int i = tid; i < nparts * G; i += NW * 32) {
-        const float* part = pbase + (size_t)i * PART;   // i = sp * G + g
-        cm[i] = __ldcg(part + D);
-        cl[i] = __ldcg(part + D + 1);
-      }
-      __syncthreads();
-      for (int g = warp; g < G; g += NW) {
-        float M = -INFINITY;
-        for (int sp = 0; sp < nparts; ++sp) M = fmaxf(M, cm[sp * G + g]);
-        float L = 0.f;
-        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp0 = 0; sp0 < nparts; sp0 += 8) {
-          float4 v[8];
+    // one warp per (segment, head) of the units this CTA completes
+    for (int p = warp; p < nseg * G; p += NW) {
+      const int jj = p / G, g = p % G;
+      if (!sh.is_last[jj]) continue;
+      const int uu = u_first + jj;
+      const uint32_t ubj = (uint32_t)uu * NI;
+      const int nparts = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj)) + 1;
+      const float* pbase = a.partials + (size_t)uu * c.max_splits * G * PART + (size_t)g * PART;
+      float M = -INFINITY;
+      for (int sp = lane; sp < nparts; sp += 32) M = fmaxf(M, __ldcg(pbase + (size_t)sp * G * PART + D));
+      M = warp_max_f32(M);
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp0 = 0; sp0 < nparts; sp0 += 8) {
+        float4 v[8];
+        float mw[8], lw[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            v[j] = sp0 + j < nparts
-                       ? __ldcg(reinterpret_cast<const float4*>(pbase + ((size_t)(sp0 + j) * G + g) * PART) + lane)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (sp0 + j >= nparts) break;
-            const float f = merge_weight(cm[(sp0 + j) * G + g], M);
-            L = fmaf(cl[(sp0 + j) * G + g], f, L);
-            O.x = fmaf(v[j].x, f, O.x); O.y = fmaf(v[j].y, f, O.y);
-            O.z = fmaf(v[j].z, f, O.z); O.w = fmaf(v[j].w, f, O.w);
-          }
+        for (int q = 0; q < 8; ++q) {
+          const bool ok = sp0 + q < nparts;
+          const float* part = pbase + (size_t)(ok ? sp0 + q : 0) * G * PART;
+          v[q] = ok ? __ldcg(reinterpret_cast<const float4*>(part) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+          mw[q] = ok ? __ldcg(part + D) : -INFINITY;
+          lw[q] = ok ? __ldcg(part + D + 1) : 0.f;
         }
-        const float il = 1.f / L;
-        *reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)h * G + g) * D + 4 * lane) =
-            make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float f = merge_weight(mw[q], M);
+          L = fmaf(lw[q], f, L);
+          O.x = fmaf(v[q].x, f, O.x); O.y = fmaf(v[q].y, f, O.y);
+          O.z = fmaf(v[q].z, f, O.z); O.w = fmaf(v[q].w, f, O.w);
+        }
       }
-      if (tid == 0) a.counters[u] = 0;
+      const float il = 1.f / L;
+      const int bb = uu / c.n_kv_heads, hh = uu % c.n_kv_heads;
+      *reinterpret_cast<float4*>(a.out + ((size_t)bb * Hq + (size_t)hh * G + g) * D + 4 * lane) =
+          make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
     }
+    if (tid < nseg && sh.is_last[tid]) a.counters[u_first + tid] = 0;
     __syncthreads();
-    fence_proxy_async();  // the stage area was written as slots; next copies overwrite it
+    fence_proxy_async();  // the stage area was written as slots; the next batch's copies overwrite it
   }
 }
 
 template <int BITS, int G, bool AFFINE>
 cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
   auto k = decode_kernel<BITS, G, AFFINE>;
+  static_assert(sizeof(Smem<BITS, G>) + 1024 <= 232448, "decode shared memory above the per-CTA limit");
   const int smem = (int)sizeof(Smem<BITS, G>) + 1024;
   static int attr_done[64] = {0};
   int dev = 0;
@@ -830,7 +908,7 @@ cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  k<<<(unsigned)a.grid, NW * 32, smem, s>>>(a, wm);
+  k<<<(unsigned)a.grid, Warps<BITS>::N * 32, smem, s>>>(a, wm);
   return cudaGetLastError();
 }
 
@@ -852,7 +930,7 @@ int occupancy_t() {
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
   int n = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, NW * 32, smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, Warps<BITS>::N * 32, smem);
   return n > 0 ? n : 1;
 }
 

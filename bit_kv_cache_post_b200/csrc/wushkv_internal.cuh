@@ -353,6 +353,8 @@ struct DecodeArgs {
   int grid;                // CTAs (stream-K shares of the units' items)
   int win_chunks;          // ceil((n_sink + n_recent) / 8)
   int pack_blocks;         // ceil(n_packed / 64)
+  int items_per_unit;      // win_chunks + pack_blocks
+  uint32_t cta_q, cta_r;   // stream-K split: CTA i starts at item i cta_q + min(i, cta_r)
   float* partials;         // split partials [unit][max_splits][G][132]
   int* counters;           // arrival counter per unit
 };
