@@ -33,7 +33,7 @@ namespace {
 
 // Warps per CTA (one CTA per SM): as many two-stage copy rings as shared
 // memory holds for the code width.
-template <int BITS> struct Warps { static constexpr int N = BITS == 2 ? 16 : BITS == 3 ? 12 : 10; };
+template <int BITS> struct Warps { static constexpr int N = BITS == 2 ? 16 : BITS == 3 ? 12 : 9; };
 constexpr int UMAX = 4;          // unit segments prepared per batch
 constexpr int PB = 64;           // packed tokens per block
 constexpr int WC = WIN_BOX_ROWS; // window tokens per chunk
@@ -79,6 +79,14 @@ struct Smem {
   float qsum[UMAX][NT * 4];                // sum of the quantised q per head
   uint8_t ps[NW][NT * 8][PS_LD];           // per-warp P terms [col][token]
   float sm[NW][G], sl[NW][G];              // per-warp softmax max / sum
+  float sf[NW][G];                         // per-warp merge weights 2^(m_w - M_segment)
+  // a warp whose item range crosses the end of segment j leaves its partial
+  // for segment j here (at most one warp per boundary)
+  float bo[UMAX - 1][G][D];
+  float bm[UMAX - 1][G], bl[UMAX - 1][G], bf[UMAX - 1][G];
+  int bused[UMAX - 1];
+  float sM[UMAX][G];                       // per-segment maximum over its partials
+  int wseg[NW];                            // segment of each warp's final state (-1: none)
   alignas(8) uint64_t bar[NW][NSTAGE];
   int is_last[UMAX];
 };
@@ -157,6 +165,40 @@ __device__ __forceinline__ void raise_max(SoftmaxState<NT>& S, const float (&lm)
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) { S.o[nt][mt][0] *= al; S.o[nt][mt][1] *= al; }
     S.m[nt] = mn;
+  }
+}
+
+// As raise_max, for scores held as differences d = s - m_used from the
+// reference in use (m_used = m, or 0 while m is still -inf): raises m to
+// the warp's score maximum when that is higher and shifts the lane's
+// differences dv to the new reference.
+template <int NT, bool KEEP, int NV>
+__device__ __forceinline__ void raise_max_d(SoftmaxState<NT>& S, const float (&lm)[NT],
+                                            float (&dv)[NV][NT]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float bm = lm[nt];
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+    const float mu = S.m[nt] == -INFINITY ? 0.f : S.m[nt];
+    const float mn = fmaxf(S.m[nt], mu + bm);
+    if (mn == S.m[nt]) continue;
+    if constexpr (KEEP) {
+      if (S.F[nt] > 0.f) flush_pv(S, nt);
+      S.F[nt] = 0.f;
+    }
+    const float al = ex2(S.m[nt] - mn);   // 0 while m is still -inf
+    S.l[nt] *= al;
+    S.e[nt] *= al;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) { S.o[nt][mt][0] *= al; S.o[nt][mt][1] *= al; }
+    S.m[nt] = mn;
+    if (mn != -INFINITY) {
+      const float sh = mn - mu;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) dv[v][nt] -= sh;
+    }
   }
 }
 
@@ -316,8 +358,12 @@ __device__ __forceinline__ void packed_block_compute(
   const int nvalid = a.n_packed - blk * PB;  // used when !FULL
 
   // ---- scores ----------------------------------------------------------------
-  float sc[4][2][NT];
+  // sc[2 mt + th]: score minus the reference in use (m, or 0 while m = -inf)
+  float sc[8][NT];
   float vs[4][2], vo[4][2];
+  float nm[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) nm[nt] = S.m[nt] == -INFINITY ? 0.f : -S.m[nt];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const KWords<BITS> kw0 = stage_k_words<BITS>(st, 16 * mt + r, c4);
@@ -349,11 +395,11 @@ __device__ __forceinline__ void packed_block_compute(
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const float xf = (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
-        float s;
-        if constexpr (AFFINE) s = fmaf(ks_, qscale[nt] * xf, ko_ * qsum[nt]);
-        else s = ks_ * fmaf(qscale[nt], xf, qoff[nt]);   // delta * (q.c + beta sum q)
-        if constexpr (!FULL) s = (t < nvalid) ? s : -INFINITY;
-        sc[mt][th][nt] = s;
+        float d;   // score minus the reference maximum in use
+        if constexpr (AFFINE) d = fmaf(ks_, qscale[nt] * xf, fmaf(ko_, qsum[nt], nm[nt]));
+        else d = fmaf(ks_, fmaf(qscale[nt], xf, qoff[nt]), nm[nt]);   // delta (q.c + beta sum q) - m
+        if constexpr (!FULL) d = (t < nvalid) ? d : -INFINITY;
+        sc[2 * mt + th][nt] = d;
       }
     }
   }
@@ -369,11 +415,11 @@ __device__ __forceinline__ void packed_block_compute(
     for (int nt = 0; nt < NT; ++nt) {
       float x = -INFINITY;
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) x = fmaxf(x, fmaxf(sc[mt][0][nt], sc[mt][1][nt]));
+      for (int v = 0; v < 8; ++v) x = fmaxf(x, sc[v][nt]);
       lm[nt] = x;
-      up |= x > S.m[nt] + TAU;
+      up |= x > TAU || S.m[nt] == -INFINITY;
     }
-    if (__any_sync(FULL_MASK, up)) raise_max<NT, KEEP>(S, lm);
+    if (__any_sync(FULL_MASK, up)) raise_max_d<NT, KEEP, 8>(S, lm, sc);
   }
   uint8_t* ps = &sh.ps[warp][0][0];
   float pmx[NT];
@@ -385,14 +431,14 @@ __device__ __forceinline__ void packed_block_compute(
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
-        const float p = ex2(sc[mt][th][nt] - S.m[nt]);   // masked tokens: exp2(-inf) = 0
+        const float p = ex2(sc[2 * mt + th][nt]);   // masked tokens: exp2(-inf) = 0
         float pt = p * vs[mt][th];
         if constexpr (!FULL) pt = (16 * mt + r + 8 * th < nvalid) ? pt : 0.f;
         ls += p;
         if constexpr (AFFINE) es = fmaf(p, vo[mt][th], es);
         else es += pt;                                 // times beta at the end
         pm = fmaxf(pm, pt);
-        sc[mt][th][nt] = pt;
+        sc[2 * mt + th][nt] = pt;
       }
     S.l[nt] += ls;
     S.e[nt] += es;
@@ -418,7 +464,11 @@ __device__ __forceinline__ void packed_block_compute(
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float inv = S.F[nt] > 0.f ? 65535.f / S.F[nt] : 0.f;
+    // 65535 / F: exact for the power-of-two F of KEEP mode; otherwise the
+    // correctly rounded reciprocal keeps pt * inv <= 65535 (1 + 2^-23)
+    float inv = 0.f;
+    if (S.F[nt] > 0.f)
+      inv = KEEP ? 65535.f * __int_as_float(0x7F000000 - __float_as_int(S.F[nt])) : 65535.f * __frcp_rn(S.F[nt]);
     const int col = nt * 8 + 2 * c4;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
@@ -426,7 +476,7 @@ __device__ __forceinline__ void packed_block_compute(
       for (int th = 0; th < 2; ++th) {
         // 1.5 * 2^23 + rint(pt * 65535 / F): the low 16 mantissa bits are the
         // rounded value; its high byte is term 0, its low byte term 1.
-        const uint32_t bits = __float_as_uint(fmaf(sc[mt][th][nt], inv, 12582912.f));
+        const uint32_t bits = __float_as_uint(fmaf(sc[2 * mt + th][nt], inv, 12582912.f));
         const int t = 16 * mt + r + 8 * th;
         ps[col * PS_LD + t] = (uint8_t)(bits >> 8);
         ps[(col + 1) * PS_LD + t] = (uint8_t)bits;
@@ -568,37 +618,45 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
   }
 }
 
+// Cursor over items laid end to end across units (global item y is item
+// y mod NI of unit y / NI).
+struct GCursor {
+  int u;
+  ItemCursor ic;
+  __device__ __forceinline__ void start(const DecodeArgs& a, uint32_t y) {
+    u = (int)(y / (uint32_t)a.items_per_unit);
+    ic.start(a, (int)(y - (uint32_t)u * (uint32_t)a.items_per_unit));
+  }
+  __device__ __forceinline__ bool take(const DecodeArgs& a, int* idx, int* unit) {
+    if (ic.i == a.items_per_unit) { ++u; ic.start(a, 0); }
+    *unit = u;
+    return ic.take(a, idx);
+  }
+};
+
 // First copies of the warp's items, issued before the query prologue.
 template <int BITS, bool AFFINE, int G>
 __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const WindowMaps& wm,
-                                                    Smem<BITS, G>& sh, int u,
-                                                    int i0, int i1, int warp, int lane, uint32_t it,
-                                                    ItemCursor& ic) {
-  ic.start(a, i0);
-  for (int j = 0; j < NSTAGE && j < i1 - i0; ++j) {
+                                                    Smem<BITS, G>& sh, uint32_t y0, uint32_t y1,
+                                                    int warp, int lane, uint32_t it, GCursor& ic) {
+  ic.start(a, y0);
+  for (uint32_t j = 0; j < (uint32_t)NSTAGE && y0 + j < y1; ++j) {
     const int stg = (it + j) % NSTAGE;
-    int idx;
-    const bool win = ic.take(a, &idx);
-    issue_item<BITS, AFFINE>(a, wm, u, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+    int idx, unit;
+    const bool win = ic.take(a, &idx, &unit);
+    issue_item<BITS, AFFINE>(a, wm, unit, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
   }
 }
 
-// The warp's items [i0, i1) of unit u through its copy ring (the first
-// NSTAGE copies were issued by warp_items_prefetch, whose cursor ic stands
-// at the next item to copy).
-template <int BITS, int G, bool AFFINE>
-__device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u, int j,
-                           int i0, int i1, int warp,
-                           int lane, uint32_t& it, ItemCursor& ic, SoftmaxState<(G + 3) / 4>& S) {
+// Reset the softmax state and load the query registers of segment j.
+template <int BITS, int G>
+__device__ __forceinline__ void begin_segment(const Smem<BITS, G>& sh, int j, int lane,
+                                              uint32_t (&qb)[(G + 3) / 4][4][2], float (&qscale)[(G + 3) / 4],
+                                              float (&qsum)[(G + 3) / 4], float (&qoff)[(G + 3) / 4],
+                                              SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
-  // int32 PV accumulators kept across items: one n-tile (registers) and 2 or
-  // 3 bits (with 4-bit codes the coarser shared P scale shows next to the
-  // finer code grid, so those flush every block at its own exact scale)
-  constexpr bool KEEP = NT == 1 && BITS <= 3;
   const int r = lane >> 2, c4 = lane & 3;
   const float beta = 0.5f - (float)(1 << (BITS - 1));
-  uint32_t qb[NT][4][2];
-  float qscale[NT], qsum[NT], qoff[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int gcol = nt * 4 + (r >> 1), term = r & 1;
@@ -618,38 +676,103 @@ __device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS,
     }
   }
   S.nacc = 0;
-  const int n = i1 - i0;
-  if (n <= 0) return;
-  ItemCursor cc;
-  cc.start(a, i0);
-  for (int i = 0; i < n; ++i, ++it) {
-    const int stg = it % NSTAGE;
-    if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
-      // A copy never completed: report it, drain what is still in flight
-      // (bounded), and contribute nothing.
-      if (lane == 0) atomicOr(a.c.status, DEV_ERR_TIMEOUT);
-      for (int j = i; j < n && j < i + NSTAGE; ++j)
-        mbar_wait_bounded(&sh.bar[warp][(it + j - i) % NSTAGE], ((it + j - i) / NSTAGE) & 1, WAIT_POLLS);
-      it += (uint32_t)(n - i);
+}
+
+// Write a warp's finished softmax state (all lanes) as one partial: o[g][d]
+// (value-space numerator, offsets included), m[g], l[g].
+template <int BITS, int G, bool AFFINE>
+__device__ __forceinline__ void state_to_slot(const SoftmaxState<(G + 3) / 4>& S, float (*o)[D], float* m,
+                                              float* l, int lane) {
+  constexpr int NT = (G + 3) / 4;
+  const int r = lane >> 2, c4 = lane & 3;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
-      return;
+  for (int nt = 0; nt < NT; ++nt) {
+    float lt = S.l[nt], et = S.e[nt];
+#pragma unroll
+    for (int sft = 4; sft < 32; sft <<= 1) {
+      lt += __shfl_xor_sync(FULL_MASK, lt, sft);
+      et += __shfl_xor_sync(FULL_MASK, et, sft);
     }
-    const unsigned char* st = sh.stage[warp][stg];
-    int idx;
-    if (cc.take(a, &idx)) {
-      window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, j, lane, S);
-    } else if ((idx + 1) * PB <= a.n_packed) {
-      packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
-    } else {
-      packed_block_compute<BITS, G, AFFINE, false, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+    if constexpr (!AFFINE) et *= 0.5f - (float)(1 << (BITS - 1));  // sum p*delta*beta
+    const int g = nt * 4 + c4;
+    if (g < G) {
+      if (r == 0) { m[g] = S.m[nt]; l[g] = lt; }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        o[g][16 * mt + r] = fmaf(S.o[nt][mt][0], 1.f / row_factor<BITS>(2 * mt), et);
+        o[g][16 * mt + r + 8] = fmaf(S.o[nt][mt][1], 1.f / row_factor<BITS>(2 * mt + 1), et);
+      }
     }
-    __syncwarp();
-    if (i + NSTAGE < n) {
-      fence_proxy_async();
-      int nidx;
-      const bool nwin = ic.take(a, &nidx);
-      issue_item<BITS, AFFINE>(a, wm, u, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+  }
+}
+
+// The warp's items [y0, y1) (global item indices, possibly spanning units)
+// through its copy ring; the first NSTAGE copies were issued by
+// warp_items_prefetch, whose cursor ic stands at the next item to copy.
+// When the items move on to the next unit, the finished unit's state goes
+// to that segment's boundary slot.  Returns the segment of the final state
+// in S (-1 if the warp had no items).
+template <int BITS, int G, bool AFFINE>
+__device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u_first,
+                        uint32_t y0, uint32_t y1, int warp, int lane, uint32_t& it, GCursor& ic,
+                        SoftmaxState<(G + 3) / 4>& S) {
+  constexpr int NT = (G + 3) / 4;
+  // int32 PV accumulators kept across items: one n-tile (registers) and 2 or
+  // 3 bits (with 4-bit codes the coarser shared P scale shows next to the
+  // finer code grid, so those flush every block at its own exact scale)
+  constexpr bool KEEP = NT == 1 && BITS <= 3;
+  uint32_t qb[NT][4][2];
+  float qscale[NT], qsum[NT], qoff[NT];
+  if (y1 <= y0) return -1;
+  const uint32_t NI = (uint32_t)a.items_per_unit;
+  int cur = -1;
+  uint32_t y = y0;
+  while (y < y1) {   // one piece per unit the range touches
+    const int unit = (int)(y / NI);
+    const uint32_t yend = min(y1, (uint32_t)(unit + 1) * NI);
+    const int j = unit - u_first;
+    if (cur >= 0) {   // leaving segment cur: its state goes to the boundary slot
+      if constexpr (KEEP) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          if (S.F[nt] > 0.f) flush_pv(S, nt);
+      }
+      state_to_slot<BITS, G, AFFINE>(S, sh.bo[cur], sh.bm[cur], sh.bl[cur], lane);
+      if (lane == 0) sh.bused[cur] = 1;
+    }
+    begin_segment<BITS, G>(sh, j, lane, qb, qscale, qsum, qoff, S);
+    cur = j;
+    ItemCursor cc;
+    cc.start(a, (int)(y - (uint32_t)unit * NI));
+    for (; y < yend; ++y, ++it) {
+      const int stg = it % NSTAGE;
+      if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
+        // A copy never completed: report it, drain what is still in flight
+        // (bounded), and contribute nothing more.
+        if (lane == 0) atomicOr(a.c.status, DEV_ERR_TIMEOUT);
+        for (uint32_t q = 0; q < (uint32_t)NSTAGE && y + q < y1; ++q)
+          mbar_wait_bounded(&sh.bar[warp][(it + q) % NSTAGE], ((it + q) / NSTAGE) & 1, WAIT_POLLS);
+        it += y1 - y;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
+        return cur;
+      }
+      const unsigned char* st = sh.stage[warp][stg];
+      int idx;
+      if (cc.take(a, &idx)) {
+        window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, j, lane, S);
+      } else if ((idx + 1) * PB <= a.n_packed) {
+        packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+      } else {
+        packed_block_compute<BITS, G, AFFINE, false, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+      }
+      __syncwarp();
+      if (y + NSTAGE < y1) {
+        fence_proxy_async();
+        int nidx, nunit;
+        const bool nwin = ic.take(a, &nidx, &nunit);
+        issue_item<BITS, AFFINE>(a, wm, nunit, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+      }
     }
   }
   if constexpr (KEEP) {
@@ -657,28 +780,17 @@ __device__ void warp_items(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS,
     for (int nt = 0; nt < NT; ++nt)
       if (S.F[nt] > 0.f) flush_pv(S, nt);
   }
+  return cur;
 }
 
 // ---- the kernel --------------------------------------------------------------------
-// Warps of a CTA whose items cover nseg unit segments: segment j (cumulative
-// start cum_j items into the range of len items) owns warps [b_j, b_{j+1})
-// with b_j = clamp(round(NW cum_j / len), b_{j-1} + 1, NW - (nseg - j)), so
-// every segment has a warp and each warp stays inside one unit.
-template <int NW>
-__device__ __forceinline__ int seg_warp_bound(int j, int nseg, uint32_t cum, uint32_t len, int prev) {
-  if (j == 0) return 0;
-  if (j >= nseg) return NW;
-  int b = (int)((2u * NW * cum + len) / (2u * len));
-  b = max(b, prev + 1);
-  return min(b, NW - (nseg - j));
-}
-
 // One CTA per SM.  The CTA's stream-K item range is handled in batches of at
-// most UMAX unit segments (one batch unless the units are short): the
-// queries of the batch's units are prepared once, every warp streams the
-// items of one segment, then the warps of each segment are merged into the
-// CTA's partial for that unit, and the last CTA to finish a unit merges its
-// partials into the output.
+// most UMAX unit segments (one batch unless the units are short).  The
+// queries of the batch's units are prepared once; warp w streams items
+// [x0 + len w / NW, x0 + len (w + 1) / NW) of the batch, crossing a unit
+// boundary when its range does; the warps' states are merged per segment
+// into the CTA's partial for that unit, and the last CTA to finish a unit
+// merges its partials into the output.
 template <int BITS, int G, bool AFFINE>
 __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm) {
@@ -690,15 +802,18 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   constexpr int NG = NT * 4;                 // heads incl. zero padding
   const DevCache& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r = lane >> 2, c4 = lane & 3;
   const int Hq = c.n_kv_heads * G;
   const uint32_t cta = blockIdx.x;
   const uint32_t NI = (uint32_t)a.items_per_unit;
   const uint32_t X0 = cta_begin(a, cta), X1 = X0 + a.cta_q + (cta < a.cta_r ? 1u : 0u);
   const int U0 = (int)(X0 / NI), U1 = (int)((X1 - 1) / NI);
 
-  if (tid < NW * NSTAGE) mbar_init(&sh.bar[tid / NSTAGE][tid % NSTAGE], 1);
-  fence_barrier_init();
+  // each warp initialises its own copy ring's barriers
+  if (lane < NSTAGE) {
+    mbar_init(&sh.bar[warp][lane], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
   uint32_t it = 0;
 
   for (int u_first = U0; u_first <= U1; u_first += UMAX) {
@@ -706,28 +821,8 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     const uint32_t x0 = max(X0, (uint32_t)u_first * NI);
     const uint32_t x1 = min(X1, (uint32_t)(u_first + nseg) * NI);
     const uint32_t len = x1 - x0;
-
-    // ---- this warp's segment and item range ------------------------------------
-    int j = 0, bj = 0, bn = NW;
-    {
-      int prev = 0;
-      bool found = false;
-      for (int jj = 1; jj <= nseg; ++jj) {
-        const uint32_t cum = min((uint32_t)(u_first + jj) * NI, x1) - x0;
-        const int b = seg_warp_bound<NW>(jj, nseg, cum, len, prev);
-        prev = b;
-        if (!found) {
-          if (warp < b) { bn = b; found = true; }
-          else { j = jj; bj = b; }
-        }
-      }
-    }
-    const int u = u_first + j;
-    const uint32_t ub = (uint32_t)u * NI;
-    const int s0 = (int)(max(x0, ub) - ub), s1 = (int)(min(x1, ub + NI) - ub);
-    const uint32_t nw_seg = (uint32_t)(bn - bj), kw = (uint32_t)(warp - bj);
-    const int w0 = s0 + (int)((uint32_t)(s1 - s0) * kw / nw_seg);
-    const int w1 = s0 + (int)((uint32_t)(s1 - s0) * (kw + 1) / nw_seg);
+    const uint32_t y0 = x0 + (uint32_t)((uint64_t)len * (uint32_t)warp / NW);
+    const uint32_t y1 = x0 + (uint32_t)((uint64_t)len * (uint32_t)(warp + 1) / NW);
 
     // ---- query loads first (ahead of the copy flood), then the first copies ------
     // pair p = (segment p / NG, head p % NG); warp w takes pairs w, w + NW, ...
@@ -743,11 +838,11 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
         qv[i] = __ldg(reinterpret_cast<const float4*>(a.q + ((size_t)pb * Hq + (size_t)ph * G + g) * D) + lane);
       }
     }
-    // barrier initialisation (first batch) or the previous batch's slot
-    // reads are complete before any copy lands
-    __syncthreads();
-    ItemCursor ic;
-    warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, u, w0, w1, warp, lane, it, ic);
+    // (the previous batch ended with a barrier: its slot reads are complete
+    // before these copies land in the stage area)
+    GCursor ic;
+    warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, y0, y1, warp, lane, it, ic);
+    if (tid < UMAX - 1) sh.bused[tid] = 0;
 
     // ---- scaled query: two int8 terms and two fp16 terms per head ----------------
 #pragma unroll
@@ -783,57 +878,56 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     }
     __syncthreads();
 
-    // ---- this warp's items ---------------------------------------------------------
+    // ---- this warp's items -----------------------------------------------------------
     SoftmaxState<NT> S;
-    warp_items<BITS, G, AFFINE>(a, wm, sh, u, j, w0, w1, warp, lane, it, ic, S);
+    const int jl = warp_run<BITS, G, AFFINE>(a, wm, sh, u_first, y0, y1, warp, lane, it, ic, S);
     __syncthreads();  // every copy ring is drained: the stage area becomes slots
 
     float (*so)[G][D] = warp_slots(sh);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float lt = S.l[nt], et = S.e[nt];
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        lt += __shfl_xor_sync(FULL_MASK, lt, o);
-        et += __shfl_xor_sync(FULL_MASK, et, o);
-      }
-      if constexpr (!AFFINE) et *= 0.5f - (float)(1 << (BITS - 1));  // sum p*delta*beta
-      const int g = nt * 4 + c4;
-      if (g < G) {
-        if (r == 0) { sh.sm[warp][g] = S.m[nt]; sh.sl[warp][g] = lt; }
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          so[warp][g][16 * mt + r] = fmaf(S.o[nt][mt][0], 1.f / row_factor<BITS>(2 * mt), et);
-          so[warp][g][16 * mt + r + 8] = fmaf(S.o[nt][mt][1], 1.f / row_factor<BITS>(2 * mt + 1), et);
-        }
-      }
-    }
+    if (jl >= 0) state_to_slot<BITS, G, AFFINE>(S, so[warp], sh.sm[warp], sh.sl[warp], lane);
+    if (lane == 0) sh.wseg[warp] = jl;
     __syncthreads();
 
-    // ---- merge the warps of each segment into this CTA's partial for the unit ----
-    {
-      int b0 = 0;
-      for (int jj = 0; jj < nseg; ++jj) {
-        const uint32_t cum = min((uint32_t)(u_first + jj + 1) * NI, x1) - x0;
-        const int b1 = seg_warp_bound<NW>(jj + 1, nseg, cum, len, b0);
-        const int uu = u_first + jj;
-        const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
-        float* part_base = a.partials + ((size_t)uu * c.max_splits + (cta - cta_u0)) * G * PART;
-        for (int e = tid; e < G * D; e += NW * 32) {
-          const int g = e / D, d = e % D;
-          float M = -INFINITY;
-          for (int w = b0; w < b1; ++w) M = fmaxf(M, sh.sm[w][g]);
-          float L = 0.f, O = 0.f;
-          for (int w = b0; w < b1; ++w) {
-            const float f = merge_weight(sh.sm[w][g], M);
-            L = fmaf(sh.sl[w][g], f, L);
-            O = fmaf(so[w][g][d], f, O);
-          }
-          float* part = part_base + (size_t)g * PART;
-          part[d] = O;
-          if (d == 0) { part[D] = M; part[D + 1] = L; }
+    // ---- merge the partials of each segment into this CTA's partial for the unit --
+    if (tid < nseg * G) {   // segment maximum over its warps and boundary slot
+      const int jj = tid / G, g = tid % G;
+      float M = (jj < nseg - 1 && sh.bused[jj]) ? sh.bm[jj][g] : -INFINITY;
+      for (int w = 0; w < NW; ++w)
+        if (sh.wseg[w] == jj) M = fmaxf(M, sh.sm[w][g]);
+      sh.sM[jj][g] = M;
+    }
+    __syncthreads();
+    if (tid < NW * G) {
+      const int w = tid / G, g = tid % G, jw = sh.wseg[w];
+      sh.sf[w][g] = jw >= 0 ? merge_weight(sh.sm[w][g], sh.sM[jw][g]) : 0.f;
+    }
+    if (tid < (nseg - 1) * G) {
+      const int jj = tid / G, g = tid % G;
+      sh.bf[jj][g] = sh.bused[jj] ? merge_weight(sh.bm[jj][g], sh.sM[jj][g]) : 0.f;
+    }
+    __syncthreads();
+    for (int jj = 0; jj < nseg; ++jj) {
+      uint32_t members = 0;   // warps whose final state belongs to segment jj
+      for (int w = 0; w < NW; ++w) members |= (sh.wseg[w] == jj ? 1u : 0u) << w;
+      const bool has_b = jj < nseg - 1 && sh.bused[jj];
+      const int uu = u_first + jj;
+      const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
+      float* part_base = a.partials + ((size_t)uu * c.max_splits + (cta - cta_u0)) * G * PART;
+      for (int e = tid; e < G * D; e += NW * 32) {
+        const int g = e / D, d = e % D;
+        float O = has_b ? sh.bf[jj][g] * sh.bo[jj][g][d] : 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+          if (members >> w & 1u) O = fmaf(so[w][g][d], sh.sf[w][g], O);
+        float* part = part_base + (size_t)g * PART;
+        part[d] = O;
+        if (d == 0) {
+          float L = has_b ? sh.bf[jj][g] * sh.bl[jj][g] : 0.f;
+          for (int w = 0; w < NW; ++w)
+            if (members >> w & 1u) L = fmaf(sh.sl[w][g], sh.sf[w][g], L);
+          part[D] = sh.sM[jj][g];
+          part[D + 1] = L;
         }
-        b0 = b1;
       }
     }
 
