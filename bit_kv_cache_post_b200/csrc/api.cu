@@ -507,7 +507,7 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
           if (kv == 0) {
             const int ks = d / 32, rem = d % 32, h2 = rem / 16, c4 = (rem % 16) / 4, beta = d % 4;
             const int rho = 4 * h2 + ks;
-            wd = word_at(L.k_plane_off[p], pk / 64, (size_t)(pk % 64) * 16 * w + 4 * (c4 * w + rho / F));
+            wd = word_at(L.k_plane_off[p], pk / 64, (size_t)k_row_pos(pk) * 16 * w + 4 * (c4 * w + rho / F));
             bit = 8 * beta + w * (rho % F);
           } else {
             const int mt = d / 16, rem = d % 16, rh = rem / 8, r = rem % 8;

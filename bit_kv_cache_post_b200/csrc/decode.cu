@@ -85,7 +85,8 @@ struct Smem {
   float bo[UMAX - 1][G][D];
   float bm[UMAX - 1][G], bl[UMAX - 1][G], bf[UMAX - 1][G];
   int bused[UMAX - 1];
-  float sM[UMAX][G];                       // per-segment maximum over its partials
+  float sM[UMAX][G], sL[UMAX][G];          // per-segment maximum and weighted sum
+  uint32_t smask[UMAX];                    // warps whose final state belongs to each segment
   int wseg[NW];                            // segment of each warp's final state (-1: none)
   alignas(8) uint64_t bar[NW][NSTAGE];
   int is_last[UMAX];
@@ -358,48 +359,72 @@ __device__ __forceinline__ void packed_block_compute(
   const int nvalid = a.n_packed - blk * PB;  // used when !FULL
 
   // ---- scores ----------------------------------------------------------------
-  // sc[2 mt + th]: score minus the reference in use (m, or 0 while m = -inf)
+  // Lane 4r + c owns tokens 8r .. 8r + 7 of the block (slot j = 2 mt + th is
+  // token 8r + j, row r + 8 th of m-tile mt).  Its K rows sit at positions
+  // 8r + (j ^ (r & 3)) (the cache's row swizzle), which spreads each load
+  // over all shared-memory banks.
+  // sc[j]: score minus the reference in use (m, or 0 while m = -inf)
   float sc[8][NT];
-  float vs[4][2], vo[4][2];
+  float vs[8], vo[8];
   float nm[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) nm[nt] = S.m[nt] == -INFINITY ? 0.f : -S.m[nt];
+  {   // per-token meta of the lane's eight tokens: two 16-byte loads (QuEST)
+    float ks_[8], ko_[8];
+    if constexpr (AFFINE) {
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const KWords<BITS> kw0 = stage_k_words<BITS>(st, 16 * mt + r, c4);
-    const KWords<BITS> kw1 = stage_k_words<BITS>(st, 16 * mt + r + 8, c4);
-    int acc[NT][4];
+      for (int hq = 0; hq < 2; ++hq) {
+        const uint4 km = *reinterpret_cast<const uint4*>(st + SL::K_META + 32 * r + 16 * hq);
+        const uint4 vm = *reinterpret_cast<const uint4*>(st + SL::V_META + 32 * r + 16 * hq);
+        const uint32_t kw[4] = {km.x, km.y, km.z, km.w}, vw[4] = {vm.x, vm.y, vm.z, vm.w};
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+          const float2 vf = __half22float2(*reinterpret_cast<const __half2*>(&vw[e]));
+          ks_[4 * hq + e] = kf.x; ko_[4 * hq + e] = kf.y;
+          vs[4 * hq + e] = vf.x; vo[4 * hq + e] = vf.y;
+        }
+      }
+    } else {
+      const uint4 km = *reinterpret_cast<const uint4*>(st + SL::K_META + 16 * r);
+      const uint4 vm = *reinterpret_cast<const uint4*>(st + SL::V_META + 16 * r);
+      const uint32_t kw[4] = {km.x, km.y, km.z, km.w}, vw[4] = {vm.x, vm.y, vm.z, vm.w};
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t a0 = k_frag<BITS>(kw0, ks, 0), a1 = k_frag<BITS>(kw1, ks, 0);
-      const uint32_t a2 = k_frag<BITS>(kw0, ks, 1), a3 = k_frag<BITS>(kw1, ks, 1);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+      for (int e = 0; e < 4; ++e) {
+        const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
+        const float2 vf = __half22float2(*reinterpret_cast<const __half2*>(&vw[e]));
+        ks_[2 * e] = kf.x; ks_[2 * e + 1] = kf.y;
+        vs[2 * e] = vf.x; vs[2 * e + 1] = vf.y;
+        ko_[2 * e] = ko_[2 * e + 1] = vo[2 * e] = vo[2 * e + 1] = 0.f;
+      }
     }
+    const int x = r & 3;
 #pragma unroll
-    for (int th = 0; th < 2; ++th) {
-      const int t = 16 * mt + r + 8 * th;
-      float ks_, ko_;
-      if constexpr (AFFINE) {
-        const float2 km = __half22float2(*reinterpret_cast<const __half2*>(st + SL::K_META + 4 * t));
-        const float2 vm = __half22float2(*reinterpret_cast<const __half2*>(st + SL::V_META + 4 * t));
-        ks_ = km.x; ko_ = km.y; vs[mt][th] = vm.x; vo[mt][th] = vm.y;
-      } else {
-        ks_ = __half2float(*reinterpret_cast<const __half*>(st + SL::K_META + 2 * t));
-        ko_ = 0.f;
-        vs[mt][th] = __half2float(*reinterpret_cast<const __half*>(st + SL::V_META + 2 * t));
-        vo[mt][th] = 0.f;
+    for (int mt = 0; mt < 4; ++mt) {
+      const KWords<BITS> kw0 = stage_k_words<BITS>(st, 8 * r + ((2 * mt) ^ x), c4);
+      const KWords<BITS> kw1 = stage_k_words<BITS>(st, 8 * r + ((2 * mt + 1) ^ x), c4);
+      int acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint32_t a0 = k_frag<BITS>(kw0, ks, 0), a1 = k_frag<BITS>(kw1, ks, 0);
+        const uint32_t a2 = k_frag<BITS>(kw0, ks, 1), a3 = k_frag<BITS>(kw1, ks, 1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
       }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float xf = (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
-        float d;   // score minus the reference maximum in use
-        if constexpr (AFFINE) d = fmaf(ks_, qscale[nt] * xf, fmaf(ko_, qsum[nt], nm[nt]));
-        else d = fmaf(ks_, fmaf(qscale[nt], xf, qoff[nt]), nm[nt]);   // delta (q.c + beta sum q) - m
-        if constexpr (!FULL) d = (t < nvalid) ? d : -INFINITY;
-        sc[2 * mt + th][nt] = d;
+      for (int th = 0; th < 2; ++th) {
+        const int j = 2 * mt + th;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float xf = (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
+          float d;   // score minus the reference maximum in use
+          if constexpr (AFFINE) d = fmaf(ks_[j], qscale[nt] * xf, fmaf(ko_[j], qsum[nt], nm[nt]));
+          else d = fmaf(ks_[j], fmaf(qscale[nt], xf, qoff[nt]), nm[nt]);   // delta (q.c + beta sum q) - m
+          if constexpr (!FULL) d = (8 * r + j < nvalid) ? d : -INFINITY;
+          sc[j][nt] = d;
+        }
       }
     }
   }
@@ -428,18 +453,16 @@ __device__ __forceinline__ void packed_block_compute(
   for (int nt = 0; nt < NT; ++nt) {
     float ls = 0.f, es = 0.f, pm = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int th = 0; th < 2; ++th) {
-        const float p = ex2(sc[2 * mt + th][nt]);   // masked tokens: exp2(-inf) = 0
-        float pt = p * vs[mt][th];
-        if constexpr (!FULL) pt = (16 * mt + r + 8 * th < nvalid) ? pt : 0.f;
-        ls += p;
-        if constexpr (AFFINE) es = fmaf(p, vo[mt][th], es);
-        else es += pt;                                 // times beta at the end
-        pm = fmaxf(pm, pt);
-        sc[2 * mt + th][nt] = pt;
-      }
+    for (int j = 0; j < 8; ++j) {
+      const float p = ex2(sc[j][nt]);   // masked tokens: exp2(-inf) = 0
+      float pt = p * vs[j];
+      if constexpr (!FULL) pt = (8 * r + j < nvalid) ? pt : 0.f;
+      ls += p;
+      if constexpr (AFFINE) es = fmaf(p, vo[j], es);
+      else es += pt;                                 // times beta at the end
+      pm = fmaxf(pm, pt);
+      sc[j][nt] = pt;
+    }
     S.l[nt] += ls;
     S.e[nt] += es;
     pmx[nt] = pm;
@@ -469,18 +492,23 @@ __device__ __forceinline__ void packed_block_compute(
     float inv = 0.f;
     if (S.F[nt] > 0.f)
       inv = KEEP ? 65535.f * __int_as_float(0x7F000000 - __float_as_int(S.F[nt])) : 65535.f * __frcp_rn(S.F[nt]);
+    // 1.5 * 2^23 + rint(pt * 65535 / F): the low 16 mantissa bits are the
+    // rounded value; its high byte is term 0, its low byte term 1.  Bytes of
+    // four tokens are gathered into one word per term.
+    uint32_t bw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) bw[j] = __float_as_uint(fmaf(sc[j][nt], inv, 12582912.f));
+    uint32_t t0w[2], t1w[2];
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      const uint32_t x01 = __byte_perm(bw[4 * hq], bw[4 * hq + 1], 0x5140);      // lo0 lo1 hi0 hi1
+      const uint32_t x23 = __byte_perm(bw[4 * hq + 2], bw[4 * hq + 3], 0x5140);  // lo2 lo3 hi2 hi3
+      t1w[hq] = __byte_perm(x01, x23, 0x5410);
+      t0w[hq] = __byte_perm(x01, x23, 0x7632);
+    }
     const int col = nt * 8 + 2 * c4;
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int th = 0; th < 2; ++th) {
-        // 1.5 * 2^23 + rint(pt * 65535 / F): the low 16 mantissa bits are the
-        // rounded value; its high byte is term 0, its low byte term 1.
-        const uint32_t bits = __float_as_uint(fmaf(sc[2 * mt + th][nt], inv, 12582912.f));
-        const int t = 16 * mt + r + 8 * th;
-        ps[col * PS_LD + t] = (uint8_t)(bits >> 8);
-        ps[(col + 1) * PS_LD + t] = (uint8_t)bits;
-      }
+    *reinterpret_cast<uint2*>(ps + col * PS_LD + 8 * r) = make_uint2(t0w[0], t0w[1]);
+    *reinterpret_cast<uint2*>(ps + (col + 1) * PS_LD + 8 * r) = make_uint2(t1w[0], t1w[1]);
   }
   __syncwarp();
 
@@ -889,26 +917,32 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     __syncthreads();
 
     // ---- merge the partials of each segment into this CTA's partial for the unit --
-    if (tid < nseg * G) {   // segment maximum over its warps and boundary slot
+    // thread (segment, head): the segment's maximum over its warps and its
+    // boundary slot, then every member's merge weight against it
+    if (tid < nseg * G) {
       const int jj = tid / G, g = tid % G;
-      float M = (jj < nseg - 1 && sh.bused[jj]) ? sh.bm[jj][g] : -INFINITY;
+      const bool has_b = jj < nseg - 1 && sh.bused[jj];
+      float M = has_b ? sh.bm[jj][g] : -INFINITY;
+      uint32_t members = 0;
+#pragma unroll
       for (int w = 0; w < NW; ++w)
-        if (sh.wseg[w] == jj) M = fmaxf(M, sh.sm[w][g]);
+        if (sh.wseg[w] == jj) { M = fmaxf(M, sh.sm[w][g]); members |= 1u << w; }
+      float L = has_b ? sh.bl[jj][g] * merge_weight(sh.bm[jj][g], M) : 0.f;
+      if (jj < nseg - 1) sh.bf[jj][g] = has_b ? merge_weight(sh.bm[jj][g], M) : 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        if (members >> w & 1u) {
+          const float f = merge_weight(sh.sm[w][g], M);
+          sh.sf[w][g] = f;
+          L = fmaf(sh.sl[w][g], f, L);
+        }
       sh.sM[jj][g] = M;
-    }
-    __syncthreads();
-    if (tid < NW * G) {
-      const int w = tid / G, g = tid % G, jw = sh.wseg[w];
-      sh.sf[w][g] = jw >= 0 ? merge_weight(sh.sm[w][g], sh.sM[jw][g]) : 0.f;
-    }
-    if (tid < (nseg - 1) * G) {
-      const int jj = tid / G, g = tid % G;
-      sh.bf[jj][g] = sh.bused[jj] ? merge_weight(sh.bm[jj][g], sh.sM[jj][g]) : 0.f;
+      sh.sL[jj][g] = L;
+      if (g == 0) sh.smask[jj] = members;
     }
     __syncthreads();
     for (int jj = 0; jj < nseg; ++jj) {
-      uint32_t members = 0;   // warps whose final state belongs to segment jj
-      for (int w = 0; w < NW; ++w) members |= (sh.wseg[w] == jj ? 1u : 0u) << w;
+      const uint32_t members = sh.smask[jj];
       const bool has_b = jj < nseg - 1 && sh.bused[jj];
       const int uu = u_first + jj;
       const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
@@ -921,13 +955,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
           if (members >> w & 1u) O = fmaf(so[w][g][d], sh.sf[w][g], O);
         float* part = part_base + (size_t)g * PART;
         part[d] = O;
-        if (d == 0) {
-          float L = has_b ? sh.bf[jj][g] * sh.bl[jj][g] : 0.f;
-          for (int w = 0; w < NW; ++w)
-            if (members >> w & 1u) L = fmaf(sh.sl[w][g], sh.sf[w][g], L);
-          part[D] = sh.sM[jj][g];
-          part[D + 1] = L;
-        }
+        if (d == 0) { part[D] = sh.sM[jj][g]; part[D + 1] = sh.sL[jj][g]; }
       }
     }
 
@@ -954,10 +982,9 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
       const uint32_t ubj = (uint32_t)uu * NI;
       const int nparts = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj)) + 1;
       const float* pbase = a.partials + (size_t)uu * c.max_splits * G * PART + (size_t)g * PART;
-      float M = -INFINITY;
-      for (int sp = lane; sp < nparts; sp += 32) M = fmaxf(M, __ldcg(pbase + (size_t)sp * G * PART + D));
-      M = warp_max_f32(M);
-      float L = 0.f;
+      // partials in rounds of eight, all loads of a round in flight at once;
+      // the running (M, L, O) is rescaled when a round raises M
+      float M = -INFINITY, L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sp0 = 0; sp0 < nparts; sp0 += 8) {
         float4 v[8];
@@ -970,6 +997,13 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
           mw[q] = ok ? __ldcg(part + D) : -INFINITY;
           lw[q] = ok ? __ldcg(part + D + 1) : 0.f;
         }
+        float Mr = M;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) Mr = fmaxf(Mr, mw[q]);
+        const float fr = merge_weight(M, Mr);
+        L *= fr;
+        O.x *= fr; O.y *= fr; O.z *= fr; O.w *= fr;
+        M = Mr;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float f = merge_weight(mw[q], M);

@@ -48,10 +48,18 @@ struct DevCache {
 // Packed tokens per block record.
 constexpr int PACK_BLOCK_TOKENS = 64;
 
+// Row position of packed token pk inside its 64-token block: token 8r + j of
+// the block sits at row 8r + (j ^ (r & 3)), so that the decode's reads of
+// one row per octet r fall on all shared-memory banks.
+__host__ __device__ __forceinline__ int k_row_pos(int64_t pk) {
+  const int i = (int)(pk & 63);
+  return (i & ~7) | ((i & 7) ^ ((i >> 3) & 3));
+}
+
 // Address of the K row (16 w bytes, plane p) of packed token pk of unit u.
 __host__ __device__ __forceinline__ uint8_t* k_row_at(const DevCache& c, int p, int64_t u, int64_t pk) {
   return c.k_plane[p] + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
-         (uint64_t)(pk & 63) * 16 * c.plane_bits[p];
+         (uint64_t)k_row_pos(pk) * 16 * c.plane_bits[p];
 }
 // Address of V quad `quad` (tokens 4 quad .. 4 quad + 3; 64 w bytes, plane p) of unit u.
 __host__ __device__ __forceinline__ uint8_t* v_quad_at(const DevCache& c, int p, int64_t u, int64_t quad) {

@@ -99,8 +99,10 @@ typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
  *     copy fetches everything the decode needs for those tokens.
  *     k_plane_off[p], v_plane_off[p], k_meta_off and v_meta_off are the
  *     offsets of these parts in unit 0's block 0; block b of unit u adds
- *     u * unit_stride + b * block_stride.  Within a record, K rows of packed
- *     token b * 64 + i sit at 16 * w * i, V quads b * 16 + q at 64 * w * q,
+ *     u * unit_stride + b * block_stride.  Within a record, the K row of
+ *     packed token b * 64 + i sits at 16 * w * pos(i) with the row swizzle
+ *     pos(i) = (i & 56) | ((i & 7) ^ ((i >> 3) & 3)) (spreads the decode's
+ *     shared-memory reads over all banks), V quads b * 16 + q at 64 * w * q,
  *     meta entries at meta_bytes * i.
  * Formats:
  *   planes: 2-bit codes -> one 2-bit plane, 4-bit -> one 4-bit plane, 3-bit

@@ -49,9 +49,16 @@ def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
     for p in range(L.n_planes):
         w = L.plane_bits[p]
         off = L.k_plane_off[p] if kv == 0 else L.v_plane_off[p]
-        part = blocks[:, off:off + 64 * 16 * w].reshape(-1)[:n_packed * 16 * w]
-        raw = np.ascontiguousarray(part).view(np.uint32)
-        out.append(raw.reshape(n_packed, 4 * w) if kv == 0 else raw.reshape(n_packed // 4, 16 * w))
+        part = np.ascontiguousarray(blocks[:, off:off + 64 * 16 * w]).view(np.uint32)
+        if kv == 0:
+            # K rows sit at the swizzled position 8r + (j ^ (r & 3)) of token
+            # 8r + j of each 64-token block
+            rows = part.reshape(-1, 64, 4 * w)
+            i = np.arange(64)
+            pos = (i & ~7) | ((i & 7) ^ ((i >> 3) & 3))
+            out.append(rows[:, pos].reshape(-1, 4 * w)[:n_packed])
+        else:
+            out.append(part.reshape(-1)[:n_packed * 4 * w].reshape(n_packed // 4, 16 * w))
     return out
 
 
