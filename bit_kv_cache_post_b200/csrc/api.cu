@@ -335,22 +335,49 @@ wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t* n_tokens, 
   return WUSHKV_OK;
 }
 
-wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
-                            int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
-                            int32_t quantizer, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Launch plan of one append: FMA-kernel quad ranges (one, or two when new
+// tokens reuse ring slots that old flushed tokens are read from) and the
+// optional tensor-core bulk kernel.
+struct AppendPlan {
+  AppendArgs a;
+  int64_t range[2][2];
+  int nranges;
+  bool tc;
+  PrefillArgs pf;
+  int64_t n1;
+};
+
+// Per-CTA quad count of an FMA-kernel range: enough CTAs to fill the GPU,
+// up to 64 quads (256 tokens) per CTA.
+void set_quad_range(AppendArgs& a, int64_t qa, int64_t qb) {
+  a.quad_begin = qa;
+  a.n_quads = qb - qa;
+  int64_t per = (a.n_quads * a.c.units) / 1184;
+  if (per < 1) per = 1;
+  if (per > 64) per = 64;
+  a.quads_per_cta = (int)per;
+}
+
+wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev, int32_t in_dtype,
+                          const float* T_k_dev, int32_t n_tok, int32_t bits, int32_t quantizer,
+                          AppendPlan* p) {
   if (!cache || !k_rope_dev || !v_dev || !valid_dtype(in_dtype) || n_tok < 0) return WUSHKV_EINVAL;
   if (reinterpret_cast<uintptr_t>(T_k_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   const wushkv_config& c = cache->cfg;
   if (bits != c.bits || quantizer != c.quantizer) return WUSHKV_EINVAL;
-  if (n_tok == 0) return WUSHKV_OK;
   if (cache->n + n_tok > c.max_ctx) return WUSHKV_ECAPACITY;
+  std::memset(p, 0, sizeof(*p));
   const int64_t n0 = cache->n, n1 = n0 + n_tok;
+  p->n1 = n1;
+  if (n_tok == 0) return WUSHKV_OK;
   const int64_t S = c.sink, W = c.recent + c.chunk;
   const int64_t P0 = packed_count(n0, c), P1 = packed_count(n1, c);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  AppendArgs a;
-  std::memset(&a, 0, sizeof(a));
+  AppendArgs& a = p->a;
   a.c = dev_view(cache);
   a.k = k_rope_dev;
   a.v = v_dev;
@@ -366,47 +393,35 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
   const bool has_old_flush = (P1 > P0) && (S + P0 < n0);
   const int64_t first = has_old_flush ? S + P0 : n0;
   const int64_t q_begin = first / 4, q_end = (n1 + 3) / 4;
-  const int units = (int)((int64_t)c.batch * c.n_kv_heads);
 
   // A bf16 block with a transform goes to the tensor-core key kernel and the
   // value kernel from the first quad boundary at or after n0 to the end;
   // the FMA kernel keeps the flush of old ring rows and the partial quad.
   const int64_t ta = (n0 + 3) / 4 * 4;
   const uintptr_t kv_addr = reinterpret_cast<uintptr_t>(k_rope_dev) | reinterpret_cast<uintptr_t>(v_dev);
-  const bool tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && n1 - ta >= TC_MIN_TOKENS &&
-                  (kv_addr & 15) == 0 && (int64_t)c.batch * n_tok < 2147483647LL &&
-                  (c.quantizer == WUSHKV_QUEST_INT || (c.clip_lo_rank <= 2 && c.clip_hi_rank >= 127));
-  const int64_t tc_qa = tc ? ta / 4 : 0;
-
-  auto launch_one = [&](int64_t qa, int64_t qb) -> cudaError_t {
-    if (qb <= qa) return cudaSuccess;
-    a.quad_begin = qa;
-    a.n_quads = qb - qa;
-    // enough CTAs to fill the GPU, up to 64 quads (256 tokens) per CTA
-    int64_t per = (a.n_quads * units) / 1184;
-    if (per < 1) per = 1;
-    if (per > 64) per = 64;
-    a.quads_per_cta = (int)per;
-    return launch_append(a, s);
-  };
+  p->tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && n1 - ta >= TC_MIN_TOKENS &&
+          (kv_addr & 15) == 0 && (int64_t)c.batch * n_tok < 2147483647LL &&
+          (c.quantizer == WUSHKV_QUEST_INT || (c.clip_lo_rank <= 2 && c.clip_hi_rank >= 127));
+  const int64_t tc_qa = p->tc ? ta / 4 : 0;
   // the FMA kernel takes every quad before the tensor-core range
-  auto launch = [&](int64_t qa, int64_t qb) -> cudaError_t {
-    return launch_one(qa, tc && qb > tc_qa ? tc_qa : qb);
+  auto add = [&](int64_t qa, int64_t qb) {
+    if (p->tc && qb > tc_qa) qb = tc_qa;
+    if (qb <= qa) return;
+    p->range[p->nranges][0] = qa;
+    p->range[p->nranges][1] = qb;
+    ++p->nranges;
   };
-
-  cudaError_t e;
   // New tokens may reuse ring slots that old flushed tokens are read from
   // only when the touched span exceeds the ring; then flush first.
   if (has_old_flush && (n1 - (S + P0) > W)) {
     const int64_t q_mid = (flush_end + 3) / 4;
-    e = launch(q_begin, q_mid);
-    if (e == cudaSuccess) e = launch(q_mid, q_end);
+    add(q_begin, q_mid);
+    add(q_mid, q_end);
   } else {
-    e = launch(q_begin, q_end);
+    add(q_begin, q_end);
   }
-  if (e == cudaSuccess && tc) {
-    PrefillArgs pf;
-    std::memset(&pf, 0, sizeof(pf));
+  if (p->tc) {
+    PrefillArgs& pf = p->pf;
     pf.c = a.c;
     pf.T = T_k_dev;
     pf.n_tok = n_tok;
@@ -423,34 +438,103 @@ wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const v
     if (per_head > by_work) per_head = by_work;
     if (per_head < 1) per_head = 1;
     pf.ctas_per_head = (int)per_head;
-    e = launch_prefill_tc(pf, k_rope_dev, v_dev, device_sms(), s);
   }
-  if (e != cudaSuccess) return WUSHKV_ECUDA;
-  cache->n = n1;
   return WUSHKV_OK;
 }
 
-wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
-                                     float* q_out_dev, int32_t batch, int32_t n_q_heads,
-                                     int32_t n_kv_heads, void* stream) {
+cudaError_t run_append(AppendPlan& p, const void* k_rope_dev, const void* v_dev, cudaStream_t s) {
+  for (int r = 0; r < p.nranges; ++r) {
+    set_quad_range(p.a, p.range[r][0], p.range[r][1]);
+    const cudaError_t e = launch_append(p.a, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (p.tc) return launch_prefill_tc(p.pf, k_rope_dev, v_dev, device_sms(), s);
+  return cudaSuccess;
+}
+
+wushkv_status check_query_args(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
+                               const float* q_out_dev, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads) {
   if (!q_dev || !T_k_invT_dev || !q_out_dev || !valid_dtype(q_dtype)) return WUSHKV_EINVAL;
   if (reinterpret_cast<uintptr_t>(T_k_invT_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads) return WUSHKV_EINVAL;
   const int g = n_q_heads / n_kv_heads;
   if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16) return WUSHKV_EUNSUPPORTED;
   if ((int64_t)batch * n_kv_heads > 2147483647LL) return WUSHKV_EUNSUPPORTED;
+  return WUSHKV_OK;
+}
+
+wushkv_status check_decode_args(const float* q_prime_dev, const wushkv_cache* cache, const float* out_dev,
+                                float scale) {
+  if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(out_dev) | reinterpret_cast<uintptr_t>(q_prime_dev)) & 15)
+    return WUSHKV_EINVAL;  // read and written as float4
+  if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
+  return WUSHKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                            int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
+                            int32_t quantizer, void* stream) {
+  AppendPlan p;
+  const wushkv_status st = plan_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, n_tok, bits, quantizer, &p);
+  if (st != WUSHKV_OK || n_tok == 0) return st;
+  if (run_append(p, k_rope_dev, v_dev, static_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSHKV_ECUDA;
+  cache->n = p.n1;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                 int32_t in_dtype, const float* T_k_dev, const void* q_dev, int32_t q_dtype,
+                                 const float* T_k_invT_dev, float* q_prime_dev, float* out_dev, float scale,
+                                 void* stream) {
+  if (!cache) return WUSHKV_EINVAL;
+  const wushkv_config& c = cache->cfg;
+  wushkv_status st = check_query_args(q_dev, q_dtype, T_k_invT_dev, q_prime_dev, c.batch, c.n_q_heads,
+                                      c.n_kv_heads);
+  if (st != WUSHKV_OK) return st;
+  st = check_decode_args(q_prime_dev, cache, out_dev, scale);
+  if (st != WUSHKV_OK) return st;
+  AppendPlan p;
+  st = plan_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, 1, c.bits, c.quantizer, &p);
+  if (st != WUSHKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!p.tc && p.nranges == 1) {   // one launch for the append and the query transform
+    set_quad_range(p.a, p.range[0][0], p.range[0][1]);
+    e = launch_append_qt(p.a, q_dev, q_dtype, T_k_invT_dev, q_prime_dev, s);
+  } else {
+    e = run_append(p, k_rope_dev, v_dev, s);
+    if (e == cudaSuccess)
+      e = launch_query_transform(q_dev, q_dtype, T_k_invT_dev, q_prime_dev, c.batch, c.n_q_heads,
+                                 c.n_kv_heads, s);
+  }
+  if (e != cudaSuccess) return WUSHKV_ECUDA;
+  cache->n = p.n1;
+  DecodeArgs a;
+  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  if (st != WUSHKV_OK) return st;
+  return cuda_status(launch_decode(a, cache->wmaps, s));
+}
+
+wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
+                                     float* q_out_dev, int32_t batch, int32_t n_q_heads,
+                                     int32_t n_kv_heads, void* stream) {
+  const wushkv_status st = check_query_args(q_dev, q_dtype, T_k_invT_dev, q_out_dev, batch, n_q_heads, n_kv_heads);
+  if (st != WUSHKV_OK) return st;
   return cuda_status(launch_query_transform(q_dev, q_dtype, T_k_invT_dev, q_out_dev, batch,
                                             n_q_heads, n_kv_heads, static_cast<cudaStream_t>(stream)));
 }
 
 wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream) {
-  if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(out_dev) | reinterpret_cast<uintptr_t>(q_prime_dev)) & 15)
-    return WUSHKV_EINVAL;  // read and written as float4
-  if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
+  wushkv_status st = check_decode_args(q_prime_dev, cache, out_dev, scale);
+  if (st != WUSHKV_OK) return st;
   DecodeArgs a;
-  const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
   if (st != WUSHKV_OK) return st;
   return cuda_status(launch_decode(a, cache->wmaps, static_cast<cudaStream_t>(stream)));
 }

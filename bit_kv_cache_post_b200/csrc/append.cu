@@ -30,24 +30,27 @@ __device__ __forceinline__ float round_f16(float x) { return __half2float(__floa
 // Token classes inside one append.
 enum : int { TOK_SKIP = 0, TOK_NEW = 1, TOK_FLUSH_OLD = 2 };
 
-__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* Tt = reinterpret_cast<float*>(smem_raw);          // [128][TT_LD] = T^T
-  float* kin = Tt + D * TT_LD;                             // [4][128] raw keys
+// Shared memory of one append CTA: staging vectors first, then (only when
+// the CTA stages the transform) T^T.
+constexpr size_t APPEND_VEC_BYTES = (size_t)3 * 4 * D * sizeof(float) + 4 * D + 16;
+
+// One append CTA: quads blockIdx-slice bx of unit u.
+__device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int u, unsigned char* smem_raw) {
+  float* kin = reinterpret_cast<float*>(smem_raw);         // [4][128] raw keys
   float* k16 = kin + 4 * D;                                // [4][128] fp16 keys
   float* v16 = k16 + 4 * D;                                // [4][128] fp16 values
   uint8_t* codes = reinterpret_cast<uint8_t*>(v16 + 4 * D);  // [4][128]
-  __shared__ int kind_s[4];
+  int* kind_s = reinterpret_cast<int*>(codes + 4 * D);     // [4]
+  float* Tt = reinterpret_cast<float*>(smem_raw + APPEND_VEC_BYTES);  // [128][TT_LD] = T^T
 
   const DevCache& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u = blockIdx.y;
   const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
   const int64_t n0 = a.n0, n1 = a.n0 + a.n_tok;
   const int64_t S = c.sink, P0 = a.packed0, P1 = a.packed1;
   const int W = c.ring_slots;
 
-  const int64_t q_first = a.quad_begin + (int64_t)blockIdx.x * a.quads_per_cta;
+  const int64_t q_first = a.quad_begin + bx * a.quads_per_cta;
   const int64_t q_last = min(q_first + a.quads_per_cta, a.quad_begin + a.n_quads);
   if (q_first >= q_last) return;
 
@@ -178,27 +181,82 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   }
 }
 
-}  // namespace
-
-size_t append_smem_bytes() {
-  return (size_t)(D * TT_LD + 3 * 4 * D) * sizeof(float) + 4 * D;
+__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  append_body(a, blockIdx.x, blockIdx.y, smem_raw);
 }
 
+// The append of a decode step and the query transform of the same step in
+// one launch: slices x < gx of row u are the append CTAs of unit u, slice gx
+// transforms the unit's G queries.
+template <int G>
+__global__ void __launch_bounds__(128) append_qt_kernel(AppendArgs a, int gx, const void* q, int q_dtype,
+                                                        const float* TinvT, float* q_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  if ((int)blockIdx.x < gx) {
+    append_body(a, blockIdx.x, blockIdx.y, smem_raw);
+  } else {
+    const int u = blockIdx.y;
+    query_transform_unit<G>(q, q_dtype, TinvT, q_out, u / a.c.n_kv_heads, u % a.c.n_kv_heads,
+                            a.c.n_kv_heads, reinterpret_cast<float*>(smem_raw));
+  }
+}
+
+// Dynamic shared memory of an append launch: T^T only when a CTA transforms
+// several quads.
+size_t append_smem(const AppendArgs& a) {
+  const bool staged = a.T != nullptr && a.quads_per_cta > 1;
+  return APPEND_VEC_BYTES + (staged ? (size_t)D * TT_LD * sizeof(float) : 0);
+}
+
+cudaError_t set_smem_attr(const void* fn, size_t bytes) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+size_t append_smem_bytes() { return APPEND_VEC_BYTES + (size_t)D * TT_LD * sizeof(float); }
+
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
-  const size_t smem = append_smem_bytes();
   int dev = 0;
   cudaGetDevice(&dev);
   static int attr_done[64] = {0};
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = set_smem_attr((const void*)append_kernel, append_smem_bytes());
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
   if (a.n_quads <= 0) return cudaSuccess;
   const int64_t gx = (a.n_quads + a.quads_per_cta - 1) / a.quads_per_cta;
   dim3 grid((unsigned)gx, (unsigned)a.c.units);
-  append_kernel<<<grid, 128, smem, s>>>(a);
+  append_kernel<<<grid, 128, append_smem(a), s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, const float* TinvT,
+                             float* q_out, cudaStream_t s) {
+  const int G = a.c.group;
+  const void* fn = G == 1 ? (const void*)append_qt_kernel<1> : G == 2 ? (const void*)append_qt_kernel<2>
+                   : G == 4 ? (const void*)append_qt_kernel<4> : (const void*)append_qt_kernel<8>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int attr_done[64][4] = {};
+  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+  if (dev < 64 && !attr_done[dev][gi]) {
+    cudaError_t e = set_smem_attr(fn, append_smem_bytes());
+    if (e != cudaSuccess) return e;
+    attr_done[dev][gi] = 1;
+  }
+  const int64_t gx = a.n_quads > 0 ? (a.n_quads + a.quads_per_cta - 1) / a.quads_per_cta : 0;
+  dim3 grid((unsigned)gx + 1, (unsigned)a.c.units);
+  const size_t smem = append_smem(a) > (size_t)G * D * sizeof(float) ? append_smem(a) : (size_t)G * D * sizeof(float);
+  switch (G) {
+    case 1: append_qt_kernel<1><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
+    case 2: append_qt_kernel<2><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
+    case 4: append_qt_kernel<4><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
+    case 8: append_qt_kernel<8><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -10,30 +10,13 @@ namespace wushkv {
 
 namespace {
 
-__device__ __forceinline__ float load_q(const void* p, int dtype, size_t i) {
-  if (dtype == WUSHKV_F16) return __half2float(static_cast<const __half*>(p)[i]);
-  if (dtype == WUSHKV_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
-  return static_cast<const float*>(p)[i];
-}
-
 template <int G>
 __global__ void __launch_bounds__(128) qtransform_kernel(const void* q, int dtype,
                                                          const float* TinvT, float* out,
                                                          int n_kv_heads) {
   __shared__ __align__(16) float qs[G][D];
-  const int Hq = n_kv_heads * G;
-  const int b = blockIdx.x / n_kv_heads, h = blockIdx.x % n_kv_heads;
-  const int tid = threadIdx.x;
-  MatRow row;
-  load_row(TinvT + (size_t)h * D * D, tid, row);
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-    qs[g][tid] = load_q(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
-  __syncthreads();
-  float dots[G];
-  row_dots<G>(row, &qs[0][0], dots);
-#pragma unroll
-  for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = dots[g];
+  query_transform_unit<G>(q, dtype, TinvT, out, blockIdx.x / n_kv_heads, blockIdx.x % n_kv_heads,
+                          n_kv_heads, &qs[0][0]);
 }
 
 }  // namespace

@@ -171,6 +171,35 @@ __device__ __forceinline__ void row_dots(const MatRow& r, const float* x, float 
   }
 }
 
+// Query transform of one (sequence b, KV head h) group on a 128-thread CTA:
+// q'[g][i] = sum_j M[i][j] q[g][j] for the G query heads of the group, M =
+// T_k^{-T} of head h (summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
+// 方法关键点 and 工作参考价值: one d x d product per query; the inverse
+// transpose keeps q'.k' = q.k).  Thread i streams row i of M against the G
+// query vectors staged in qs ([G][128] floats of shared memory).
+__device__ __forceinline__ float load_any(const void* p, int dtype, size_t i) {
+  if (dtype == WUSHKV_F16) return __half2float(static_cast<const __half*>(p)[i]);
+  if (dtype == WUSHKV_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  return static_cast<const float*>(p)[i];
+}
+
+template <int G>
+__device__ __forceinline__ void query_transform_unit(const void* q, int dtype, const float* TinvT, float* out,
+                                                     int b, int h, int n_kv_heads, float* qs) {
+  const int Hq = n_kv_heads * G;
+  const int tid = threadIdx.x;
+  MatRow row;
+  load_row(TinvT + (size_t)h * D * D, tid, row);
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    qs[g * D + tid] = load_any(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
+  __syncthreads();
+  float dots[G];
+  row_dots<G>(row, qs, dots);
+#pragma unroll
+  for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = dots[g];
+}
+
 // ---------------------------------------------------------------------------
 // Per-token quantisers on one warp.  Lane l holds dims 4l..4l+3 of the token
 // as float values that are exactly fp16 values.
@@ -310,6 +339,10 @@ struct AppendArgs {
   int quads_per_cta;
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+// The append launch of a (single-phase, FMA-path) decode-step append fused
+// with the query transform of the step (q_out = T_k^{-T} q per query head).
+cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, const float* TinvT,
+                             float* q_out, cudaStream_t s);
 
 // Bulk append on the tensor cores: every token t in [ta, tb) of every unit
 // comes straight from the bf16 input (keys through T) and goes to the fp16

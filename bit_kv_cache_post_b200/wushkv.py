@@ -20,7 +20,7 @@ EXPORTED = [
     "wushkv_cache_bytes", "wushkv_cache_create", "wushkv_cache_destroy", "wushkv_cache_layout",
     "wushkv_cache_tokens", "wushkv_append", "wushkv_query_transform", "wushkv_decode",
     "wushkv_export", "wushkv_device_status", "wushkv_default_quest_alpha", "wushkv_strerror",
-    "wushkv_decode_noalloc",
+    "wushkv_decode_noalloc", "wushkv_decode_step",
 ]
 
 
@@ -79,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_query_transform.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp]
     lib.wushkv_decode.argtypes = [vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_decode_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, vp]
+    lib.wushkv_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_export.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.wushkv_device_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
     lib.wushkv_default_quest_alpha.argtypes = [i32]
@@ -97,15 +98,22 @@ def _check(status: int, what: str):
         raise WushKVError(status, what)
 
 
+_DTYPES = None
+
+
 def _dtype_code(t) -> int:
-    import torch
-    return {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}[t.dtype]
+    global _DTYPES
+    if _DTYPES is None:
+        import torch
+        _DTYPES = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+    return _DTYPES[t.dtype]
 
 
 def _stream_ptr(stream) -> int | None:
-    import torch
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream or None
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream or None
 
 
 def make_config(batch, n_kv_heads, n_q_heads, max_ctx, bits=2, quantizer=QUEST_INT, sink=64,
@@ -196,6 +204,23 @@ class Cache:
             out = torch.empty_like(q_prime)
         _check(load().wushkv_decode(q_prime.data_ptr(), self._handle, out.data_ptr(), scale,
                                     _stream_ptr(stream)), "wushkv_decode")
+        return out
+
+    def decode_step(self, k, v, T, q, TinvT, q_prime=None, out=None, scale: float = 0.0, stream=None):
+        """Append one token per sequence (k, v: [B, 1, Hkv, 128]), transform
+        the queries (q: [B, Hq, 128]) into q_prime and decode them; returns
+        out ([B, Hq, 128] fp32)."""
+        import torch
+        assert k.is_contiguous() and v.is_contiguous() and q.is_contiguous() and TinvT.is_contiguous()
+        assert k.shape == v.shape and k.shape[1] == 1 and T is not None and T.is_contiguous()
+        if q_prime is None:
+            q_prime = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        _check(load().wushkv_decode_step(self._handle, k.data_ptr(), v.data_ptr(), _dtype_code(k),
+                                         T.data_ptr(), q.data_ptr(), _dtype_code(q), TinvT.data_ptr(),
+                                         q_prime.data_ptr(), out.data_ptr(), scale, _stream_ptr(stream)),
+               "wushkv_decode_step")
         return out
 
     def decode_noalloc(self, q_prime, out=None, scale: float = 0.0, stream=None):

@@ -206,6 +206,28 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
 WUSHKV_API wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream);
 
+/* One decode step: append one token to every sequence (wushkv_append with
+ * n_tok = 1), transform the step's queries (wushkv_query_transform into
+ * q_prime_dev) and decode them (wushkv_decode), in stream order.
+ *   Source: the three calls above; the pages describe the step as append
+ *   with the key transform, the query-side transform and attention over the
+ *   packed cache plus the fp16 windows (summary page 方法关键点).
+ *   k_rope_dev, v_dev: [batch][1][n_kv_heads][128], dtype in_dtype.
+ *   T_k_dev: as wushkv_append.  q_dev: [batch][n_q_heads][128], dtype
+ *   q_dtype.  T_k_invT_dev: as wushkv_query_transform.  q_prime_dev:
+ *   [batch][n_q_heads][128] fp32, receives q' (16-byte aligned).  out_dev,
+ *   scale: as wushkv_decode.
+ * When the append needs a single append launch (every one-token append
+ * whose flush does not reach the new token, i.e. recent >= 1) the append
+ * and the query transform share one launch, so a step is two launches.
+ * Results are identical to the three separate calls.  Errors as those
+ * calls; on an argument error nothing is launched and the cache is
+ * unchanged. */
+WUSHKV_API wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                            int32_t in_dtype, const float* T_k_dev, const void* q_dev,
+                                            int32_t q_dtype, const float* T_k_invT_dev, float* q_prime_dev,
+                                            float* out_dev, float scale, void* stream);
+
 /* Decode for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is a deployment convenience around wushkv_decode.
  * Some callers cannot call cudaMalloc when they decode -- code running inside
