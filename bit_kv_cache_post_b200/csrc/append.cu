@@ -60,34 +60,48 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int
   const bool transform = (a.T != nullptr) && has_new;
   const bool staged = transform && (q_last - q_first > 1);
   if (staged) stage_transpose_128(a.T + (size_t)h * D * D, Tt, TT_LD);
-  MatRow trow;   // single quad: this thread's row of T, requested before the inputs
-  if (transform && !staged) load_row(a.T + (size_t)h * D * D, tid, trow);
 
   for (int64_t Q = q_first; Q < q_last; ++Q) {
     __syncthreads();  // previous quad's smem consumers are done
-    // ---- gather the quad's four tokens -------------------------------------
-    for (int j = 0; j < 4; ++j) {
-      const int64_t t = 4 * Q + j;
-      int kind = TOK_SKIP;
-      if (t >= n0 && t < n1) kind = TOK_NEW;
-      else if (t < n0 && t >= S + P0 && t < S + P1) kind = TOK_FLUSH_OLD;
-      if (tid == 0) kind_s[j] = kind;
-      if (kind == TOK_NEW) {
-        const size_t row = (((size_t)b * a.n_tok + (size_t)(t - n0)) * c.n_kv_heads + h) * D;
-        kin[j * D + tid] = load_in(a.k, a.dtype, row + tid);
-        v16[j * D + tid] = round_f16(load_in(a.v, a.dtype, row + tid));
-      } else if (kind == TOK_FLUSH_OLD) {
-        const int slot = (int)((t - S) % W);
-        const size_t off = ((size_t)u * W + slot) * D + tid;
-        k16[j * D + tid] = __half2float(c.ring_k[off]);
-        v16[j * D + tid] = __half2float(c.ring_v[off]);
+    // ---- gather the quad's four tokens (all loads in flight at once) --------
+    {
+      int kind[4];
+      float kx[4], vx[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t t = 4 * Q + j;
+        kind[j] = TOK_SKIP;
+        if (t >= n0 && t < n1) kind[j] = TOK_NEW;
+        else if (t < n0 && t >= S + P0 && t < S + P1) kind[j] = TOK_FLUSH_OLD;
+        kx[j] = vx[j] = 0.f;
+        if (kind[j] == TOK_NEW) {
+          const size_t row = (((size_t)b * a.n_tok + (size_t)(t - n0)) * c.n_kv_heads + h) * D;
+          kx[j] = load_in(a.k, a.dtype, row + tid);
+          vx[j] = load_in(a.v, a.dtype, row + tid);
+        } else if (kind[j] == TOK_FLUSH_OLD) {
+          const int slot = (int)((t - S) % W);
+          const size_t off = ((size_t)u * W + slot) * D + tid;
+          kx[j] = __half2float(c.ring_k[off]);
+          vx[j] = __half2float(c.ring_v[off]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (tid == 0) kind_s[j] = kind[j];
+        if (kind[j] == TOK_NEW) {
+          kin[j * D + tid] = kx[j];
+          v16[j * D + tid] = round_f16(vx[j]);
+        } else if (kind[j] == TOK_FLUSH_OLD) {
+          k16[j * D + tid] = kx[j];
+          v16[j * D + tid] = vx[j];
+        }
       }
     }
     __syncthreads();
     // ---- key transform k' = T k (fp32 FMA), one output dim per thread ------
     if (transform && !staged) {
       float dots[4];
-      row_dots<4>(trow, kin, dots);
+      matvec128_smem<4>(a.T + (size_t)h * D * D, kin, Tt, dots);
       for (int j = 0; j < 4; ++j)
         if (kind_s[j] == TOK_NEW) k16[j * D + tid] = round_f16(dots[j]);
     } else {
@@ -181,7 +195,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int
   }
 }
 
-__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(128, 4) append_kernel(AppendArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   append_body(a, blockIdx.x, blockIdx.y, smem_raw);
 }
@@ -190,9 +204,12 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
 // one launch: slices x < gx of row u are the append CTAs of unit u, slice gx
 // transforms the unit's G queries.
 template <int G>
-__global__ void __launch_bounds__(128) append_qt_kernel(AppendArgs a, int gx, const void* q, int q_dtype,
+__global__ void __launch_bounds__(128, G >= 8 ? 3 : 4) append_qt_kernel(AppendArgs a, int gx, const void* q, int q_dtype,
                                                         const float* TinvT, float* q_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  grid_dependents_may_launch();
+  // every input and the cache may come from the kernel launched just before
+  grid_dependency_wait();
   if ((int)blockIdx.x < gx) {
     append_body(a, blockIdx.x, blockIdx.y, smem_raw);
   } else {
@@ -205,8 +222,8 @@ __global__ void __launch_bounds__(128) append_qt_kernel(AppendArgs a, int gx, co
 // Dynamic shared memory of an append launch: T^T only when a CTA transforms
 // several quads.
 size_t append_smem(const AppendArgs& a) {
-  const bool staged = a.T != nullptr && a.quads_per_cta > 1;
-  return APPEND_VEC_BYTES + (staged ? (size_t)D * TT_LD * sizeof(float) : 0);
+  if (a.T == nullptr) return APPEND_VEC_BYTES;
+  return APPEND_VEC_BYTES + (size_t)D * (a.quads_per_cta > 1 ? TT_LD : MS_LD) * sizeof(float);
 }
 
 cudaError_t set_smem_attr(const void* fn, size_t bytes) {
@@ -215,7 +232,7 @@ cudaError_t set_smem_attr(const void* fn, size_t bytes) {
 
 }  // namespace
 
-size_t append_smem_bytes() { return APPEND_VEC_BYTES + (size_t)D * TT_LD * sizeof(float); }
+size_t append_smem_bytes() { return APPEND_VEC_BYTES + (size_t)D * MS_LD * sizeof(float); }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
   int dev = 0;
@@ -243,18 +260,21 @@ cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, co
   static int attr_done[64][4] = {};
   const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
   if (dev < 64 && !attr_done[dev][gi]) {
-    cudaError_t e = set_smem_attr(fn, append_smem_bytes());
+    cudaError_t e = set_smem_attr(fn, append_smem_bytes() + query_transform_smem(8));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_done[dev][gi] = 1;
   }
   const int64_t gx = a.n_quads > 0 ? (a.n_quads + a.quads_per_cta - 1) / a.quads_per_cta : 0;
   dim3 grid((unsigned)gx + 1, (unsigned)a.c.units);
-  const size_t smem = append_smem(a) > (size_t)G * D * sizeof(float) ? append_smem(a) : (size_t)G * D * sizeof(float);
+  size_t smem = append_smem(a);
+  if (smem < query_transform_smem(G)) smem = query_transform_smem(G);
   switch (G) {
-    case 1: append_qt_kernel<1><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
-    case 2: append_qt_kernel<2><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
-    case 4: append_qt_kernel<4><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
-    case 8: append_qt_kernel<8><<<grid, 128, smem, s>>>(a, (int)gx, q, q_dtype, TinvT, q_out); break;
+    case 1: return launch_with_overlap(append_qt_kernel<1>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);
+    case 2: return launch_with_overlap(append_qt_kernel<2>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);
+    case 4: return launch_with_overlap(append_qt_kernel<4>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);
+    case 8: return launch_with_overlap(append_qt_kernel<8>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -286,11 +286,12 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps
     }
     if (mk != nullptr) {
       if (lane == 0) {
+        const uint64_t pol = l2_evict_first_policy();
         mbar_arrive_expect_tx(bar, 2u * WIN_V);
-        tma_load_2d(st, mk, 0, y, bar);
-        tma_load_2d(st + 1024, mk, 64, y, bar);
-        tma_load_2d(st + WIN_V, mv, 0, y, bar);
-        tma_load_2d(st + WIN_V + 1024, mv, 64, y, bar);
+        tma_load_2d_hint(st, mk, 0, y, bar, pol);
+        tma_load_2d_hint(st + 1024, mk, 64, y, bar, pol);
+        tma_load_2d_hint(st + WIN_V, mv, 0, y, bar, pol);
+        tma_load_2d_hint(st + WIN_V + 1024, mv, 64, y, bar, pol);
       }
       return;
     }
@@ -307,7 +308,8 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps
   }
   if (lane != 0) return;
   mbar_arrive_expect_tx(bar, (uint32_t)SL::PACKED);
-  bulk_copy_g2s(st, k_row_at(c, 0, u, (int64_t)idx * PB), (uint32_t)SL::PACKED, bar);
+  bulk_copy_g2s_hint(st, k_row_at(c, 0, u, (int64_t)idx * PB), (uint32_t)SL::PACKED, bar,
+                     l2_evict_first_policy());
 }
 
 // ---- packed blocks: copy ring + integer tensor cores ------------------------------
@@ -836,6 +838,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   const uint32_t X0 = cta_begin(a, cta), X1 = X0 + a.cta_q + (cta < a.cta_r ? 1u : 0u);
   const int U0 = (int)(X0 / NI), U1 = (int)((X1 - 1) / NI);
 
+  grid_dependents_may_launch();
   // each warp initialises its own copy ring's barriers
   if (lane < NSTAGE) {
     mbar_init(&sh.bar[warp][lane], 1);
@@ -843,6 +846,8 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   }
   __syncwarp();
   uint32_t it = 0;
+  // q' and the cache may come from the kernel launched just before this one
+  grid_dependency_wait();
 
   for (int u_first = U0; u_first <= U1; u_first += UMAX) {
     const int nseg = min(UMAX, U1 - u_first + 1);
@@ -1033,11 +1038,12 @@ cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) 
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  k<<<(unsigned)a.grid, Warps<BITS>::N * 32, smem, s>>>(a, wm);
-  return cudaGetLastError();
+  return launch_with_overlap(k, dim3((unsigned)a.grid), dim3(Warps<BITS>::N * 32), (size_t)smem, s, a, wm);
 }
 
 template <int BITS, bool AFFINE>

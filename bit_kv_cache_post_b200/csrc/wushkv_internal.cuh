@@ -80,6 +80,37 @@ __host__ __device__ __forceinline__ uint8_t* v_meta_at(const DevCache& c, int64_
 enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2, DEV_ERR_TIMEOUT = 4 };
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with
+// launch_with_overlap() may begin while the previous kernel on the stream
+// is still running; it must call grid_dependency_wait() before touching
+// memory that kernel writes or reads (a no-op when there is no such
+// kernel).  grid_dependents_may_launch() lets the next such kernel be
+// scheduled; it never skips the wait on the other side.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_may_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_with_overlap(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ---------------------------------------------------------------------------
 // Exact-rounding helpers
 // ---------------------------------------------------------------------------
 
@@ -171,6 +202,46 @@ __device__ __forceinline__ void row_dots(const MatRow& r, const float* x, float 
   }
 }
 
+// y = M x for NV vectors and a row-major 128 x 128 fp32 matrix M, on a
+// 128-thread CTA: M is staged into shared memory with coalesced 16-byte
+// loads (row stride MS_LD floats, so that a warp's 16-byte reads of 32
+// consecutive rows at one column spread over all banks), then thread t
+// forms row t's dot products against the vectors xs ([NV][128] floats in
+// shared memory, read as broadcasts).  Ends with the outputs in y (thread t:
+// row t); ms must hold 128 * MS_LD floats.  Contains one CTA barrier before
+// the dot products: xs must be written before the call.
+constexpr int MS_LD = 132;
+template <int NV>
+__device__ __forceinline__ void matvec128_smem(const float* __restrict__ M, const float* xs, float* ms,
+                                               float (&y)[NV]) {
+  const int tid = threadIdx.x;
+  const float4* M4 = reinterpret_cast<const float4*>(M);
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __ldg(M4 + tid + 128 * (8 * b + k));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = tid + 128 * (8 * b + k);   // float4 index: row e / 32, column 4 (e % 32)
+      *reinterpret_cast<float4*>(ms + (e >> 5) * MS_LD + 4 * (e & 31)) = v[k];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int v = 0; v < NV; ++v) y[v] = 0.f;
+  const float* row = ms + tid * MS_LD;
+#pragma unroll 8
+  for (int c = 0; c < 128; c += 4) {
+    const float4 m = *reinterpret_cast<const float4*>(row + c);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const float4 x = *reinterpret_cast<const float4*>(xs + v * 128 + c);
+      y[v] = fmaf(m.x, x.x, fmaf(m.y, x.y, fmaf(m.z, x.z, fmaf(m.w, x.w, y[v]))));
+    }
+  }
+}
+
 // Query transform of one (sequence b, KV head h) group on a 128-thread CTA:
 // q'[g][i] = sum_j M[i][j] q[g][j] for the G query heads of the group, M =
 // T_k^{-T} of head h (summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
@@ -185,19 +256,23 @@ __device__ __forceinline__ float load_any(const void* p, int dtype, size_t i) {
 
 template <int G>
 __device__ __forceinline__ void query_transform_unit(const void* q, int dtype, const float* TinvT, float* out,
-                                                     int b, int h, int n_kv_heads, float* qs) {
+                                                     int b, int h, int n_kv_heads, float* smem) {
   const int Hq = n_kv_heads * G;
   const int tid = threadIdx.x;
-  MatRow row;
-  load_row(TinvT + (size_t)h * D * D, tid, row);
+  float* xs = smem;                 // [G][128]
+  float* ms = smem + G * D;         // [128][MS_LD]
 #pragma unroll
   for (int g = 0; g < G; ++g)
-    qs[g * D + tid] = load_any(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
-  __syncthreads();
-  float dots[G];
-  row_dots<G>(row, qs, dots);
+    xs[g * D + tid] = load_any(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
+  float y[G];
+  matvec128_smem<G>(TinvT + (size_t)h * D * D, xs, ms, y);
 #pragma unroll
-  for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = dots[g];
+  for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = y[g];
+}
+
+// Shared memory of query_transform_unit.
+__host__ __device__ constexpr size_t query_transform_smem(int G) {
+  return ((size_t)G * D + (size_t)D * MS_LD) * sizeof(float);
 }
 
 // ---------------------------------------------------------------------------
