@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--copies", type=int, default=64)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     return ap.parse_args()
 
 
@@ -294,6 +295,56 @@ def run_ours(args, rank, world, device, torch, dist):
                 l2_bytes=sum(decode_bytes(w, bits, window_state(c, w)) for c in counts))
 
 
+PREFILL_WORKLOAD = "qwen3-8b-stack36-b64-prefill32768"
+
+
+def run_prefill(device, torch, reps=5):
+    """Bulk append of one layer of the 36-layer workload (batch 64, 32768
+    bf16 tokens per sequence, 2-bit percentile-clipped affine): key transform
+    on the tensor cores, quantise + pack, values packed.  Each timed append
+    goes into a freshly created (zeroed) cache; CUDA events bracket the
+    append call alone."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[PREFILL_WORKLOAD]
+    n = w.context
+    k, v = I.device_kv(w, 0, n, device=device)
+    T, _ = I.key_transforms(w, 0)
+    Td = torch.from_numpy(T).to(device)
+    cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, n, bits=2, quantizer=wk.AFFINE_PCTCLIP,
+                         sink=w.sink, recent=w.recent, chunk=w.chunk,
+                         clip_lo_rank=w.r_lo, clip_hi_rank=w.r_hi)
+    buf = torch.empty(wk.cache_bytes(cfg) + 256, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    times = []
+    for r in range(reps + 1):
+        cache = wk.Cache(cfg, device=device, buffer=buf)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.append(k, v, Td, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        status = cache.device_status()
+        cache.close()
+        if r > 0:
+            times.append(e0.elapsed_time(e1))
+    ms = float(np.median(times))
+    token_heads = w.batch * n * w.n_kv_heads
+    nbytes = token_heads * (2 * 128 * 2 + 2 * (16 * 2 + 4))      # bf16 K, V in; codes + (s, lo) out
+    flops = token_heads * 2 * 128 * 128
+    peak, src = peaks()
+    del k, v, buf
+    return {"workload": f"{w.name} (one layer: batch {w.batch}, {n} tokens per sequence, "
+                        f"{w.n_kv_heads} KV heads, 2-bit affine ranks {w.r_lo}/{w.r_hi})",
+            "ms_per_layer": ms, "tokens_per_s": w.batch * n / (ms / 1e3),
+            "token_heads_per_s": token_heads / (ms / 1e3),
+            "gbs": nbytes / (ms / 1e3) / 1e9, "frac": nbytes / (ms / 1e3) / 1e9 / peak,
+            "key_transform_tflops": flops / (ms / 1e3) / 1e12, "device_status": status,
+            "bytes_per_token_head": 2 * 128 * 2 + 2 * (16 * 2 + 4), "peak_source": src,
+            "timing": f"median of {reps} appends into a fresh cache, CUDA events"}
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
@@ -482,6 +533,9 @@ def main():
                 "steps": E, "counts": "step bytes / step time incl. pinned host<->device copies"},
         "gpu_launches": r["launches"], "clocks": r["clocks"], "device_status": r["status"],
     }
+    if rank == 0 and world == 1 and not args.no_prefill:
+        torch.cuda.empty_cache()
+        line["prefill"] = run_prefill(device, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, bits)
     if dist is not None:
