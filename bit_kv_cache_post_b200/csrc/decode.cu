@@ -922,28 +922,40 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     __syncthreads();
 
     // ---- merge the partials of each segment into this CTA's partial for the unit --
-    // thread (segment, head): the segment's maximum over its warps and its
-    // boundary slot, then every member's merge weight against it
-    if (tid < nseg * G) {
-      const int jj = tid / G, g = tid % G;
-      const bool has_b = jj < nseg - 1 && sh.bused[jj];
-      float M = has_b ? sh.bm[jj][g] : -INFINITY;
-      uint32_t members = 0;
+    // Half-warp per head: lane w of the half holds warp w's final state for
+    // that head; each segment's maximum (its warps and its boundary slot),
+    // the merge weights and the weighted sum come from 16-lane shuffles.
+    static_assert(NW <= 16, "one half-warp per head");
+    if (warp < (16 * G + 31) / 32) {   // whole warps (G = 1 leaves a half idle)
+      const int w = tid & 15, g = tid >> 4;
+      const bool gv = g < G;
+      const int jw = (w < NW && gv) ? sh.wseg[w] : -1;
+      const float mw = jw >= 0 ? sh.sm[w][g] : -INFINITY;
+      const float lw = jw >= 0 ? sh.sl[w][g] : 0.f;
+      float fw = 0.f;
+      for (int jj = 0; jj < nseg; ++jj) {
+        const bool has_b = gv && jj < nseg - 1 && sh.bused[jj];
+        float M = jw == jj ? mw : -INFINITY;
+        if (w == 0 && has_b) M = fmaxf(M, sh.bm[jj][g]);
 #pragma unroll
-      for (int w = 0; w < NW; ++w)
-        if (sh.wseg[w] == jj) { M = fmaxf(M, sh.sm[w][g]); members |= 1u << w; }
-      float L = has_b ? sh.bl[jj][g] * merge_weight(sh.bm[jj][g], M) : 0.f;
-      if (jj < nseg - 1) sh.bf[jj][g] = has_b ? merge_weight(sh.bm[jj][g], M) : 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w)
-        if (members >> w & 1u) {
-          const float f = merge_weight(sh.sm[w][g], M);
-          sh.sf[w][g] = f;
-          L = fmaf(sh.sl[w][g], f, L);
+        for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
+        float L = 0.f;
+        if (jw == jj) { fw = merge_weight(mw, M); L = lw * fw; }
+        if (w == 0 && has_b) {
+          const float fb = merge_weight(sh.bm[jj][g], M);
+          sh.bf[jj][g] = fb;
+          L = fmaf(sh.bl[jj][g], fb, L);
         }
-      sh.sM[jj][g] = M;
-      sh.sL[jj][g] = L;
-      if (g == 0) sh.smask[jj] = members;
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) L += __shfl_xor_sync(FULL_MASK, L, o);
+        const uint32_t bal = __ballot_sync(FULL_MASK, jw == jj);
+        if (w == 0 && gv) {
+          sh.sM[jj][g] = M;
+          sh.sL[jj][g] = L;
+          if (g == 0) sh.smask[jj] = (bal >> (tid & 16)) & 0xFFFFu;
+        }
+      }
+      if (w < NW && gv) sh.sf[w][g] = fw;
     }
     __syncthreads();
     for (int jj = 0; jj < nseg; ++jj) {
