@@ -503,7 +503,17 @@ wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, co
   if (st != WUSHKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (!p.tc && p.nranges == 1) {   // one launch for the append and the query transform
+  const int64_t S = c.sink;
+  const bool new_in_window = p.n1 - 1 < S || p.n1 - 1 >= S + p.a.packed1;
+  if (!p.tc && p.nranges == 1 && new_in_window) {
+    // one launch: the new key's rows, the query rows and the flushed chunk
+    const int64_t f0 = (S + p.a.packed0) / 4, f1 = (S + p.a.packed1) / 4;   // quad-aligned
+    AppendArgs fa = p.a;
+    fa.quad_begin = f0;
+    fa.n_quads = f1 - f0;
+    fa.quads_per_cta = 1;
+    e = launch_step_rows(fa, (int)(f1 - f0), q_dev, q_dtype, T_k_invT_dev, q_prime_dev, s);
+  } else if (!p.tc && p.nranges == 1) {   // one launch for the append and the query transform
     set_quad_range(p.a, p.range[0][0], p.range[0][1]);
     e = launch_append_qt(p.a, q_dev, q_dtype, T_k_invT_dev, q_prime_dev, s);
   } else {

@@ -100,10 +100,21 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int
     __syncthreads();
     // ---- key transform k' = T k (fp32 FMA), one output dim per thread ------
     if (transform && !staged) {
-      float dots[4];
-      matvec128_smem<4>(a.T + (size_t)h * D * D, kin, Tt, dots);
-      for (int j = 0; j < 4; ++j)
-        if (kind_s[j] == TOK_NEW) k16[j * D + tid] = round_f16(dots[j]);
+      // rows 32 warp .. 32 warp + 31 in four groups of eight (the same
+      // arithmetic as every other single-token and query transform)
+      float4 x4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x4[j] = *reinterpret_cast<const float4*>(kin + j * D + 4 * lane);
+      const int rsel = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+#pragma unroll 1
+      for (int rg = 0; rg < 4; ++rg) {
+        float dots[4];
+        const int row0 = 32 * warp + 8 * rg;
+        matvec_rows8<4>(a.T + (size_t)h * D * D, row0, x4, dots);
+        if ((lane & 3) == 0)
+          for (int j = 0; j < 4; ++j)
+            if (kind_s[j] == TOK_NEW) k16[j * D + row0 + rsel] = round_f16(dots[j]);
+      }
     } else {
       for (int j = 0; j < 4; ++j) {
         if (kind_s[j] != TOK_NEW) continue;
@@ -215,15 +226,74 @@ __global__ void __launch_bounds__(128, G >= 8 ? 3 : 4) append_qt_kernel(AppendAr
   } else {
     const int u = blockIdx.y;
     query_transform_unit<G>(q, q_dtype, TinvT, q_out, u / a.c.n_kv_heads, u % a.c.n_kv_heads,
-                            a.c.n_kv_heads, reinterpret_cast<float*>(smem_raw));
+                            a.c.n_kv_heads);
+  }
+}
+
+// A decode step whose single new token stays in the fp16 windows: row
+// slices x < 4 of unit u transform the new key (rows 32x .. 32x + 31 of
+// k' = T k) and store those dims of k' and v in the sink or the ring;
+// slices 4 .. 7 transform the unit's G queries (rows 32(x - 4) ..); slices
+// x >= 8 are the append CTAs of the chunk this step flushes (quads from
+// a.quad_begin, no transform).  Each CTA reads only 16 KB of a matrix.
+template <int G>
+__global__ void __launch_bounds__(128) step_rows_kernel(AppendArgs a, const void* q, int q_dtype,
+                                                        const float* TinvT, float* q_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  grid_dependents_may_launch();
+  grid_dependency_wait();   // every input and the cache may come from the kernel launched just before
+  const int x = blockIdx.x, u = blockIdx.y;
+  const DevCache& c = a.c;
+  const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rsel = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+  if (x >= 8) {
+    append_body(a, x - 8, u, smem_raw);
+    return;
+  }
+  const int row0 = 32 * (x & 3) + 8 * warp;
+  if (x < 4) {
+    const size_t src = ((size_t)b * c.n_kv_heads + h) * D;   // n_tok = 1: [B][1][Hkv][128]
+    const int64_t t = a.n0;
+    __half* kdst;
+    __half* vdst;
+    if (t < c.sink) {
+      kdst = c.sink_k + ((size_t)u * c.sink + (size_t)t) * D;
+      vdst = c.sink_v + ((size_t)u * c.sink + (size_t)t) * D;
+    } else {
+      const size_t slot = (size_t)((t - c.sink) % c.ring_slots);
+      kdst = c.ring_k + ((size_t)u * c.ring_slots + slot) * D;
+      vdst = c.ring_v + ((size_t)u * c.ring_slots + slot) * D;
+    }
+    float y[1];
+    if (a.T != nullptr) {
+      float4 x4[1] = {load4_any(a.k, a.dtype, src + 4 * lane)};
+      matvec_rows8<1>(a.T + (size_t)h * D * D, row0, x4, y);
+    } else {
+      y[0] = load_in(a.k, a.dtype, src + row0 + rsel);
+    }
+    if ((lane & 3) == 0) kdst[row0 + rsel] = __float2half_rn(y[0]);
+    if (lane < 8) vdst[row0 + lane] = __float2half_rn(load_in(a.v, a.dtype, src + row0 + lane));
+  } else {
+    const int Hq = c.n_kv_heads * G;
+    float4 x4[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      x4[g] = load4_any(q, q_dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + 4 * lane);
+    float y[G];
+    matvec_rows8<G>(TinvT + (size_t)h * D * D, row0, x4, y);
+    if ((lane & 3) == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) q_out[((size_t)b * Hq + (size_t)h * G + g) * D + row0 + rsel] = y[g];
+    }
   }
 }
 
 // Dynamic shared memory of an append launch: T^T only when a CTA transforms
 // several quads.
 size_t append_smem(const AppendArgs& a) {
-  if (a.T == nullptr) return APPEND_VEC_BYTES;
-  return APPEND_VEC_BYTES + (size_t)D * (a.quads_per_cta > 1 ? TT_LD : MS_LD) * sizeof(float);
+  const bool staged = a.T != nullptr && a.quads_per_cta > 1;
+  return APPEND_VEC_BYTES + (staged ? (size_t)D * TT_LD * sizeof(float) : 0);
 }
 
 cudaError_t set_smem_attr(const void* fn, size_t bytes) {
@@ -232,7 +302,21 @@ cudaError_t set_smem_attr(const void* fn, size_t bytes) {
 
 }  // namespace
 
-size_t append_smem_bytes() { return APPEND_VEC_BYTES + (size_t)D * MS_LD * sizeof(float); }
+cudaError_t launch_step_rows(const AppendArgs& a, int n_flush_quads, const void* q, int q_dtype,
+                             const float* TinvT, float* q_out, cudaStream_t s) {
+  const int G = a.c.group;
+  dim3 grid((unsigned)(8 + n_flush_quads), (unsigned)a.c.units);
+  const size_t smem = APPEND_VEC_BYTES;
+  switch (G) {
+    case 1: return launch_with_overlap(step_rows_kernel<1>, grid, dim3(128), smem, s, a, q, q_dtype, TinvT, q_out);
+    case 2: return launch_with_overlap(step_rows_kernel<2>, grid, dim3(128), smem, s, a, q, q_dtype, TinvT, q_out);
+    case 4: return launch_with_overlap(step_rows_kernel<4>, grid, dim3(128), smem, s, a, q, q_dtype, TinvT, q_out);
+    case 8: return launch_with_overlap(step_rows_kernel<8>, grid, dim3(128), smem, s, a, q, q_dtype, TinvT, q_out);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+size_t append_smem_bytes() { return APPEND_VEC_BYTES + (size_t)D * TT_LD * sizeof(float); }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
   int dev = 0;
@@ -260,7 +344,7 @@ cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, co
   static int attr_done[64][4] = {};
   const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
   if (dev < 64 && !attr_done[dev][gi]) {
-    cudaError_t e = set_smem_attr(fn, append_smem_bytes() + query_transform_smem(8));
+    cudaError_t e = set_smem_attr(fn, append_smem_bytes());
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
@@ -268,8 +352,7 @@ cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, co
   }
   const int64_t gx = a.n_quads > 0 ? (a.n_quads + a.quads_per_cta - 1) / a.quads_per_cta : 0;
   dim3 grid((unsigned)gx + 1, (unsigned)a.c.units);
-  size_t smem = append_smem(a);
-  if (smem < query_transform_smem(G)) smem = query_transform_smem(G);
+  const size_t smem = append_smem(a);
   switch (G) {
     case 1: return launch_with_overlap(append_qt_kernel<1>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);
     case 2: return launch_with_overlap(append_qt_kernel<2>, grid, dim3(128), smem, s, a, (int)gx, q, q_dtype, TinvT, q_out);

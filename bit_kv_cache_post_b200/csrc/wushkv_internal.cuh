@@ -170,75 +170,54 @@ __device__ __forceinline__ void stage_transpose_128(const float* __restrict__ M,
   }
 }
 
-// One row of a row-major 128 x 128 fp32 matrix in registers (32 x 16 bytes),
-// loaded with every request in flight at once.  Used when a CTA has too few
-// vectors to amortise staging the whole matrix: load the row first, then the
-// vectors, so that both latencies overlap.
-struct MatRow {
-  float4 v[32];
-};
-
-__device__ __forceinline__ void load_row(const float* __restrict__ M, int row, MatRow& r) {
-  const float4* r4 = reinterpret_cast<const float4*>(M + (size_t)row * 128);
-#pragma unroll
-  for (int k = 0; k < 32; ++k) r.v[k] = __ldg(r4 + k);
+// Element i of a device array of the given input dtype, as fp32.
+__device__ __forceinline__ float load_any(const void* p, int dtype, size_t i) {
+  if (dtype == WUSHKV_F16) return __half2float(static_cast<const __half*>(p)[i]);
+  if (dtype == WUSHKV_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  return static_cast<const float*>(p)[i];
 }
 
-// out[j] = dot(row, x[j][0..127]) for NV vectors in shared memory ([NV][128]).
-template <int NV>
-__device__ __forceinline__ void row_dots(const MatRow& r, const float* x, float (&out)[NV]) {
-#pragma unroll
-  for (int j = 0; j < NV; ++j) out[j] = 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const float4 xv = *reinterpret_cast<const float4*>(x + j * 128 + 4 * k);
-      out[j] = fmaf(r.v[k].x, xv.x, out[j]);
-      out[j] = fmaf(r.v[k].y, xv.y, out[j]);
-      out[j] = fmaf(r.v[k].z, xv.z, out[j]);
-      out[j] = fmaf(r.v[k].w, xv.w, out[j]);
-    }
-  }
+__device__ __forceinline__ float4 load4_any(const void* p, int dtype, size_t i) {
+  return make_float4(load_any(p, dtype, i), load_any(p, dtype, i + 1), load_any(p, dtype, i + 2),
+                     load_any(p, dtype, i + 3));
 }
 
-// y = M x for NV vectors and a row-major 128 x 128 fp32 matrix M, on a
-// 128-thread CTA: M is staged into shared memory with coalesced 16-byte
-// loads (row stride MS_LD floats, so that a warp's 16-byte reads of 32
-// consecutive rows at one column spread over all banks), then thread t
-// forms row t's dot products against the vectors xs ([NV][128] floats in
-// shared memory, read as broadcasts).  Ends with the outputs in y (thread t:
-// row t); ms must hold 128 * MS_LD floats.  Contains one CTA barrier before
-// the dot products: xs must be written before the call.
-constexpr int MS_LD = 132;
+// Eight rows of y = M x for NV vectors on one warp: lane l reads columns
+// 4l .. 4l + 3 of rows row0 .. row0 + 7 (eight coalesced 512-byte row loads)
+// against x4[v] = x_v[4l .. 4l + 3]; the per-row partial sums are reduced
+// across lanes by three halving exchanges and two full sums, after which
+// lane l holds row row0 + rsel(l), rsel(l) = 4 bit4(l) + 2 bit3(l) + bit2(l).
 template <int NV>
-__device__ __forceinline__ void matvec128_smem(const float* __restrict__ M, const float* xs, float* ms,
-                                               float (&y)[NV]) {
-  const int tid = threadIdx.x;
-  const float4* M4 = reinterpret_cast<const float4*>(M);
+__device__ __forceinline__ void matvec_rows8(const float* __restrict__ M, int row0, const float4 (&x4)[NV],
+                                             float (&y)[NV]) {
+  const int lane = threadIdx.x & 31;
+  const float4* rows = reinterpret_cast<const float4*>(M + (size_t)row0 * D) + lane;
+  float4 t[8];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    float4 v[8];
+  for (int i = 0; i < 8; ++i) t[i] = __ldg(rows + i * 32);
+  float p[NV][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = __ldg(M4 + tid + 128 * (8 * b + k));
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int e = tid + 128 * (8 * b + k);   // float4 index: row e / 32, column 4 (e % 32)
-      *reinterpret_cast<float4*>(ms + (e >> 5) * MS_LD + 4 * (e & 31)) = v[k];
-    }
+    for (int v = 0; v < NV; ++v)
+      p[v][i] = fmaf(t[i].x, x4[v].x, fmaf(t[i].y, x4[v].y, fmaf(t[i].z, x4[v].z, t[i].w * x4[v].w)));
+#pragma unroll
+  for (int o = 16, n = 4; o >= 4; o >>= 1, n >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int k = 0; k < n; ++k) {
+        const float a = p[v][k], b = p[v][k + n];
+        p[v][k] = (up ? b : a) + __shfl_xor_sync(FULL, up ? a : b, o);
+      }
   }
-  __syncthreads();
 #pragma unroll
-  for (int v = 0; v < NV; ++v) y[v] = 0.f;
-  const float* row = ms + tid * MS_LD;
-#pragma unroll 8
-  for (int c = 0; c < 128; c += 4) {
-    const float4 m = *reinterpret_cast<const float4*>(row + c);
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const float4 x = *reinterpret_cast<const float4*>(xs + v * 128 + c);
-      y[v] = fmaf(m.x, x.x, fmaf(m.y, x.y, fmaf(m.z, x.z, fmaf(m.w, x.w, y[v]))));
-    }
+  for (int v = 0; v < NV; ++v) {
+    float r = p[v][0];
+    r += __shfl_xor_sync(FULL, r, 2);
+    r += __shfl_xor_sync(FULL, r, 1);
+    y[v] = r;
   }
 }
 
@@ -248,31 +227,30 @@ __device__ __forceinline__ void matvec128_smem(const float* __restrict__ M, cons
 // 方法关键点 and 工作参考价值: one d x d product per query; the inverse
 // transpose keeps q'.k' = q.k).  Thread i streams row i of M against the G
 // query vectors staged in qs ([G][128] floats of shared memory).
-__device__ __forceinline__ float load_any(const void* p, int dtype, size_t i) {
-  if (dtype == WUSHKV_F16) return __half2float(static_cast<const __half*>(p)[i]);
-  if (dtype == WUSHKV_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
-  return static_cast<const float*>(p)[i];
-}
 
 template <int G>
 __device__ __forceinline__ void query_transform_unit(const void* q, int dtype, const float* TinvT, float* out,
-                                                     int b, int h, int n_kv_heads, float* smem) {
+                                                     int b, int h, int n_kv_heads) {
   const int Hq = n_kv_heads * G;
-  const int tid = threadIdx.x;
-  float* xs = smem;                 // [G][128]
-  float* ms = smem + G * D;         // [128][MS_LD]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rsel = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+  float4 x4[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-    xs[g * D + tid] = load_any(q, dtype, ((size_t)b * Hq + (size_t)h * G + g) * D + tid);
-  float y[G];
-  matvec128_smem<G>(TinvT + (size_t)h * D * D, xs, ms, y);
+  for (int g = 0; g < G; ++g) {
+    const size_t base = ((size_t)b * Hq + (size_t)h * G + g) * D + 4 * lane;
+    x4[g] = make_float4(load_any(q, dtype, base), load_any(q, dtype, base + 1), load_any(q, dtype, base + 2),
+                        load_any(q, dtype, base + 3));
+  }
+#pragma unroll 1
+  for (int rg = 0; rg < 4; ++rg) {
+    const int row0 = 32 * warp + 8 * rg;
+    float y[G];
+    matvec_rows8<G>(TinvT + (size_t)h * D * D, row0, x4, y);
+    if ((lane & 3) == 0) {
 #pragma unroll
-  for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + tid] = y[g];
-}
-
-// Shared memory of query_transform_unit.
-__host__ __device__ constexpr size_t query_transform_smem(int G) {
-  return ((size_t)G * D + (size_t)D * MS_LD) * sizeof(float);
+      for (int g = 0; g < G; ++g) out[((size_t)b * Hq + (size_t)h * G + g) * D + row0 + rsel] = y[g];
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -414,6 +392,12 @@ struct AppendArgs {
   int quads_per_cta;
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+// A one-token decode-step append whose new token stays in the fp16 windows,
+// fused with the step's query transform: per unit, four CTAs for the key
+// rows, four for the query rows, and n_flush_quads append CTAs for the quads
+// of the chunk this step flushes (a.quad_begin, no transform).
+cudaError_t launch_step_rows(const AppendArgs& a, int n_flush_quads, const void* q, int q_dtype,
+                             const float* TinvT, float* q_out, cudaStream_t s);
 // The append launch of a (single-phase, FMA-path) decode-step append fused
 // with the query transform of the step (q_out = T_k^{-T} q per query head).
 cudaError_t launch_append_qt(const AppendArgs& a, const void* q, int q_dtype, const float* TinvT,
