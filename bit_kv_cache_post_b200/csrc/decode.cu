@@ -79,14 +79,11 @@ struct Smem {
   float qsum[UMAX][NT * 4];                // sum of the quantised q per head
   uint8_t ps[NW][NT * 8][PS_LD];           // per-warp P terms [col][token]
   float sm[NW][G], sl[NW][G];              // per-warp softmax max / sum
-  float sf[NW][G];                         // per-warp merge weights 2^(m_w - M_segment)
   // a warp whose item range crosses the end of segment j leaves its partial
   // for segment j here (at most one warp per boundary)
   float bo[UMAX - 1][G][D];
-  float bm[UMAX - 1][G], bl[UMAX - 1][G], bf[UMAX - 1][G];
+  float bm[UMAX - 1][G], bl[UMAX - 1][G];
   int bused[UMAX - 1];
-  float sM[UMAX][G], sL[UMAX][G];          // per-segment maximum and weighted sum
-  uint32_t smask[UMAX];                    // warps whose final state belongs to each segment
   int wseg[NW];                            // segment of each warp's final state (-1: none)
   alignas(8) uint64_t bar[NW][NSTAGE];
   int is_last[UMAX];
@@ -922,57 +919,39 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     __syncthreads();
 
     // ---- merge the partials of each segment into this CTA's partial for the unit --
-    // Half-warp per head: lane w of the half holds warp w's final state for
-    // that head; each segment's maximum (its warps and its boundary slot),
-    // the merge weights and the weighted sum come from 16-lane shuffles.
-    static_assert(NW <= 16, "one half-warp per head");
-    if (warp < (16 * G + 31) / 32) {   // whole warps (G = 1 leaves a half idle)
-      const int w = tid & 15, g = tid >> 4;
-      const bool gv = g < G;
-      const int jw = (w < NW && gv) ? sh.wseg[w] : -1;
-      const float mw = jw >= 0 ? sh.sm[w][g] : -INFINITY;
-      const float lw = jw >= 0 ? sh.sl[w][g] : 0.f;
-      float fw = 0.f;
-      for (int jj = 0; jj < nseg; ++jj) {
-        const bool has_b = gv && jj < nseg - 1 && sh.bused[jj];
-        float M = jw == jj ? mw : -INFINITY;
-        if (w == 0 && has_b) M = fmaxf(M, sh.bm[jj][g]);
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
-        float L = 0.f;
-        if (jw == jj) { fw = merge_weight(mw, M); L = lw * fw; }
-        if (w == 0 && has_b) {
-          const float fb = merge_weight(sh.bm[jj][g], M);
-          sh.bf[jj][g] = fb;
-          L = fmaf(sh.bl[jj][g], fb, L);
-        }
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) L += __shfl_xor_sync(FULL_MASK, L, o);
-        const uint32_t bal = __ballot_sync(FULL_MASK, jw == jj);
-        if (w == 0 && gv) {
-          sh.sM[jj][g] = M;
-          sh.sL[jj][g] = L;
-          if (g == 0) sh.smask[jj] = (bal >> (tid & 16)) & 0xFFFFu;
-        }
-      }
-      if (w < NW && gv) sh.sf[w][g] = fw;
-    }
-    __syncthreads();
+    // thread (head g, dim d): the segment's maximum over its warps and its
+    // boundary slot, then the weighted sums, all from shared-memory broadcasts
     for (int jj = 0; jj < nseg; ++jj) {
-      const uint32_t members = sh.smask[jj];
       const bool has_b = jj < nseg - 1 && sh.bused[jj];
       const int uu = u_first + jj;
       const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
       float* part_base = a.partials + ((size_t)uu * c.max_splits + (cta - cta_u0)) * G * PART;
       for (int e = tid; e < G * D; e += NW * 32) {
         const int g = e / D, d = e % D;
-        float O = has_b ? sh.bf[jj][g] * sh.bo[jj][g][d] : 0.f;
+        float M = has_b ? sh.bm[jj][g] : -INFINITY;
+        float mv[NW];
+        uint32_t members = 0;   // slots of other segments or of idle warps are never read
 #pragma unroll
-        for (int w = 0; w < NW; ++w)
-          if (members >> w & 1u) O = fmaf(so[w][g][d], sh.sf[w][g], O);
+        for (int w = 0; w < NW; ++w) {
+          const bool in = sh.wseg[w] == jj;
+          members |= (in ? 1u : 0u) << w;
+          mv[w] = in ? sh.sm[w][g] : -INFINITY;
+          M = fmaxf(M, mv[w]);
+        }
+        const float fb = has_b ? merge_weight(sh.bm[jj][g], M) : 0.f;
+        float O = has_b ? fb * sh.bo[jj][g][d] : 0.f;
+        float L = has_b ? fb * sh.bl[jj][g] : 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          if (members >> w & 1u) {
+            const float f = merge_weight(mv[w], M);
+            O = fmaf(so[w][g][d], f, O);
+            L = fmaf(sh.sl[w][g], f, L);
+          }
+        }
         float* part = part_base + (size_t)g * PART;
         part[d] = O;
-        if (d == 0) { part[D] = sh.sM[jj][g]; part[D + 1] = sh.sL[jj][g]; }
+        if (d == 0) { part[D] = M; part[D + 1] = L; }
       }
     }
 
