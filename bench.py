@@ -131,6 +131,22 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (every rank gets it).  The job's
+    time is the slowest rank's: each rank runs an independent replica of the
+    workload (weak scaling, no data-path collective)."""
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(step_bytes_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job GB/s: every rank moved step_bytes_per_rank in the timed
+    region, and the region took ms (max over ranks)."""
+    return world * step_bytes_per_rank / (ms / 1e3) / 1e9
+
+
 def build_inputs(w, torch, device):
     """Prefill keys/values (context - 1 tokens) and a pool of per-step tokens."""
     from bit_kv_cache_post_b200 import inputs as I
@@ -226,9 +242,7 @@ def run_ours(args, rank, world, device, torch, dist):
         dist.barrier()
     ms = t0.elapsed_time(t1)
     if dist is not None:
-        tt = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, device)
     launches_per_step = 2
     status = max(c.device_status() for c in caches)
 
@@ -292,9 +306,7 @@ def run_ours(args, rank, world, device, torch, dist):
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
     if dist is not None:
-        tt = torch.tensor([e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
+        e_ms = max_over_ranks(e_ms, dist, device)
 
     return dict(w=w, bits=bits, K=K, ms=ms, dec_total=dec_total, rest_total=rest_total,
                 dec_ms=dec_ms, dec_launch_bytes=dec_launch_bytes, clocks=clocks.summary(),
@@ -516,7 +528,7 @@ def main():
     r = run_ours(args, rank, world, device, torch, dist)
     w, bits, K = r["w"], r["bits"], r["K"]
     step_bytes = r["dec_total"] + r["rest_total"]
-    value = world * step_bytes / (r["ms"] / 1e3) / 1e9
+    value = job_value(step_bytes, r["ms"], world)
     dec_avg_ms = float(np.mean(r["dec_ms"]))
     dec_launch_bytes = float(np.mean(r["dec_launch_bytes"]))
     achieved = dec_launch_bytes / (dec_avg_ms / 1e3) / 1e9
