@@ -12,10 +12,11 @@
 // Work items: a unit's cache is a sequence of items -- packed blocks of 64
 // tokens and window chunks of 8 fp16 tokens, each about 4 KB -- with the
 // window chunks spread evenly among the packed blocks.  The units' items are
-// laid end to end and CTA i of the one-wave grid takes the i-th equal share
-// (stream-K): usually part of one unit, sometimes the end of one and the
-// start of the next.  Each unit segment of a CTA is cut into four equal item
-// ranges, one per warp.  A warp streams its items through a ring of
+// laid end to end and CTA i of the one-wave grid (one CTA per SM) takes the
+// i-th equal share (stream-K): usually the end of one unit and the start of
+// the next.  The CTA's share is cut into equal warp ranges; a range that
+// crosses a unit boundary leaves the finished unit's state in a shared-memory
+// boundary slot.  A warp streams its items through a ring of
 // shared-memory stages filled by bulk asynchronous copies (the TMA engine)
 // and runs them on tensor cores with mma.sync: packed blocks on the integer
 // pipe (codes u8 x two int8 terms of the query for the scores; codes u8 x
