@@ -84,6 +84,8 @@ def test_null_arguments_are_rejected_without_a_gpu(wk):
     assert lib.wushkv_append(None, None, None, 0, None, 1, 2, 0, None) == wk.EINVAL
     assert lib.wushkv_decode(None, None, None, 0.0, None) == wk.EINVAL
     assert lib.wushkv_query_transform(None, 0, None, None, 1, 4, 1, None) == wk.EINVAL
+    assert lib.wushkv_decode_step(None, None, None, 0, None, None, 0, None, None, None, 0.0, None) == wk.EINVAL
+    assert lib.wushkv_decode_noalloc(None, None, None, 0.0, None) == wk.EINVAL
     out = ctypes.c_void_p()
     cfg = wk.make_config(1, 1, 4, 100)
     assert lib.wushkv_cache_create(ctypes.byref(cfg), None, 0, None, ctypes.byref(out)) == wk.EINVAL
