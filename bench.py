@@ -49,7 +49,7 @@ def parse():
 
 
 # ---------------------------------------------------------------------------
-# byte model (algorithmic bytes)
+# byte model: algorithmic bytes (packed codes, per-token scales, fp16 windows)
 # ---------------------------------------------------------------------------
 
 def meta_bytes(quantizer: str) -> int:
@@ -450,7 +450,7 @@ def run_reference(args):
     v = nbytes / el / 1e9
     sample = (f"one (sequence, KV head) unit of {w.name}; each step appends 1 token and decodes "
               f"{w.group} heads over {'all' if frac >= 1 else f'{frac:.3%} of the packed'} tokens; 1 thread")
-    return {"impl": "reference", "metric": BASELINE_METRIC, "value": v, "unit": "GB/s",
+    return {"impl": "reference", "metric": METRIC_NAME, "value": v, "unit": "GB/s",
             "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_block(w, args.bits, None),
@@ -460,7 +460,7 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------
 
-BASELINE_METRIC = "2-bit KV decode-attention GB/s (% of HBM peak); KV append tokens/s"
+METRIC_NAME = "2-bit KV decode-attention GB/s (% of HBM peak); KV append tokens/s"
 
 
 DECODE_SOURCES = ["bit_kv_cache_post_b200/csrc/decode.cu", "bit_kv_cache_post_b200/csrc/decode_frag.cuh",
@@ -535,7 +535,7 @@ def main():
     peak, peak_src = peaks()
     E, e_ms, e_dec, h2d, d2h = r["e2e"]
     line = {
-        "metric": BASELINE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "metric": METRIC_NAME, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": r["ms"] / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": config_block(w, bits, r["copies"]),
