@@ -197,7 +197,8 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
 /* GQA decode attention of one query per query head over the whole cache.
  *   Source: review "[논문리뷰] WUSH-KV ..." (secrett2633), Key Terms (GQA);
  *   dequantisation happens inside the score and PV loops.
- *   q_prime_dev: [batch][n_q_heads][128] fp32 transformed queries.
+ *   q_prime_dev: [batch][n_q_heads][128] fp32 transformed queries, 16-byte
+ *                aligned (EINVAL otherwise; read as float4).
  *   out_dev:     [batch][n_q_heads][128] fp32 = softmax(scale q'.k'^T) v
  *                in the transformed value space; 16-byte aligned (EINVAL otherwise).
  *   scale: softmax scale; 0 selects 1/sqrt(128).
