@@ -131,16 +131,4 @@ __device__ __forceinline__ float v_row_scale(int rho) {
   else return (rho & 1) ? 1.f / 16.f : 1.f;
 }
 
-// Per-token dequantisation parameters: value = scale * code + offset.
-template <bool AFFINE>
-__device__ __forceinline__ float2 load_meta(const uint8_t* meta, int tok, float beta) {
-  if constexpr (AFFINE) {
-    const __half2 sl = *reinterpret_cast<const __half2*>(meta + (size_t)tok * 4);
-    return make_float2(__low2float(sl), __high2float(sl));
-  } else {
-    const float d = __half2float(*reinterpret_cast<const __half*>(meta + (size_t)tok * 2));
-    return make_float2(d, d * beta);
-  }
-}
-
 }  // namespace wushkv

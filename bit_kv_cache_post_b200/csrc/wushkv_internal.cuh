@@ -142,12 +142,6 @@ __device__ __forceinline__ float warp_max_f32(float v) {
   return v;
 }
 
-__device__ __forceinline__ float warp_sum_f32(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  return v;
-}
-
 // Stage the transpose of a row-major 128 x 128 fp32 matrix into shared
 // memory (row stride ld, padded against bank conflicts) with a 128-thread
 // block: 16-byte loads, eight in flight per thread.
