@@ -1,6 +1,7 @@
 // Host side of the libwushkv C ABI: configuration checks, cache layout, the
 // window/flush bookkeeping of each append, decode split policy, export and
 // status.  See include/wushkv.h for the contract of every entry point.
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -40,6 +41,11 @@ constexpr int MAX_PARTS_PER_UNIT = 256;
 // quad boundary) take the tensor-core kernel (two 128-token tiles).
 constexpr int64_t TC_MIN_TOKENS = 256;
 constexpr int64_t TC_MIN_CTA_TILES = 6;
+// Each unit's arrival counter sits on its own 128-byte line, so that the
+// atomics of different units at the end of a decode do not queue on one line.
+constexpr size_t COUNTER_BYTES = 128;
+// Fault injection for tests (wushkv_inject_decode_timeout): 0 = off.
+std::atomic<uint32_t> g_inject_polls{0};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -131,20 +137,34 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
   L->v_meta_off = in_block; in_block += 64 * L->meta_bytes;
   L->block_stride = in_block;                                   // a multiple of 128
   L->unit_stride = (size_t)(L->packed_capacity / 64) * L->block_stride;
-  size_t off = align_up(U * L->unit_stride, 256);               // packed region at offset 0
+  // every region is followed by a guard band (see guard_spans)
+  size_t off = align_up(U * L->unit_stride + WUSHKV_GUARD_BYTES, 256);   // packed region at offset 0
   L->sink_unit_stride = (size_t)c.sink * 128 * 2;
-  L->sink_k_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
-  L->sink_v_off = off; off = align_up(off + U * L->sink_unit_stride, 256);
+  L->sink_k_off = off; off = align_up(off + U * L->sink_unit_stride + WUSHKV_GUARD_BYTES, 256);
+  L->sink_v_off = off; off = align_up(off + U * L->sink_unit_stride + WUSHKV_GUARD_BYTES, 256);
   L->ring_slots = c.recent + c.chunk;
   L->ring_unit_stride = (size_t)L->ring_slots * 128 * 2;
-  L->ring_k_off = off; off = align_up(off + U * L->ring_unit_stride, 256);
-  L->ring_v_off = off; off = align_up(off + U * L->ring_unit_stride, 256);
+  L->ring_k_off = off; off = align_up(off + U * L->ring_unit_stride + WUSHKV_GUARD_BYTES, 256);
+  L->ring_v_off = off; off = align_up(off + U * L->ring_unit_stride + WUSHKV_GUARD_BYTES, 256);
   const int ms = max_splits_for(c, L->packed_capacity);
   L->workspace_off = off;
-  L->workspace_bytes = U * (size_t)ms * G * PARTIAL_FLOATS * sizeof(float) + U * sizeof(int);
-  off = align_up(off + L->workspace_bytes, 256);
+  L->workspace_bytes = align_up(U * (size_t)ms * G * PARTIAL_FLOATS * sizeof(float), COUNTER_BYTES) +
+                       U * COUNTER_BYTES;
+  off = align_up(off + L->workspace_bytes + WUSHKV_GUARD_BYTES, 256);
   L->status_off = off; off = align_up(off + 256, 256);
   L->total_bytes = off;
+}
+
+// Start offsets of the guard bands that follow the packed region, sink K,
+// sink V, ring K, ring V and the workspace.
+void guard_spans(const wushkv_config& c, const wushkv_layout& L, size_t out[6]) {
+  const size_t U = (size_t)c.batch * c.n_kv_heads;
+  out[0] = U * L.unit_stride;
+  out[1] = L.sink_k_off + U * L.sink_unit_stride;
+  out[2] = L.sink_v_off + U * L.sink_unit_stride;
+  out[3] = L.ring_k_off + U * L.ring_unit_stride;
+  out[4] = L.ring_v_off + U * L.ring_unit_stride;
+  out[5] = L.workspace_off + L.workspace_bytes;
 }
 
 DevCache dev_view(const wushkv_cache* h) {
@@ -175,8 +195,10 @@ DevCache dev_view(const wushkv_cache* h) {
   const size_t U = (size_t)c.batch * c.n_kv_heads;
   d.partials = reinterpret_cast<float*>(h->base + L.workspace_off);
   d.counters = reinterpret_cast<int*>(h->base + L.workspace_off +
-                                      U * (size_t)d.max_splits * (c.n_q_heads / c.n_kv_heads) *
-                                          PARTIAL_FLOATS * sizeof(float));
+                                      align_up(U * (size_t)d.max_splits * (c.n_q_heads / c.n_kv_heads) *
+                                                   PARTIAL_FLOATS * sizeof(float),
+                                               COUNTER_BYTES));
+  d.counter_stride = (int)(COUNTER_BYTES / sizeof(int));
   d.status = reinterpret_cast<int*>(h->base + L.status_off);
   d.units = (int)U;
   d.n_kv_heads = c.n_kv_heads;
@@ -254,6 +276,7 @@ wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, flo
   a->cta_r = (uint32_t)(items % grid);
   a->partials = a->c.partials;
   a->counters = a->c.counters;
+  a->inject_polls = g_inject_polls.load(std::memory_order_relaxed);
   return WUSHKV_OK;
 }
 
@@ -305,7 +328,12 @@ wushkv_status wushkv_cache_create(const wushkv_config* cfg, void* dev_mem, size_
   h->n = 0;
   h->alpha = cfg->quest_alpha > 0 ? cfg->quest_alpha : wushkv_default_quest_alpha(cfg->bits);
   make_window_maps(dev_view(h), &h->wmaps);
-  const cudaError_t e = cudaMemsetAsync(dev_mem, 0, L.total_bytes, static_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaMemsetAsync(dev_mem, 0, L.total_bytes, static_cast<cudaStream_t>(stream));
+  size_t guards[6];
+  guard_spans(*cfg, L, guards);
+  for (int i = 0; i < 6 && e == cudaSuccess; ++i)
+    e = cudaMemsetAsync(static_cast<uint8_t*>(dev_mem) + guards[i], WUSHKV_GUARD_FILL, WUSHKV_GUARD_BYTES,
+                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { delete h; return WUSHKV_ECUDA; }
   *out = h;
   return WUSHKV_OK;
@@ -635,6 +663,8 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
   return WUSHKV_OK;
 }
 
+void wushkv_inject_decode_timeout(uint32_t polls) { g_inject_polls.store(polls, std::memory_order_relaxed); }
+
 wushkv_status wushkv_device_status(const wushkv_cache* cache, int32_t clear, int32_t* out) {
   if (!cache || !out) return WUSHKV_EINVAL;
   int32_t v = 0;
@@ -665,9 +695,10 @@ constexpr size_t NOALLOC_COUNTER_BYTES = size_t(65536) * sizeof(int);  // one pe
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch, looked up once per device.  In host
+// Device address of g_noalloc_scratch, looked up once per device (by
+// whichever thread gets there first; the lookup is idempotent).  In host
 // code the symbol itself is only a host-side stand-in for the array.
-void* g_noalloc_addr[64] = {nullptr};
+std::atomic<void*> g_noalloc_addr[64];
 
 }  // namespace
 
@@ -681,10 +712,10 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WUSHKV_ECUDA;
   if (dev < 0 || dev >= 64) return WUSHKV_EUNSUPPORTED;
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return WUSHKV_ECUDA;
-    g_noalloc_addr[dev] = p;
+  void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch) return WUSHKV_ECUDA;
+    g_noalloc_addr[dev].store(scratch, std::memory_order_release);
   }
   DecodeArgs a;
   const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
@@ -699,10 +730,11 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   if (units * sizeof(int) > NOALLOC_COUNTER_BYTES ||
       partial_bytes > NOALLOC_SCRATCH_BYTES - NOALLOC_COUNTER_BYTES)
     return WUSHKV_ECAPACITY;
-  unsigned char* base = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+  unsigned char* base = static_cast<unsigned char*>(scratch);
   a.counters = reinterpret_cast<int*>(base);
   a.partials = reinterpret_cast<float*>(base + NOALLOC_COUNTER_BYTES);
   a.c.counters = a.counters;
+  a.c.counter_stride = 1;
   a.c.partials = a.partials;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps the previous call's contents: arrival counters must

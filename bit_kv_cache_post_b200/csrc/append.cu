@@ -154,6 +154,10 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int
     }
     // ---- quantise + pack a whole quad -------------------------------------------
     const int64_t pk = t0 - S;  // packed index of the quad's first token
+    if (pk + 4 > c.packed_capacity) {   // the host's bookkeeping went wrong: never write past the region
+      if (tid == 0) atomicOr(c.status, DEV_ERR_RANGE);
+      continue;
+    }
     for (int kv = 0; kv < 2; ++kv) {
       const float* src = (kv == 0 ? k16 : v16) + warp * D;
       float x[4];
@@ -218,9 +222,10 @@ template <int G>
 __global__ void __launch_bounds__(128, G >= 8 ? 3 : 4) append_qt_kernel(AppendArgs a, int gx, const void* q, int q_dtype,
                                                         const float* TinvT, float* q_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  grid_dependents_may_launch();
-  // every input and the cache may come from the kernel launched just before
+  // every input and the cache may come from the kernel launched just before;
+  // the next kernel is released only after that wait (see grid_dependency_wait)
   grid_dependency_wait();
+  grid_dependents_may_launch();
   if ((int)blockIdx.x < gx) {
     append_body(a, blockIdx.x, blockIdx.y, smem_raw);
   } else {
@@ -240,8 +245,8 @@ template <int G>
 __global__ void __launch_bounds__(128) step_rows_kernel(AppendArgs a, const void* q, int q_dtype,
                                                         const float* TinvT, float* q_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  grid_dependents_may_launch();
   grid_dependency_wait();   // every input and the cache may come from the kernel launched just before
+  grid_dependents_may_launch();
   const int x = blockIdx.x, u = blockIdx.y;
   const DevCache& c = a.c;
   const int b = u / c.n_kv_heads, h = u % c.n_kv_heads;

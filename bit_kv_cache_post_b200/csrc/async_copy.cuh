@@ -79,6 +79,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// Bring a tensor map's descriptor into the TMA unit's cache ahead of its
+// first use (the map lives in kernel parameter space).
+__device__ __forceinline__ void prefetch_tensormap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 // Plain arrival (no transaction bytes) on a barrier initialised with count 1.
 __device__ __forceinline__ void mbar_arrive_once(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");

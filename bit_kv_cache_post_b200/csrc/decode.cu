@@ -87,16 +87,51 @@ struct Smem {
   int bused[UMAX - 1];
   int wseg[NW];                            // segment of each warp's final state (-1: none)
   alignas(8) uint64_t bar[NW][NSTAGE];
+  uint64_t never;                          // a barrier nothing arrives on (fault injection)
   int is_last[UMAX];
+  // CTA merge: weight of each warp's slot in each segment (0 for warps of
+  // other segments) and of the boundary slots; each segment's maximum (an
+  // ordered integer while the warps raise it) and sum
+  float wf[UMAX][NW][G], bf[UMAX - 1][G];
+  int segMi[UMAX][G];
+  float segL[UMAX][G];
+  // other CTAs holding items of each segment's unit (0: no exchange)
+  int others[UMAX];
 };
 
-// Per-warp partial outputs, placed over the stage buffers once every warp
-// has drained its copy ring.
+// A warp's final partial output goes into its own copy stages once its ring
+// has drained (no other warp touches them); the CTA's merged numerator of
+// segment j follows the slot in warp j's stages.
 template <int BITS, int G>
-__device__ __forceinline__ float (*warp_slots(Smem<BITS, G>& sh))[G][D] {
-  static_assert(sizeof(float) * Smem<BITS, G>::NW * G * D <= sizeof(sh.stage), "stage area too small");
-  return reinterpret_cast<float(*)[G][D]>(&sh.stage[0][0][0]);
+__device__ __forceinline__ float (*warp_slot(Smem<BITS, G>& sh, int w))[D] {
+  static_assert(2 * sizeof(float) * G * D <= sizeof(sh.stage[0]), "stage area too small");
+  static_assert(UMAX <= Smem<BITS, G>::NW, "segments per batch");
+  return reinterpret_cast<float(*)[D]>(&sh.stage[w][0][0]);
 }
+template <int BITS, int G>
+__device__ __forceinline__ float (*segment_sum(Smem<BITS, G>& sh, int j))[D] {
+  return warp_slot(sh, j) + G;
+}
+
+// Order-preserving map of floats to ints (for integer max); -inf maps below
+// every finite value.
+__device__ __forceinline__ int float_order(float x) {
+  const int i = __float_as_int(x);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float order_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
+
+// Raise segment j's maximum to the warp's reference maxima (lanes 0..3
+// hold head 4 nt + lane).
+template <int BITS, int G>
+__device__ __forceinline__ void raise_segment_max(Smem<BITS, G>& sh, int j, const float* m, int lane) {
+  constexpr int NT = (G + 3) / 4;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+    if (lane < 4 && nt * 4 + lane < G) atomicMax(&sh.segMi[j][nt * 4 + lane], float_order(m[nt]));
+}
+
+
 
 // 2^x with the SFU (approximate, flushes denormal results to zero; 2^-inf = 0).
 __device__ __forceinline__ float ex2(float x) {
@@ -662,7 +697,7 @@ struct GCursor {
   }
 };
 
-// First copies of the warp's items, issued before the query prologue.
+// First copies of the warp's items [y0, y1), issued before the query prologue.
 template <int BITS, bool AFFINE, int G>
 __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const WindowMaps& wm,
                                                     Smem<BITS, G>& sh, uint32_t y0, uint32_t y1,
@@ -766,6 +801,7 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
           if (S.F[nt] > 0.f) flush_pv(S, nt);
       }
       state_to_slot<BITS, G, AFFINE>(S, sh.bo[cur], sh.bm[cur], sh.bl[cur], lane);
+      raise_segment_max(sh, cur, S.m, lane);
       if (lane == 0) sh.bused[cur] = 1;
     }
     begin_segment<BITS, G>(sh, j, lane, qb, qscale, qsum, qoff, S);
@@ -774,13 +810,18 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
     cc.start(a, (int)(y - (uint32_t)unit * NI));
     for (; y < yend; ++y, ++it) {
       const int stg = it % NSTAGE;
-      if (!mbar_wait_bounded(&sh.bar[warp][stg], (it / NSTAGE) & 1, WAIT_POLLS)) {
+      // (fault injection for tests: the warp's first wait is made on a
+      // barrier that nothing completes, so it runs out)
+      const bool injected = a.inject_polls != 0 && y == y0;
+      if (!mbar_wait_bounded(injected ? &sh.never : &sh.bar[warp][stg], injected ? 0u : (it / NSTAGE) & 1,
+                             injected ? a.inject_polls : WAIT_POLLS)) {
         // A copy never completed: report it, drain what is still in flight
-        // (bounded), and contribute nothing more.
+        // (bounded, at the full limit), and contribute nothing more.
         if (lane == 0) atomicOr(a.c.status, DEV_ERR_TIMEOUT);
-        for (uint32_t q = 0; q < (uint32_t)NSTAGE && y + q < y1; ++q)
+        const uint32_t inflight = min((uint32_t)NSTAGE, y1 - y);
+        for (uint32_t q = 0; q < inflight; ++q)
           mbar_wait_bounded(&sh.bar[warp][(it + q) % NSTAGE], ((it + q) / NSTAGE) & 1, WAIT_POLLS);
-        it += y1 - y;
+        it += inflight;   // the ring is empty again, its phases in step
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
         return cur;
@@ -836,16 +877,22 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   const uint32_t X0 = cta_begin(a, cta), X1 = X0 + a.cta_q + (cta < a.cta_r ? 1u : 0u);
   const int U0 = (int)(X0 / NI), U1 = (int)((X1 - 1) / NI);
 
-  grid_dependents_may_launch();
+  // the window maps' descriptors are kernel parameters: fetch them now
+  if (tid == 0) {
+    prefetch_tensormap(&wm.sink_k); prefetch_tensormap(&wm.sink_v);
+    prefetch_tensormap(&wm.ring_k); prefetch_tensormap(&wm.ring_v);
+  }
   // each warp initialises its own copy ring's barriers
   if (lane < NSTAGE) {
     mbar_init(&sh.bar[warp][lane], 1);
+    if (warp == 0 && lane == 0) mbar_init(&sh.never, 1);
     fence_barrier_init();
   }
-  __syncwarp();
+  __syncthreads();
   uint32_t it = 0;
   // q' and the cache may come from the kernel launched just before this one
   grid_dependency_wait();
+  grid_dependents_may_launch();
 
   for (int u_first = U0; u_first <= U1; u_first += UMAX) {
     const int nseg = min(UMAX, U1 - u_first + 1);
@@ -874,6 +921,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     GCursor ic;
     warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, y0, y1, warp, lane, it, ic);
     if (tid < UMAX - 1) sh.bused[tid] = 0;
+    if (tid < UMAX * G) sh.segMi[tid / G][tid % G] = float_order(-INFINITY);
 
     // ---- scaled query: two int8 terms and two fp16 terms per head ----------------
 #pragma unroll
@@ -882,25 +930,30 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
       if (pj < nseg) {
         float x[4] = {qv[i].x * a.scale_log2, qv[i].y * a.scale_log2, qv[i].z * a.scale_log2,
                       qv[i].w * a.scale_log2};
-        float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-        mx = warp_max_f32(mx);
+        // |x| >= 0 orders like its bit pattern: one integer warp reduction
+        const float mx = __uint_as_float(__reduce_max_sync(
+            FULL_MASK, __float_as_uint(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))))));
         const float sigma = mx / 127.f;
         const float inv = mx > 0.f ? 127.f / mx : 0.f;
         int sum = 0;
+        uint32_t w0 = 0, w1 = 0;
+        __half hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float y = x[e] * inv;
           const float t0 = fminf(fmaxf(rintf(y), -127.f), 127.f);
           const float t1 = fminf(fmaxf(rintf((y - t0) * 254.f), -127.f), 127.f);
-          sh.qterm[pj][g][0][4 * lane + e] = (int8_t)t0;
-          sh.qterm[pj][g][1][4 * lane + e] = (int8_t)t1;
+          w0 |= (uint32_t)(uint8_t)(int8_t)t0 << (8 * e);
+          w1 |= (uint32_t)(uint8_t)(int8_t)t1 << (8 * e);
           sum += (int)t0 * 254 + (int)t1;
-          const __half hi = __float2half_rn(x[e]);
-          sh.qh[pj][g][0][4 * lane + e] = hi;
-          sh.qh[pj][g][1][4 * lane + e] = __float2half_rn(x[e] - __half2float(hi));
+          hi[e] = __float2half_rn(x[e]);
+          lo[e] = __float2half_rn(x[e] - __half2float(hi[e]));
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+        *reinterpret_cast<uint32_t*>(&sh.qterm[pj][g][0][4 * lane]) = w0;
+        *reinterpret_cast<uint32_t*>(&sh.qterm[pj][g][1][4 * lane]) = w1;
+        *reinterpret_cast<uint2*>(&sh.qh[pj][g][0][4 * lane]) = *reinterpret_cast<const uint2*>(hi);
+        *reinterpret_cast<uint2*>(&sh.qh[pj][g][1][4 * lane]) = *reinterpret_cast<const uint2*>(lo);
+        sum = __reduce_add_sync(FULL_MASK, sum);
         if (lane == 0) {
           sh.qscale[pj][g] = sigma / 254.f;
           sh.qsum[pj][g] = (sigma / 254.f) * (float)sum;
@@ -912,47 +965,84 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     // ---- this warp's items -----------------------------------------------------------
     SoftmaxState<NT> S;
     const int jl = warp_run<BITS, G, AFFINE>(a, wm, sh, u_first, y0, y1, warp, lane, it, ic, S);
-    __syncthreads();  // every copy ring is drained: the stage area becomes slots
-
-    float (*so)[G][D] = warp_slots(sh);
-    if (jl >= 0) state_to_slot<BITS, G, AFFINE>(S, so[warp], sh.sm[warp], sh.sl[warp], lane);
+    // The warp's ring has drained: its final state goes into its own stages
+    // (an idle warp's slot, maximum and sum are neutral: every slot is read
+    // below, with weight 0 where the warp is not a member).
+    if (jl >= 0) {
+      state_to_slot<BITS, G, AFFINE>(S, warp_slot(sh, warp), sh.sm[warp], sh.sl[warp], lane);
+      raise_segment_max(sh, jl, S.m, lane);
+    } else {
+      for (int e = lane; e < G * D; e += 32) warp_slot(sh, warp)[e / D][e % D] = 0.f;
+      if (lane < G) { sh.sm[warp][lane] = -INFINITY; sh.sl[warp][lane] = 0.f; }
+    }
     if (lane == 0) sh.wseg[warp] = jl;
     __syncthreads();
 
-    // ---- merge the partials of each segment into this CTA's partial for the unit --
-    // thread (head g, dim d): the segment's maximum over its warps and its
-    // boundary slot, then the weighted sums, all from shared-memory broadcasts
-    for (int jj = 0; jj < nseg; ++jj) {
-      const bool has_b = jj < nseg - 1 && sh.bused[jj];
-      const int uu = u_first + jj;
-      const uint32_t cta_u0 = cta_of(a, (uint32_t)uu * NI);
-      float* part_base = a.partials + ((size_t)uu * c.max_splits + (cta - cta_u0)) * G * PART;
-      for (int e = tid; e < G * D; e += NW * 32) {
-        const int g = e / D, d = e % D;
-        float M = has_b ? sh.bm[jj][g] : -INFINITY;
-        float mv[NW];
-        uint32_t members = 0;   // slots of other segments or of idle warps are never read
+    // ---- merge weights: thread (segment j, warp w, head g) --------------------------
+    for (int t = tid; t < UMAX * NW * G; t += NW * 32) {
+      const int j = t / (NW * G), w = (t / G) % NW, g = t % G;
+      sh.wf[j][w][g] = (j < nseg && sh.wseg[w] == j)
+                           ? merge_weight(sh.sm[w][g], order_float(sh.segMi[j][g])) : 0.f;
+      if (t < (UMAX - 1) * G) {
+        const int jb = t / G, gb = t % G;
+        sh.bf[jb][gb] = (jb < nseg - 1 && sh.bused[jb])
+                            ? merge_weight(sh.bm[jb][gb], order_float(sh.segMi[jb][gb])) : 0.f;
+      }
+    }
+    if (tid < nseg) {   // arrivals before the last one (0: the unit lies in this CTA alone)
+      const uint32_t ubj = (uint32_t)(u_first + tid) * NI;
+      sh.others[tid] = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj));
+    }
+    __syncthreads();
+
+    // ---- weighted sums: thread (head g, dim d), the slots in two halves of
+    // independent loads.  Segments that other CTAs also hold are published
+    // straight away.
+    constexpr int NH = (NW + 1) / 2;
+    for (int e = tid; e < G * D; e += NW * 32) {
+      const int g = e / D, d = e % D;
+      float Oj[UMAX];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const bool in = sh.wseg[w] == jj;
-          members |= (in ? 1u : 0u) << w;
-          mv[w] = in ? sh.sm[w][g] : -INFINITY;
-          M = fmaxf(M, mv[w]);
-        }
-        const float fb = has_b ? merge_weight(sh.bm[jj][g], M) : 0.f;
-        float O = has_b ? fb * sh.bo[jj][g][d] : 0.f;
-        float L = has_b ? fb * sh.bl[jj][g] : 0.f;
+      for (int jj = 0; jj < UMAX; ++jj)
+        Oj[jj] = (jj < nseg - 1 && sh.bused[jj]) ? sh.bf[jj][g] * sh.bo[jj][g][d] : 0.f;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          if (members >> w & 1u) {
-            const float f = merge_weight(mv[w], M);
-            O = fmaf(so[w][g][d], f, O);
-            L = fmaf(sh.sl[w][g], f, L);
+      for (int h0 = 0; h0 < NW; h0 += NH) {
+        float x[NH];
+#pragma unroll
+        for (int w = 0; w < NH; ++w) x[w] = h0 + w < NW ? warp_slot(sh, h0 + w)[g][d] : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < UMAX; ++jj) {
+          if (jj < nseg) {
+#pragma unroll
+            for (int w = 0; w < NH; ++w)
+              if (h0 + w < NW) Oj[jj] = fmaf(sh.wf[jj][h0 + w][g], x[w], Oj[jj]);
           }
         }
-        float* part = part_base + (size_t)g * PART;
-        part[d] = O;
-        if (d == 0) { part[D] = M; part[D + 1] = L; }
+      }
+#pragma unroll
+      for (int jj = 0; jj < UMAX; ++jj) {
+        if (jj >= nseg) break;
+        const bool has_b = jj < nseg - 1 && sh.bused[jj];
+        const float O = Oj[jj];
+        segment_sum(sh, jj)[g][d] = O;
+        float L = 0.f;
+        if (d == 0) {
+          L = has_b ? sh.bf[jj][g] * sh.bl[jj][g] : 0.f;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) L = fmaf(sh.wf[jj][w][g], sh.sl[w][g], L);
+          sh.segL[jj][g] = L;
+        }
+        if (sh.others[jj] > 0) {
+          const int uu = u_first + jj;
+          const uint32_t slot = cta - cta_of(a, (uint32_t)uu * NI);
+          if (slot < (uint32_t)c.max_splits) {
+            float* part = a.partials + (((size_t)uu * c.max_splits + slot) * G + g) * PART;
+            part[d] = O;
+            if (d == 0) { part[D] = order_float(sh.segMi[jj][g]); part[D + 1] = L; }
+          } else if (e == 0) {
+            atomicOr(c.status, DEV_ERR_SPLITS);   // the host's split bound was wrong: never write past it
+          }
+        }
       }
     }
 
@@ -962,13 +1052,15 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     // arrival, make the other CTAs' partials visible (acquire).
     __syncthreads();
     if (tid < nseg) {
-      const int uu = u_first + tid;
-      const uint32_t ubj = (uint32_t)uu * NI;
-      const int nparts = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj)) + 1;
-      int prevc;
-      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;\n"
-                   : "=r"(prevc) : "l"(a.counters + uu) : "memory");
-      sh.is_last[tid] = (prevc == nparts - 1);
+      int last = 1;
+      if (sh.others[tid] > 0) {
+        const int uu = u_first + tid;
+        int prevc;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;\n"
+                     : "=r"(prevc) : "l"(a.counters + (size_t)uu * c.counter_stride) : "memory");
+        last = prevc == sh.others[tid];
+      }
+      sh.is_last[tid] = last;
     }
     __syncthreads();
     // one warp per (segment, head) of the units this CTA completes
@@ -976,13 +1068,21 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
       const int jj = p / G, g = p % G;
       if (!sh.is_last[jj]) continue;
       const int uu = u_first + jj;
-      const uint32_t ubj = (uint32_t)uu * NI;
-      const int nparts = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj)) + 1;
+      const int bb = uu / c.n_kv_heads, hh = uu % c.n_kv_heads;
+      float* dst = a.out + ((size_t)bb * Hq + (size_t)hh * G + g) * D + 4 * lane;
+      if (sh.others[jj] == 0) {   // the whole unit lies in this CTA
+        const float4 O = reinterpret_cast<const float4*>(segment_sum(sh, jj)[g])[lane];
+        const float il = 1.f / sh.segL[jj][g];
+        *reinterpret_cast<float4*>(dst) = make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
+        continue;
+      }
+      const int nparts = min(sh.others[jj] + 1, c.max_splits);
       const float* pbase = a.partials + (size_t)uu * c.max_splits * G * PART + (size_t)g * PART;
-      // partials in rounds of eight, all loads of a round in flight at once;
-      // the running (M, L, O) is rescaled when a round raises M
       float M = -INFINITY, L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      // the partials in index order, in rounds of eight with all loads of a
+      // round in flight at once; the running (M, L, O) is rescaled when a
+      // round raises M
       for (int sp0 = 0; sp0 < nparts; sp0 += 8) {
         float4 v[8];
         float mw[8], lw[8];
@@ -1010,11 +1110,9 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
         }
       }
       const float il = 1.f / L;
-      const int bb = uu / c.n_kv_heads, hh = uu % c.n_kv_heads;
-      *reinterpret_cast<float4*>(a.out + ((size_t)bb * Hq + (size_t)hh * G + g) * D + 4 * lane) =
-          make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
+      *reinterpret_cast<float4*>(dst) = make_float4(O.x * il, O.y * il, O.z * il, O.w * il);
     }
-    if (tid < nseg && sh.is_last[tid]) a.counters[u_first + tid] = 0;
+    if (tid < nseg && sh.is_last[tid]) a.counters[(size_t)(u_first + tid) * c.counter_stride] = 0;
     __syncthreads();
     fence_proxy_async();  // the stage area was written as slots; the next batch's copies overwrite it
   }

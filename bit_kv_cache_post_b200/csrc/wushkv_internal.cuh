@@ -37,7 +37,8 @@ struct DevCache {
   int sink, recent, chunk, ring_slots;
   int packed_capacity;
   float* partials;                   // split-K workspace
-  int* counters;                     // one arrival counter per unit
+  int* counters;                     // one arrival counter per unit, counter_stride ints apart
+  int counter_stride;
   int max_splits;
   int* status;                       // sticky device error word
   int units, n_kv_heads, group;
@@ -76,8 +77,12 @@ __host__ __device__ __forceinline__ uint8_t* v_meta_at(const DevCache& c, int64_
          (uint64_t)(pk & 63) * c.meta_bytes;
 }
 
-// Status bits a kernel may set in the sticky word.
-enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2, DEV_ERR_TIMEOUT = 4 };
+// Status bits a kernel may set in the sticky word (values documented in
+// wushkv.h): a packed index past the capacity (the write is skipped), a
+// split partial index past the workspace (skipped), a copy that did not
+// complete within the wait limit.
+enum : int { DEV_ERR_RANGE = WUSHKV_DEV_RANGE, DEV_ERR_SPLITS = WUSHKV_DEV_SPLITS,
+             DEV_ERR_TIMEOUT = WUSHKV_DEV_TIMEOUT };
 
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch.  A kernel launched with
@@ -86,6 +91,10 @@ enum : int { DEV_ERR_RANGE = 1, DEV_ERR_SPLITS = 2, DEV_ERR_TIMEOUT = 4 };
 // memory that kernel writes or reads (a no-op when there is no such
 // kernel).  grid_dependents_may_launch() lets the next such kernel be
 // scheduled; it never skips the wait on the other side.
+//
+// Every kernel of this library calls grid_dependents_may_launch() only
+// after its own grid_dependency_wait(), so at most one kernel before it (its
+// immediate predecessor) can still be running when one of them starts.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
@@ -451,6 +460,8 @@ struct DecodeArgs {
   uint32_t cta_q, cta_r;   // stream-K split: CTA i starts at item i cta_q + min(i, cta_r)
   float* partials;         // split partials [unit][max_splits][G][132]
   int* counters;           // arrival counter per unit
+  uint32_t inject_polls;   // 0, or fault injection for tests: each warp's first copy wait is made on a
+                           // barrier nothing completes and gives up after this many polls
 };
 cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& m, cudaStream_t s);
 int decode_ctas_per_sm(int bits, int group, int quantizer);

@@ -20,8 +20,12 @@ EXPORTED = [
     "wushkv_cache_bytes", "wushkv_cache_create", "wushkv_cache_destroy", "wushkv_cache_layout",
     "wushkv_cache_tokens", "wushkv_append", "wushkv_query_transform", "wushkv_decode",
     "wushkv_export", "wushkv_device_status", "wushkv_default_quest_alpha", "wushkv_strerror",
-    "wushkv_decode_noalloc", "wushkv_decode_step",
+    "wushkv_decode_noalloc", "wushkv_decode_step", "wushkv_inject_decode_timeout",
 ]
+
+# bits of the sticky device status word; guard bands after each cache region
+DEV_RANGE, DEV_SPLITS, DEV_TIMEOUT = 1, 2, 4
+GUARD_BYTES, GUARD_FILL = 256, 0xA5
 
 
 class Config(ctypes.Structure):
@@ -82,12 +86,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_export.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.wushkv_device_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
+    lib.wushkv_inject_decode_timeout.argtypes = [ctypes.c_uint32]
+    lib.wushkv_inject_decode_timeout.restype = None
     lib.wushkv_default_quest_alpha.argtypes = [i32]
     lib.wushkv_default_quest_alpha.restype = ctypes.c_double
     lib.wushkv_strerror.argtypes = [i32]
     lib.wushkv_strerror.restype = ctypes.c_char_p
     for name in EXPORTED:
-        if name not in ("wushkv_cache_bytes", "wushkv_default_quest_alpha", "wushkv_strerror"):
+        if name not in ("wushkv_cache_bytes", "wushkv_default_quest_alpha", "wushkv_strerror",
+                        "wushkv_inject_decode_timeout"):
             getattr(lib, name).restype = ctypes.c_int32
     _LIB = lib
     return lib
@@ -130,6 +137,12 @@ def cache_bytes(cfg: Config) -> int:
 
 def default_quest_alpha(bits: int) -> float:
     return float(load().wushkv_default_quest_alpha(bits))
+
+
+def inject_decode_timeout(polls: int) -> None:
+    """Failure injection for tests: with polls > 0 each decode warp's first
+    copy wait runs out after that many polls (0 turns it off)."""
+    load().wushkv_inject_decode_timeout(int(polls))
 
 
 class Cache:
@@ -246,6 +259,15 @@ class Cache:
         _check(load().wushkv_export(self._handle, seq, head, kv, tok0, ntok, p(codes), p(meta),
                                     p(rows), p(kinds)), "wushkv_export")
         return codes, meta, rows, kinds
+
+    def guard_offsets(self) -> list[int]:
+        """Offsets (from the cache base) of the guard bands that follow the
+        packed region, sink K, sink V, ring K, ring V and the workspace."""
+        L = self.layout()
+        U = self.cfg.batch * self.cfg.n_kv_heads
+        return [U * L.unit_stride, L.sink_k_off + U * L.sink_unit_stride,
+                L.sink_v_off + U * L.sink_unit_stride, L.ring_k_off + U * L.ring_unit_stride,
+                L.ring_v_off + U * L.ring_unit_stride, L.workspace_off + L.workspace_bytes]
 
     def device_status(self, clear: bool = False) -> int:
         out = ctypes.c_int32()

@@ -62,6 +62,15 @@ typedef enum {
 } wushkv_status;
 
 typedef enum { WUSHKV_QUEST_INT = 0, WUSHKV_AFFINE_PCTCLIP = 1 } wushkv_quantizer;
+
+/* Bits of the sticky device status word (wushkv_device_status).  A kernel
+ * that detects one of these conditions skips the offending access, sets the
+ * bit and finishes; the call's results are then not to be trusted.
+ *   WUSHKV_DEV_RANGE:   a packed token index beyond the cache's capacity.
+ *   WUSHKV_DEV_SPLITS:  a decode split partial beyond the workspace.
+ *   WUSHKV_DEV_TIMEOUT: an asynchronous copy did not complete within the
+ *                       wait limit (about a second by default). */
+enum { WUSHKV_DEV_RANGE = 1, WUSHKV_DEV_SPLITS = 2, WUSHKV_DEV_TIMEOUT = 4 };
 typedef enum { WUSHKV_F16 = 0, WUSHKV_BF16 = 1, WUSHKV_F32 = 2 } wushkv_dtype;
 
 /* Cache configuration (one layer).
@@ -122,7 +131,13 @@ typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
  *   meta: per token, fp16 delta (QuEST, 2 bytes) or fp16 (scale, lo) pair
  *     (affine, 4 bytes); K and V separately.
  *   sink, ring: fp16 [unit][slot][128]; ring slot of post-sink token t is
- *     (t - sink) mod (recent + chunk). */
+ *     (t - sink) mod (recent + chunk).
+ * Guard bands: the packed region, sink K, sink V, ring K, ring V and the
+ *   workspace are each followed by WUSHKV_GUARD_BYTES bytes set to
+ *   WUSHKV_GUARD_FILL at creation, which no kernel writes (a test that finds
+ *   them changed has found an out-of-bounds write). */
+#define WUSHKV_GUARD_BYTES 256
+#define WUSHKV_GUARD_FILL 0xA5
 typedef struct {
   int32_t n_planes;
   int32_t plane_bits[2];
@@ -241,8 +256,10 @@ WUSHKV_API wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_r
  * the cache buffer's workspace.  It calls no cudaMalloc, cudaFree or other
  * allocating routine.
  *   - The first call on each device looks up the array's device address
- *     (with that device current); make that first call before any stream
- *     capture.
+ *     (with that device current).  Under lazy module loading that lookup
+ *     can load the library's device code and allocate the array, so make
+ *     the first call on each device during start-up, where allocation is
+ *     still allowed, and before any stream capture.
  *   - All calls share the one array, which keeps the previous call's
  *     contents; each call zeroes its arrival counters first.  Calls that
  *     overlap on the GPU (other streams, threads or caches) race: issue
@@ -267,8 +284,20 @@ WUSHKV_API wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, i
                             uint16_t* fp16_host, int8_t* kinds_host);
 
 /* Read (and with clear != 0, reset) the sticky device status word;
- * synchronises the device.  0 means no kernel reported an error. */
+ * synchronises the device.  0 means no kernel reported an error; otherwise
+ * an OR of the WUSHKV_DEV_* bits. */
 WUSHKV_API wushkv_status wushkv_device_status(const wushkv_cache* cache, int32_t clear, int32_t* out);
+
+/* Failure injection, for tests of the timeout path without a GPU fault.
+ * With polls > 0, every decode launched afterwards (from any thread) makes
+ * each warp's first copy wait on a barrier that nothing completes, giving
+ * up after `polls` polls.  The warp then takes its real timeout path: it
+ * records WUSHKV_DEV_TIMEOUT in the cache's status word, waits (at the full
+ * limit, about a second) for the copies it has in flight, and contributes
+ * nothing more; the call returns normally, its output is not meaningful,
+ * and later decodes are unaffected.  polls = 0 turns the injection off.
+ * Not part of the method: the paper has no counterpart. */
+WUSHKV_API void wushkv_inject_decode_timeout(uint32_t polls);
 
 /* Gaussian-MSE-optimal QuEST clip ratio for 2, 3 or 4 bits (0 otherwise). */
 WUSHKV_API double wushkv_default_quest_alpha(int32_t bits);

@@ -110,6 +110,7 @@ def compare_cache_bitexact(cache, oc: O.OracleCache, units=None):
             ring = unit_window(cache, u, kv, "ring")[oc.recent_order()]
             oring = (oc.ring_k if kv == 0 else oc.ring_v)[u, oc.recent_order()]
             assert np.array_equal(ring.view(np.uint16), oring.view(np.uint16)), (u, kv)
+    check_guards(cache)
 
 
 def rel_rms_err(got: np.ndarray, want: np.ndarray) -> float:
@@ -153,3 +154,33 @@ def check_unit_transformed(cache, oc: O.OracleCache, ou: int, T_h, k_h, u: int):
     assert np.array_equal(unit_meta(cache, u, 1, P).view(np.uint16),
                           oc.meta_v[ou, :P, :gm.shape[1]].view(np.uint16))
     return mism
+
+
+def check_guards(cache):
+    """The guard bands after every cache region still hold their fill byte
+    (no kernel wrote past a region)."""
+    from bit_kv_cache_post_b200 import wushkv as wk
+    for off in cache.guard_offsets():
+        band = region(cache, off, wk.GUARD_BYTES)
+        assert np.all(band == wk.GUARD_FILL), ("guard band written", off)
+
+
+def unit_state_from_export(cache, b: int, h: int):
+    """(K, V) of unit (b, h) as the GPU cache holds them, read through
+    wushkv_export and dequantised with the oracle's reconstruction rules:
+    fp16 rows for window tokens, (codes, scales) for packed ones."""
+    cfg = cache.cfg
+    n = cache.tokens()[0]
+    out = []
+    for kv in (0, 1):
+        codes, meta, rows, kinds = cache.export(b, h, kv, 0, n)
+        x = rows.view(np.float16).astype(np.float64)
+        pk = kinds == 1
+        if pk.any():
+            m = meta[pk].view(np.float16)
+            if cfg.quantizer == O.QUEST_INT:
+                x[pk] = O.quest_dequantize(codes[pk], m[:, 0], cfg.bits)
+            else:
+                x[pk] = O.affine_dequantize(codes[pk], m[:, 0], m[:, 1])
+        out.append(x)
+    return out[0], out[1]

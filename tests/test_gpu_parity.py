@@ -90,6 +90,57 @@ def test_degenerate_tokens(wk):
         H.compare_cache_bitexact(cache, oc)
 
 
+@pytest.mark.parametrize("ranks", [(1, 128), (8, 121), (3, 124)])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_affine_ranks_bitexact(wk, bits, ranks):
+    """Order statistics other than the default (2, 127): the extreme ranks
+    (no clipping) and the deepest supported ones, on one bulk append and on
+    single-token appends across flushes; then a decode."""
+    n = sum(SCHEDULE)
+    cfg = wk.make_config(2, 2, 8, 720, bits=bits, quantizer=O.AFFINE_PCTCLIP,
+                         clip_lo_rank=ranks[0], clip_hi_rank=ranks[1])
+    k, v = _kv(100 * bits + ranks[0], 2, n, 2)
+    for sched in ([n], SCHEDULE):
+        cache, oc = _append_both(wk, cfg, k, v, None, "f32", sched)
+        H.compare_cache_bitexact(cache, oc)
+    out, want = _decode_both(wk, cache, oc, 17)
+    assert H.rel_rms_err(out, want) <= DECODE_TOL
+
+
+@pytest.mark.parametrize("quantizer", [O.QUEST_INT, O.AFFINE_PCTCLIP])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_export_matches_oracle(wk, bits, quantizer):
+    """wushkv_export unpacks K and V of sink, packed and recent tokens of a
+    unit: codes, scales and fp16 rows equal the oracle's state."""
+    n = 64 + 256 + 8 * 23 + 5
+    cfg = wk.make_config(2, 3, 6, n + 8, bits=bits, quantizer=quantizer)
+    k, v = _kv(7 * bits + quantizer, 2, n, 3)
+    cache, oc = _append_both(wk, cfg, k, v, None, "f32", [n - 9] + [1] * 9)
+    ns, P, nr = oc.split()
+    W = cfg.recent + cfg.chunk
+    for (b, h) in [(0, 0), (1, 2)]:
+        u = b * cfg.n_kv_heads + h
+        for kv in (0, 1):
+            codes, meta, rows, kinds = cache.export(b, h, kv, 0, n)
+            sink = oc.sink_k if kv == 0 else oc.sink_v
+            ring = oc.ring_k if kv == 0 else oc.ring_v
+            ocodes = oc.codes_k if kv == 0 else oc.codes_v
+            ometa = oc.meta_k if kv == 0 else oc.meta_v
+            assert np.array_equal(kinds[:ns], np.zeros(ns))
+            assert np.array_equal(kinds[ns:ns + P], np.ones(P))
+            assert np.array_equal(kinds[ns + P:], np.full(nr, 2))
+            assert np.array_equal(rows[:ns], sink[u, :ns].view(np.uint16))
+            slots = [(t - cfg.sink) % W for t in range(ns + P, n)]
+            assert np.array_equal(rows[ns + P:], ring[u, slots].view(np.uint16))
+            assert np.array_equal(codes[ns:ns + P], ocodes[u, :P])
+            nm = 2 if quantizer == O.AFFINE_PCTCLIP else 1
+            assert np.array_equal(meta[ns:ns + P, :nm], ometa[u, :P, :nm].view(np.uint16))
+            assert not codes[:ns].any() and not codes[ns + P:].any() and not rows[ns:ns + P].any()
+        # a range starting and ending inside the packed tokens
+        codes, _, _, kinds = cache.export(b, h, 0, ns + 5, 70)
+        assert np.array_equal(codes, oc.codes_k[u, 5:75]) and np.all(kinds == 1)
+
+
 def _decode_both(wk, cache, oc, seed, scale=0.0):
     import torch
     cfg = cache.cfg
@@ -97,6 +148,8 @@ def _decode_both(wk, cache, oc, seed, scale=0.0):
     qd = torch.from_numpy(q).cuda()
     out = cache.decode(qd, scale=scale).cpu().numpy()
     want = oc.decode(q.astype(np.float64), None if scale == 0.0 else scale)
+    assert cache.device_status() == 0
+    H.check_guards(cache)
     return out, want
 
 
@@ -110,6 +163,23 @@ def test_decode_matches_oracle(wk, G, n):
     cache, oc = _append_both(wk, cfg, k, v, None, "f32", [n])
     out, want = _decode_both(wk, cache, oc, n + G)
     assert H.rel_rms_err(out, want) <= DECODE_TOL
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_decode_many_ctas_per_unit(wk, G):
+    """Two units of 30000 tokens: every CTA of the grid holds a few items of
+    one unit (most warps one item, several none), ~70 partials per unit;
+    repeated decodes give the same bits."""
+    import torch
+    n = 30000
+    cfg = wk.make_config(1, 2, 2 * G, n, bits=2)
+    k, v = _kv(4000 + G, 1, n, 2)
+    cache, oc = _append_both(wk, cfg, k, v, None, "f32", [n])
+    out, want = _decode_both(wk, cache, oc, 11)
+    assert H.rel_rms_err(out, want) <= DECODE_TOL
+    q = torch.from_numpy(np.random.default_rng(11).standard_normal((1, 2 * G, 128)).astype(np.float32)).cuda()
+    for _ in range(3):
+        assert np.array_equal(cache.decode(q).cpu().numpy(), out)
 
 
 @pytest.mark.parametrize("quantizer", [O.QUEST_INT, O.AFFINE_PCTCLIP])

@@ -44,7 +44,7 @@ def _transforms(Hkv):
     return T[:Hkv], TinvT[:Hkv]
 
 
-def _run(wk, cfg, k, v, q, T, TinvT, schedule, units):
+def _run(wk, cfg, k, v, q, T, TinvT, schedule, units, decode_on_gpu_state=False):
     import torch
     cache = wk.Cache(cfg)
     Td = torch.from_numpy(T).cuda()
@@ -72,7 +72,13 @@ def _run(wk, cfg, k, v, q, T, TinvT, schedule, units):
         assert oc.split() == cache.tokens()[1:]
         mism.append(H.check_unit_transformed(cache, oc, 0, T[h], k[b, :, h], u))
         qprime = O.transform_query(q[b, h * G:(h + 1) * G], TinvT[h].astype(np.float64))
-        want = oc.decode(qprime[None])[0]
+        if decode_on_gpu_state:
+            # the decode against exact attention over the cache the GPU built
+            # (boundary flips of k' codes then cannot enter the comparison)
+            Kg, Vg = H.unit_state_from_export(cache, b, h)
+            want = O.attention_f64(qprime, Kg, Vg, 1.0 / np.sqrt(128.0))
+        else:
+            want = oc.decode(qprime[None])[0]
         assert H.rel_rms_err(out[b, h * G:(h + 1) * G], want) <= DECODE_TOL
     return cache, mism
 
@@ -114,3 +120,32 @@ def test_many_units_short_prefill(wk):
     cfg = wk.make_config(B, Hkv, 4 * Hkv, n + 32, bits=2, quantizer=O.AFFINE_PCTCLIP, chunk=16)
     cache, _ = _run(wk, cfg, k, v, q, T, TinvT, [n], [(0, 0), (5, 3), (15, 7)])
     assert cache.tokens()[2] == 304
+
+
+@pytest.mark.parametrize("ranks", [(1, 128), (2, 128), (1, 127)])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_bulk_prefill_affine_ranks(wk, bits, ranks):
+    """Affine ranks other than (2, 127) that the tensor-core append serves
+    (lowest rank <= 2, highest >= 127): the epilogue's branches without the
+    second order statistic."""
+    B, Hkv, n = 2, 2, 64 + 256 + 8 * 60 + 3
+    k, v, q = _inputs(1000 * bits + ranks[0] + ranks[1], B, n, Hkv)
+    T, TinvT = _transforms(Hkv)
+    cfg = wk.make_config(B, Hkv, 4 * Hkv, n + 16, bits=bits, quantizer=O.AFFINE_PCTCLIP,
+                         clip_lo_rank=ranks[0], clip_hi_rank=ranks[1])
+    cache, _ = _run(wk, cfg, k, v, q, T, TinvT, [n], [(b, h) for b in range(B) for h in range(Hkv)],
+                    decode_on_gpu_state=True)
+    H.check_guards(cache)
+
+
+def test_bulk_prefill_deep_ranks_fma_path(wk):
+    """Affine ranks (8, 121) with bf16 keys through T: the FMA append path
+    (warp rank selection) against the oracle."""
+    B, Hkv, n = 2, 2, 64 + 256 + 8 * 30 + 1
+    k, v, q = _inputs(4242, B, n, Hkv)
+    T, TinvT = _transforms(Hkv)
+    cfg = wk.make_config(B, Hkv, 4 * Hkv, n + 16, bits=2, quantizer=O.AFFINE_PCTCLIP,
+                         clip_lo_rank=8, clip_hi_rank=121)
+    cache, _ = _run(wk, cfg, k, v, q, T, TinvT, [n - 40] + [1] * 40,
+                    [(b, h) for b in range(B) for h in range(Hkv)], decode_on_gpu_state=True)
+    H.check_guards(cache)

@@ -27,9 +27,9 @@ def wk():
     return wushkv
 
 
-def _filled_cache(wk, B, Hkv, G, n, seed):
+def _filled_cache(wk, B, Hkv, G, n, seed, quantizer=0):
     import torch
-    cfg = wk.make_config(B, Hkv, Hkv * G, n + 8, bits=2)
+    cfg = wk.make_config(B, Hkv, Hkv * G, n + 8, bits=2, quantizer=quantizer)
     cache = wk.Cache(cfg)
     g = np.random.default_rng(seed)
     k = torch.from_numpy(g.standard_normal((B, n, Hkv, 128)).astype(np.float32)).cuda()
@@ -38,14 +38,24 @@ def _filled_cache(wk, B, Hkv, G, n, seed):
     return cache
 
 
-def test_noalloc_matches_decode_two_calls(wk):
+# (batch, KV heads, G, tokens, quantizer): QuEST at G = 4; the affine
+# quantizer at G = 8 (larger partials); one long sequence of 2 units spread
+# over many CTAs each (the partials-per-unit bound is reached)
+CASES = [(4, 4, 4, 2000, 0), (2, 2, 8, 1500, 1), (1, 2, 4, 40000, 0)]
+
+
+@pytest.mark.parametrize("B,Hkv,G,n,quantizer", CASES)
+def test_noalloc_matches_decode_two_calls(wk, B, Hkv, G, n, quantizer):
+    """Same plan, same arithmetic, same merge order as wushkv_decode: the
+    outputs are bitwise equal (and within the decode tolerance, which the
+    parity tests hold wushkv_decode to)."""
     import torch
     lib = wk.load()
-    cache = _filled_cache(wk, 4, 4, 4, 2000, 0)
+    cache = _filled_cache(wk, B, Hkv, G, n, 0, quantizer)
     stream = torch.cuda.current_stream().cuda_stream or None
     g = np.random.default_rng(1)
     for call in range(2):
-        q = torch.from_numpy(g.standard_normal((4, 16, 128)).astype(np.float32)).cuda()
+        q = torch.from_numpy(g.standard_normal((B, Hkv * G, 128)).astype(np.float32)).cuda()
         ref = torch.empty_like(q)
         out = torch.full_like(q, float("nan"))
         assert lib.wushkv_decode(q.data_ptr(), cache.handle, ref.data_ptr(), ctypes.c_float(0.0),
@@ -56,6 +66,7 @@ def test_noalloc_matches_decode_two_calls(wk):
         r, o = ref.cpu().numpy(), out.cpu().numpy()
         err = np.abs(o - r).max() / np.sqrt(np.mean(r ** 2))
         assert np.isfinite(o).all() and err <= DECODE_TOL, (call, err)
+        assert torch.equal(out, ref), call
     assert cache.device_status() == 0
 
 
