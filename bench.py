@@ -45,6 +45,11 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--only-prefill", action="store_true",
+                    help="run only the bulk-prefill measurement (for profiling)")
+    ap.add_argument("--prefill-batch", type=int, default=0,
+                    help="sequences of the bulk prefill (default: the workload's 64)")
     return ap.parse_args()
 
 
@@ -173,6 +178,38 @@ def window_state(n, w):
     return n, ns, P, m - P
 
 
+def decode_graph_us(caches, qprime, out, torch, device, launches=4000):
+    """Microseconds per decode launch: one launch per cache back to back in a
+    CUDA graph (no host gaps), the replays bracketed by CUDA events on the
+    launching stream; time / launches.  The caches are cycled, so every
+    launch reads bytes that the previous ones evicted from L2."""
+    stream = torch.cuda.current_stream()
+    capture = torch.cuda.Stream(device=device)
+    capture.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(capture):
+        for c in caches:                      # untimed: attributes, first-use set-up
+            c.decode(qprime, out=out, stream=capture)
+        capture.synchronize()
+        with torch.cuda.graph(graph, stream=capture):
+            for c in caches:
+                c.decode(qprime, out=out, stream=capture)
+    stream.wait_stream(capture)
+    reps = max(3, min(200, launches // len(caches)))
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    us = g0.elapsed_time(g1) * 1e3 / (reps * len(caches))
+    del graph
+    return us
+
+
 def run_ours(args, rank, world, device, torch, dist):
     from bit_kv_cache_post_b200 import inputs as I
     from bit_kv_cache_post_b200 import wushkv as wk
@@ -234,8 +271,10 @@ def run_ours(args, rank, world, device, torch, dist):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
         t0.record(stream)
+        h0 = time.perf_counter()
         for i in range(args.warmup, args.warmup + K):
             step(i, *dev_pool[i % STEP_POOL])
+        host_s = time.perf_counter() - h0
         t1.record(stream)
         torch.cuda.synchronize()
     if dist is not None:
@@ -246,33 +285,9 @@ def run_ours(args, rank, world, device, torch, dist):
     launches_per_step = 2
     status = max(c.device_status() for c in caches)
 
-    # ---- the decode kernel alone (roofline): one decode per cycled cache,
-    # back to back in a CUDA graph (no host gaps), the replays bracketed by
-    # CUDA events on the launching stream; per-launch time = total / launches
-    capture = torch.cuda.Stream(device=device)
-    capture.wait_stream(stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(capture):
-        for c in range(args.copies):          # untimed: attributes, first-use set-up
-            caches[c].decode(qprime, out=out, stream=capture)
-        capture.synchronize()
-        with torch.cuda.graph(graph, stream=capture):
-            for c in range(args.copies):
-                caches[c].decode(qprime, out=out, stream=capture)
-    stream.wait_stream(capture)
-    reps = max(3, min(200, 4000 // args.copies))
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    g1.record(stream)
-    torch.cuda.synchronize()
-    dec_ms = [g0.elapsed_time(g1) / (reps * args.copies)]
+    # ---- the decode kernel alone (roofline) ------------------------------------
+    dec_ms = [decode_graph_us(caches, qprime, out, torch, device) / 1e3]
     dec_launch_bytes = [decode_bytes(w, bits, window_state(counts_after[c], w)) for c in range(args.copies)]
-    del graph
     counts = counts_after
 
     # ---- e2e: host buffers, copies inside the timed region --------------------
@@ -308,7 +323,7 @@ def run_ours(args, rank, world, device, torch, dist):
     if dist is not None:
         e_ms = max_over_ranks(e_ms, dist, device)
 
-    return dict(w=w, bits=bits, K=K, ms=ms, dec_total=dec_total, rest_total=rest_total,
+    return dict(w=w, bits=bits, K=K, ms=ms, dec_total=dec_total, rest_total=rest_total, host_s=host_s,
                 dec_ms=dec_ms, dec_launch_bytes=dec_launch_bytes, clocks=clocks.summary(),
                 launches=launches_per_step * K,
                 status=status, e2e=(E, e_ms, e_dec, h2d, d2h), copies=args.copies,
@@ -318,7 +333,7 @@ def run_ours(args, rank, world, device, torch, dist):
 PREFILL_WORKLOAD = "qwen3-8b-stack36-b64-prefill32768"
 
 
-def run_prefill(device, torch, reps=5):
+def run_prefill(device, torch, reps=5, batch=0):
     """Bulk append of one layer of the 36-layer workload (batch 64, 32768
     bf16 tokens per sequence, 2-bit percentile-clipped affine): key transform
     on the tensor cores, quantise + pack, values packed.  Each timed append
@@ -327,6 +342,9 @@ def run_prefill(device, torch, reps=5):
     from bit_kv_cache_post_b200 import inputs as I
     from bit_kv_cache_post_b200 import wushkv as wk
     w = I.WORKLOADS[PREFILL_WORKLOAD]
+    if batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=batch)
     n = w.context
     k, v = I.device_kv(w, 0, n, device=device)
     T, _ = I.key_transforms(w, 0)
@@ -363,6 +381,89 @@ def run_prefill(device, torch, reps=5):
             "key_transform_tflops": flops / (ms / 1e3) / 1e12, "device_status": status,
             "bytes_per_token_head": 2 * 128 * 2 + 2 * (16 * 2 + 4), "peak_source": src,
             "timing": f"median of {reps} appends into a fresh cache, CUDA events"}
+
+
+def run_workload_decode(name, device, torch, copies, bits=2):
+    """Decode throughput of one of the other workloads: `copies` independent
+    caches (together larger than L2) filled by one bulk bf16 append through
+    the key transform, then decode launches back to back in a CUDA graph."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[name]
+    n = w.context
+    affine = w.quantizer == "affine"
+    k, v = I.device_kv(w, 0, n, device=device)
+    T, TinvT = I.key_transforms(w, 0)
+    Td, TinvTd = torch.from_numpy(T).to(device), torch.from_numpy(TinvT).to(device)
+    cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, n + 128, bits=bits,
+                         quantizer=wk.AFFINE_PCTCLIP if affine else wk.QUEST_INT,
+                         sink=w.sink, recent=w.recent, chunk=w.chunk,
+                         clip_lo_rank=w.r_lo, clip_hi_rank=w.r_hi)
+    caches = []
+    for _ in range(copies):
+        c = wk.Cache(cfg, device=device)
+        c.append(k, v, Td)
+        caches.append(c)
+    del k, v
+    qprime = wk.query_transform(I.device_queries(w, 0, 0, device=device), TinvTd)
+    out = torch.empty_like(qprime)
+    torch.cuda.synchronize()
+    us = decode_graph_us(caches, qprime, out, torch, device)
+    status = max(c.device_status() for c in caches)
+    nbytes = decode_bytes(w, bits, window_state(n, w))
+    peak, _ = peaks()
+    res = {"workload": f"{name} ({bits}-bit {'affine' if affine else 'QuEST INT'}, G {w.group}, "
+                       f"batch {w.batch}, {n} tokens)",
+           "decode_us": us, "bytes_per_launch": nbytes, "gbs": nbytes / us / 1e3,
+           "frac": nbytes / us / 1e3 / peak, "copies": copies,
+           "l2": f"{copies} cycled caches of {nbytes / 1e6:.1f} MB", "device_status": status}
+    return res, caches, w, Td
+
+
+def run_append_steps(caches, w, Td, device, torch, steps=64):
+    """One-token appends (key transform, fp16 ring, a chunk flush every
+    `chunk` steps) on one cache, each a separate call as a serving loop
+    makes them; CUDA events around the whole run."""
+    from bit_kv_cache_post_b200 import inputs as I
+    cache = caches[0]
+    ks, vs = I.device_kv(w, 0, steps, device=device, step=1)
+    stream = torch.cuda.current_stream()
+    for i in range(4):                       # untimed warm-up of the launch path
+        cache.append(ks[:, i:i + 1].contiguous(), vs[:, i:i + 1].contiguous(), Td)
+    rows = [(ks[:, i:i + 1].contiguous(), vs[:, i:i + 1].contiguous()) for i in range(4, steps)]
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for kk, vv in rows:
+        cache.append(kk, vv, Td)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"tokens_per_s": len(rows) * w.batch / (ms / 1e3), "us_per_append": ms * 1e3 / len(rows),
+            "appends": len(rows), "flushes": len(rows) // w.chunk, "chunk": w.chunk,
+            "device_status": cache.device_status(),
+            "timing": "one-token wushkv_append calls back to back, CUDA events around the run"}
+
+
+def run_extra(device, torch):
+    """Decode GB/s of the 32B-shaped, 4B-shaped long-context and 36-layer
+    (one layer, affine) workloads, config-1 decode at 3 and 4 bits, and the
+    long-context workload's one-token appends with their 16-token flushes."""
+    out = {}
+    for name, copies, bits in (("qwen3-32b-layer-b32-ctx32768", 2, 2), ("qwen3-4b-b1-ctx131072", 8, 2),
+                               ("qwen3-8b-stack36-b64-prefill32768", 2, 2),
+                               ("qwen3-8b-layer-b16-ctx8192", 8, 3), ("qwen3-8b-layer-b16-ctx8192", 8, 4)):
+        res, caches, w, Td = run_workload_decode(name, device, torch, copies, bits)
+        key = f"{name}_{bits}bit"
+        if w.layers > 1:
+            res["decode_us_all_layers"] = res["decode_us"] * w.layers
+            res["layers"] = w.layers
+        if name == "qwen3-4b-b1-ctx131072":
+            out["append_" + name] = run_append_steps(caches, w, Td, device, torch)
+        out[key] = res
+        del caches
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -468,23 +569,25 @@ DECODE_SOURCES = ["bit_kv_cache_post_b200/csrc/decode.cu", "bit_kv_cache_post_b2
                   "bit_kv_cache_post_b200/csrc/wushkv_internal.cuh"]
 
 
-def decode_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, or None
-    when the decode kernel's sources changed since that capture."""
+def decode_traffic(bytes_per_launch):
+    """DRAM bytes (read + write) of one decode launch, from the committed ncu
+    record of this workload, scaled from the captured launch's algorithmic
+    bytes to this run's (the traffic grows with the cache bytes); None when
+    the decode kernel's sources changed since that capture."""
     import hashlib
     try:
-        txt = open(os.path.join(ROOT, "profiles", "decode_kernel_qwen3-8b-layer-b16-ctx8192.md")).read()
-        rec = dict(line.split(": ", 1) for line in txt.splitlines()
-                   if line.startswith(("traffic_bytes_per_launch: ", "kernel_sources_sha256: ")))
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+            rec = json.load(f)
         h = hashlib.sha256()
         for p in DECODE_SOURCES:
             with open(os.path.join(ROOT, p), "rb") as f:
                 h.update(f.read())
-        if h.hexdigest() != rec["kernel_sources_sha256"].strip():
-            return None
-        return int(rec["traffic_bytes_per_launch"])
+        if h.hexdigest() != rec["kernel_sources_sha256"]:
+            return None, None
+        ratio = rec["traffic_bytes_per_launch"] / rec["algorithmic_bytes_per_launch"]
+        return int(round(ratio * bytes_per_launch)), ratio
     except Exception:
-        return None
+        return None, None
 
 
 def peaks():
@@ -525,6 +628,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.only_prefill:
+        if rank == 0:
+            print(json.dumps({"prefill": run_prefill(device, torch, batch=args.prefill_batch)}))
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     r = run_ours(args, rank, world, device, torch, dist)
     w, bits, K = r["w"], r["bits"], r["K"]
     step_bytes = r["dec_total"] + r["rest_total"]
@@ -533,6 +642,7 @@ def main():
     dec_launch_bytes = float(np.mean(r["dec_launch_bytes"]))
     achieved = dec_launch_bytes / (dec_avg_ms / 1e3) / 1e9
     peak, peak_src = peaks()
+    traffic, traffic_ratio = decode_traffic(dec_launch_bytes)
     E, e_ms, e_dec, h2d, d2h = r["e2e"]
     line = {
         "metric": METRIC_NAME, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -542,7 +652,8 @@ def main():
         "decode_gbs": world * r["dec_total"] / (r["ms"] / 1e3) / 1e9,
         "append_tokens_per_s": w.batch * K / (r["ms"] / 1e3),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": decode_traffic(), "kernel": "decode",
+                     "frac": achieved / peak, "traffic": traffic, "traffic_over_algorithmic": traffic_ratio,
+                     "kernel": "decode",
                      "peak_source": peak_src, "frac_of_8tbs": achieved / 8000.0,
                      "launch_ms": dec_avg_ms, "bytes_per_launch": dec_launch_bytes,
                      "timing": "decode launches alone over the same cycled caches after the timed steps: "
@@ -551,11 +662,20 @@ def main():
         "e2e": {"value": world * e_dec / (e_ms / 1e3) / 1e9 if E else None,
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": E, "counts": "step bytes / step time incl. pinned host<->device copies"},
+        "step_breakdown": {"host_enqueue_us_per_step": r["host_s"] * 1e6 / K,
+                           "decode_us": dec_avg_ms * 1e3,
+                           "append_and_query_transform_us": r["ms"] * 1e3 / K - dec_avg_ms * 1e3,
+                           "note": "per step: the step kernel (key append, query transform, chunk flush "
+                                   "every 8th step) runs before the decode; its time here is the step "
+                                   "time minus the decode launch time"},
         "gpu_launches": r["launches"], "clocks": r["clocks"], "device_status": r["status"],
     }
     if rank == 0 and world == 1 and not args.no_prefill:
         torch.cuda.empty_cache()
         line["prefill"] = run_prefill(device, torch)
+    if rank == 0 and world == 1 and not args.no_extra:
+        torch.cuda.empty_cache()
+        line["workloads"] = run_extra(device, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, bits)
     if dist is not None:
