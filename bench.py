@@ -466,6 +466,48 @@ def run_extra(device, torch):
     return out
 
 
+def run_output_error(device, torch, B=4, n=2048):
+    """Module-output-error diagnostic through the library (summary page
+    关键实验: relative error of the attention output with the quantised cache,
+    geometric mean over (sequence, query head)).  Qwen3-8B-shaped heads with
+    the x20 outlier-channel keys, bf16 inputs; transforms: identity, a
+    randomised Hadamard rotation, a random invertible T.  The reference is
+    exact float64 attention over the same bf16 keys and values, computed with
+    plain torch ops."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[WORKLOAD]
+    k = torch.from_numpy(np.stack([I.keys(w, 1, b, n) for b in range(B)])).to(device).bfloat16()
+    v = torch.from_numpy(np.stack([I.values(w, 1, b, n) for b in range(B)])).to(device).bfloat16()
+    q = torch.from_numpy(np.stack([I.queries(w, 1, b) for b in range(B)])).to(device).bfloat16()
+    G = w.group
+    # exact reference: softmax(q k^T / sqrt(d)) v per (sequence, query head)
+    k64, v64, q64 = k.double(), v.double(), q.double()
+    kh = k64.permute(0, 2, 1, 3).repeat_interleave(G, dim=1)          # [B, Hq, n, d]
+    vh = v64.permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    p = torch.softmax(torch.einsum("bhd,bhnd->bhn", q64, kh) / math.sqrt(128.0), dim=-1)
+    ref = torch.einsum("bhn,bhnd->bhd", p, vh)
+    arms = {"identity": I.identity_transforms(w), "hadamard": I.hadamard_transforms(w, 1),
+            "random_invertible": I.key_transforms(w, 1)}
+    table = {}
+    for name, (T, TinvT) in arms.items():
+        Td, TinvTd = torch.from_numpy(T).to(device), torch.from_numpy(TinvT).to(device)
+        for quantizer, qname in ((wk.QUEST_INT, "quest"), (wk.AFFINE_PCTCLIP, "affine")):
+            row = {}
+            for bits in (2, 3, 4):
+                cache = wk.Cache(wk.make_config(B, w.n_kv_heads, w.n_q_heads, n, bits=bits,
+                                                quantizer=quantizer), device=device)
+                cache.append(k, v, Td)
+                out = cache.decode(wk.query_transform(q, TinvTd)).double()
+                e = (out - ref).norm(dim=-1) / ref.norm(dim=-1)
+                row[f"{bits}bit"] = float(torch.exp(torch.log(e).mean()))
+            table[f"{name}_{qname}"] = row
+    return {"table": table, "workload": f"{w.name} heads, batch {B}, {n} tokens, bf16, x20 outlier keys",
+            "definition": "geometric mean over (sequence, query head) of ||o_quant - o|| / ||o||",
+            "pages": "2-bit module-output error on Qwen3-8B: 0.208 (data-adaptive), 0.309 (OSCAR), "
+                     "0.325 (Hadamard); context only (needs the model and its data)"}
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
@@ -676,6 +718,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_extra:
         torch.cuda.empty_cache()
         line["workloads"] = run_extra(device, torch)
+        line["module_output_error"] = run_output_error(device, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, bits)
     if dist is not None:

@@ -152,6 +152,36 @@ def key_transform(w: Workload, layer: int, head: int) -> tuple[np.ndarray, np.nd
     return T.astype(np.float32), TinvT.astype(np.float32)
 
 
+_HADAMARD_SIGNS = 8   # tensor id of the seed scheme (random signs of the rotation)
+
+
+def _sylvester(d: int) -> np.ndarray:
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def hadamard_transform(w: Workload, layer: int, head: int) -> tuple[np.ndarray, np.ndarray]:
+    """(T, T^{-T}) of a randomised Hadamard rotation for one KV head: the
+    Sylvester Hadamard matrix scaled by 1/sqrt(128) times a diagonal of
+    seeded random signs (orthogonal, so T^{-T} = T).  The data-independent
+    rotation the pages compare against."""
+    signs = _rng(w.wid, layer, _HADAMARD_SIGNS, head).choice([-1.0, 1.0], HEAD_DIM)
+    T = (_sylvester(HEAD_DIM) / np.sqrt(HEAD_DIM)) * signs[None, :]
+    return T.astype(np.float32), T.astype(np.float32)
+
+
+def hadamard_transforms(w: Workload, layer: int) -> tuple[np.ndarray, np.ndarray]:
+    pairs = [hadamard_transform(w, layer, h) for h in range(w.n_kv_heads)]
+    return np.stack([p[0] for p in pairs]), np.stack([p[1] for p in pairs])
+
+
+def identity_transforms(w: Workload) -> tuple[np.ndarray, np.ndarray]:
+    eye = np.broadcast_to(np.eye(HEAD_DIM, dtype=np.float32), (w.n_kv_heads, HEAD_DIM, HEAD_DIM))
+    return np.ascontiguousarray(eye), np.ascontiguousarray(eye)
+
+
 def key_transforms(w: Workload, layer: int) -> tuple[np.ndarray, np.ndarray]:
     """(T [Hkv,128,128], T^{-T} [Hkv,128,128]) float32."""
     pairs = [key_transform(w, layer, h) for h in range(w.n_kv_heads)]

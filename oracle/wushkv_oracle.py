@@ -637,3 +637,38 @@ class OracleCache:
             K, V = self.unit_kv(u)
             out[b, h * G:(h + 1) * G] = attention_f64(q_prime[b, h * G:(h + 1) * G], K, V, scale)
         return out
+
+
+# ---------------------------------------------------------------------------
+# Module-output error (summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
+# 关键实验, first bullet: the relative error of the attention module's output
+# with the quantised cache, summarised by a geometric mean; the pages report it
+# for 2-bit caches on real model data).  READING: per (sequence, query head),
+# e = ||o_q - o|| / ||o|| where o is exact float64 attention over the keys and
+# values as given and o_q the decode output over the quantised cache built
+# with transform T; the summary is exp(mean(log e)).
+# ---------------------------------------------------------------------------
+
+def output_errors(k: np.ndarray, v: np.ndarray, q: np.ndarray, T: np.ndarray, TinvT: np.ndarray,
+                  cfg: CacheConfig) -> np.ndarray:
+    """Relative output error per (sequence, query head) of one decode query
+    per head after appending all of k, v ([B, n, Hkv, 128]) through T;
+    q [B, Hq, 128].  Returns [B, Hq]."""
+    B, n, Hkv, d = k.shape
+    oc = OracleCache(cfg)
+    oc.append(k, v, np.asarray(T, np.float64))
+    qp = query_transform_gqa(q, np.asarray(TinvT, np.float64))
+    got = oc.decode(qp)
+    G = cfg.group
+    scale = 1.0 / math.sqrt(HEAD_DIM)
+    err = np.empty((B, q.shape[1]))
+    for b in range(B):
+        for h in range(Hkv):
+            ref = attention_f64(q[b, h * G:(h + 1) * G], k[b, :, h], v[b, :, h], scale)
+            diff = got[b, h * G:(h + 1) * G] - ref
+            err[b, h * G:(h + 1) * G] = np.linalg.norm(diff, axis=-1) / np.linalg.norm(ref, axis=-1)
+    return err
+
+
+def geometric_mean(x: np.ndarray) -> float:
+    return float(np.exp(np.mean(np.log(np.asarray(x, np.float64)))))
