@@ -1,6 +1,7 @@
 // Host side of the libwushkv C ABI: configuration checks, cache layout, the
 // window/flush bookkeeping of each append, decode split policy, export and
 // status.  See include/wushkv.h for the contract of every entry point.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdlib>
@@ -15,9 +16,14 @@ struct wushkv_cache {
   wushkv_layout lay;
   uint8_t* base;
   size_t bytes;
-  int64_t n;        // tokens per sequence
+  std::vector<int64_t> seq_n;   // tokens of each sequence
+  bool uniform;                 // every sequence holds n tokens
+  int64_t n;
   double alpha;     // QuEST clip ratio in use
   wushkv::WindowMaps wmaps;   // tensor maps over the fp16 windows (decode)
+  const int32_t* page_table;  // paged caches: the caller's page table (device), row stride pt_stride
+  int32_t pt_stride;
+  mutable wushkv::RaggedTable rt;   // the ragged decode's kernel parameter, rebuilt per call
 };
 
 namespace {
@@ -111,6 +117,7 @@ wushkv_status check_config(const wushkv_config* c) {
     if (c->clip_lo_rank > 8 || c->clip_hi_rank < 121) return WUSHKV_EUNSUPPORTED;
   }
   if ((int64_t)c->batch * c->n_kv_heads > 65535) return WUSHKV_EUNSUPPORTED;
+  if (c->num_pages < 0) return WUSHKV_EINVAL;
   return WUSHKV_OK;
 }
 
@@ -119,6 +126,14 @@ int max_splits_for(const wushkv_config& c, int packed_capacity) {
   const int units = c.batch * c.n_kv_heads;
   const int ms = MAX_GRID / units + 2;
   return ms < 3 ? 3 : (ms > MAX_PARTS_PER_UNIT ? MAX_PARTS_PER_UNIT : ms);
+}
+
+// Bytes of the packed region: per unit its block records, or the page
+// pool (num_pages + 1 pages: the last one is the spare page that
+// out-of-range page ids are sent to).
+size_t packed_region_bytes(const wushkv_config& c, const wushkv_layout& L) {
+  if (c.num_pages > 0) return (size_t)(c.num_pages + 1) * L.page_bytes;
+  return (size_t)c.batch * c.n_kv_heads * L.unit_stride;
 }
 
 void make_layout(const wushkv_config& c, wushkv_layout* L) {
@@ -137,8 +152,12 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
   L->v_meta_off = in_block; in_block += 64 * L->meta_bytes;
   L->block_stride = in_block;                                   // a multiple of 128
   L->unit_stride = (size_t)(L->packed_capacity / 64) * L->block_stride;
+  if (c.num_pages > 0) {   // pages of n_kv_heads block records, one spare page at the end
+    L->num_pages = c.num_pages;
+    L->page_bytes = (size_t)c.n_kv_heads * L->block_stride;
+  }
   // every region is followed by a guard band (see guard_spans)
-  size_t off = align_up(U * L->unit_stride + WUSHKV_GUARD_BYTES, 256);   // packed region at offset 0
+  size_t off = align_up(packed_region_bytes(c, *L) + WUSHKV_GUARD_BYTES, 256);   // packed region at offset 0
   L->sink_unit_stride = (size_t)c.sink * 128 * 2;
   L->sink_k_off = off; off = align_up(off + U * L->sink_unit_stride + WUSHKV_GUARD_BYTES, 256);
   L->sink_v_off = off; off = align_up(off + U * L->sink_unit_stride + WUSHKV_GUARD_BYTES, 256);
@@ -159,7 +178,7 @@ void make_layout(const wushkv_config& c, wushkv_layout* L) {
 // sink V, ring K, ring V and the workspace.
 void guard_spans(const wushkv_config& c, const wushkv_layout& L, size_t out[6]) {
   const size_t U = (size_t)c.batch * c.n_kv_heads;
-  out[0] = U * L.unit_stride;
+  out[0] = packed_region_bytes(c, L);
   out[1] = L.sink_k_off + U * L.sink_unit_stride;
   out[2] = L.sink_v_off + U * L.sink_unit_stride;
   out[3] = L.ring_k_off + U * L.ring_unit_stride;
@@ -206,6 +225,32 @@ DevCache dev_view(const wushkv_cache* h) {
   d.alpha = h->alpha;
   d.r_lo = c.clip_lo_rank;
   d.r_hi = c.clip_hi_rank;
+  d.page_table = c.num_pages > 0 ? h->page_table : nullptr;
+  d.pt_stride = h->pt_stride;
+  d.num_pages = c.num_pages;
+  return d;
+}
+
+// The batch-1 view of sequence b used by its own append launches: every
+// per-unit region starts at the sequence's first unit.
+DevCache seq_view(const wushkv_cache* h, int b) {
+  DevCache d = dev_view(h);
+  const size_t u0 = (size_t)b * d.n_kv_heads;
+  if (d.page_table == nullptr) {
+    for (int p = 0; p < d.n_planes; ++p) {
+      d.k_plane[p] += u0 * d.unit_stride;
+      d.v_plane[p] += u0 * d.unit_stride;
+    }
+    d.k_meta += u0 * d.unit_stride;
+    d.v_meta += u0 * d.unit_stride;
+  } else {
+    d.page_table += (size_t)b * d.pt_stride;
+  }
+  d.sink_k += u0 * d.sink * D;
+  d.sink_v += u0 * d.sink * D;
+  d.ring_k += u0 * d.ring_slots * D;
+  d.ring_v += u0 * d.ring_slots * D;
+  d.units = d.n_kv_heads;
   return d;
 }
 
@@ -239,26 +284,58 @@ int64_t parts_per_unit_bound(int64_t items, int64_t grid, int64_t ni) {
 // Fill the decode arguments of the cache's current state: window/packed
 // counts and the split plan.  EINVAL if the cache is empty, EUNSUPPORTED if
 // the item indices would not fit the kernel's 32-bit arithmetic.
-wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, float scale, DecodeArgs* a) {
+// Fill the decode arguments of the cache's current state: window/packed
+// counts and the split plan.  For sequences of unequal lengths *rt is set to
+// the cache's table of per-sequence counts and item offsets (else null).
+// EINVAL if every sequence is empty, EUNSUPPORTED if the item indices would
+// not fit the kernel's 32-bit arithmetic or a ragged batch is too large.
+wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, float scale, DecodeArgs* a,
+                          const RaggedTable** rt) {
   const wushkv_config& c = h->cfg;
   std::memset(a, 0, sizeof(*a));
+  *rt = nullptr;
   a->c = dev_view(h);
+  if (c.num_pages > 0 && h->page_table == nullptr) return WUSHKV_EINVAL;
   a->q = q;
   a->out = out;
   const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
   a->scale_log2 = sc * 1.4426950408889634f;
-  const int64_t n = h->n;
-  if (n == 0) return WUSHKV_EINVAL;
-  a->n_sink = (int)(n < c.sink ? n : c.sink);
-  a->n_packed = (int)packed_count(n, c);
-  a->n_recent = (int)(n - a->n_sink - a->n_packed);
-  a->ring_first = (int)(a->n_packed % (c.recent + c.chunk));
-  a->win_chunks = (a->n_sink + a->n_recent + WIN_CHUNK - 1) / WIN_CHUNK;
-  a->pack_blocks = (a->n_packed + PACK_BLOCK - 1) / PACK_BLOCK;
+  const int W = c.recent + c.chunk;
   const int64_t units = a->c.units;
-  const int64_t ni = (int64_t)a->win_chunks + a->pack_blocks;
-  const int64_t items = units * ni;
-  if (items >= (int64_t(1) << 31) || ni * a->win_chunks >= (int64_t(1) << 32)) return WUSHKV_EUNSUPPORTED;
+  int64_t items = 0, ni_max = 0, wc_max = 0;
+  if (h->uniform) {
+    const int64_t n = h->n;
+    if (n == 0) return WUSHKV_EINVAL;
+    const SeqGeom g = seq_geom(n, c.sink, c.recent, c.chunk, W);
+    a->n_sink = g.n_sink;
+    a->n_packed = g.n_packed;
+    a->n_recent = g.n_recent;
+    a->ring_first = g.ring_first;
+    a->win_chunks = g.win_chunks;
+    a->pack_blocks = g.pack_blocks;
+    ni_max = (int64_t)g.win_chunks + g.pack_blocks;
+    wc_max = g.win_chunks;
+    items = units * ni_max;
+    a->items_per_unit = (int)ni_max;
+  } else {
+    if (c.batch > MAX_RAGGED_SEQS) return WUSHKV_EUNSUPPORTED;
+    RaggedTable& t = h->rt;
+    t.nseq = c.batch;
+    for (int b = 0; b < c.batch; ++b) {
+      const SeqGeom g = seq_geom(h->seq_n[b], c.sink, c.recent, c.chunk, W);
+      const int64_t ni = (int64_t)g.win_chunks + g.pack_blocks;
+      if (items >= (int64_t(1) << 31)) return WUSHKV_EUNSUPPORTED;
+      t.item_start[b] = (uint32_t)items;
+      t.n[b] = (int32_t)h->seq_n[b];
+      items += (int64_t)c.n_kv_heads * ni;
+      if (ni > ni_max) ni_max = ni;
+      if (g.win_chunks > wc_max) wc_max = g.win_chunks;
+    }
+    t.item_start[c.batch] = (uint32_t)(items < (int64_t(1) << 32) ? items : 0);
+    if (items == 0) return WUSHKV_EINVAL;
+    *rt = &t;
+  }
+  if (items >= (int64_t(1) << 31) || ni_max * wc_max >= (int64_t(1) << 32)) return WUSHKV_EUNSUPPORTED;
   static int occ[5][9][2] = {};
   int& o = occ[c.bits][a->c.group][c.quantizer];
   if (!o) {
@@ -269,9 +346,8 @@ wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, flo
   if (grid > items / MIN_CTA_ITEMS) grid = items / MIN_CTA_ITEMS;
   if (grid > (int64_t)(a->c.max_splits - 1) * units) grid = (int64_t)(a->c.max_splits - 1) * units;
   if (grid < 1) grid = 1;
-  while (grid > 1 && parts_per_unit_bound(items, grid, ni) > a->c.max_splits) --grid;
+  while (grid > 1 && parts_per_unit_bound(items, grid, ni_max) > a->c.max_splits) --grid;
   a->grid = (int)grid;
-  a->items_per_unit = (int)ni;
   a->cta_q = (uint32_t)(items / grid);
   a->cta_r = (uint32_t)(items % grid);
   a->partials = a->c.partials;
@@ -326,6 +402,10 @@ wushkv_status wushkv_cache_create(const wushkv_config* cfg, void* dev_mem, size_
   h->base = static_cast<uint8_t*>(dev_mem);
   h->bytes = bytes;
   h->n = 0;
+  h->seq_n.assign((size_t)cfg->batch, 0);
+  h->uniform = true;
+  h->page_table = nullptr;
+  h->pt_stride = 0;
   h->alpha = cfg->quest_alpha > 0 ? cfg->quest_alpha : wushkv_default_quest_alpha(cfg->bits);
   make_window_maps(dev_view(h), &h->wmaps);
   cudaError_t e = cudaMemsetAsync(dev_mem, 0, L.total_bytes, static_cast<cudaStream_t>(stream));
@@ -352,8 +432,13 @@ wushkv_status wushkv_cache_layout(const wushkv_cache* cache, wushkv_layout* out)
 
 wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t* n_tokens, int64_t* n_sink,
                                   int64_t* n_packed, int64_t* n_recent) {
-  if (!cache) return WUSHKV_EINVAL;
-  const int64_t n = cache->n;
+  return wushkv_sequence_tokens(cache, 0, n_tokens, n_sink, n_packed, n_recent);
+}
+
+wushkv_status wushkv_sequence_tokens(const wushkv_cache* cache, int32_t seq, int64_t* n_tokens, int64_t* n_sink,
+                                     int64_t* n_packed, int64_t* n_recent) {
+  if (!cache || seq < 0 || seq >= cache->cfg.batch) return WUSHKV_EINVAL;
+  const int64_t n = cache->seq_n[seq];
   const int64_t ns = n < cache->cfg.sink ? n : cache->cfg.sink;
   const int64_t P = packed_count(n, cache->cfg);
   if (n_tokens) *n_tokens = n;
@@ -390,23 +475,33 @@ void set_quad_range(AppendArgs& a, int64_t qa, int64_t qb) {
   a.quads_per_cta = (int)per;
 }
 
-wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev, int32_t in_dtype,
-                          const float* T_k_dev, int32_t n_tok, int32_t bits, int32_t quantizer,
-                          AppendPlan* p) {
-  if (!cache || !k_rope_dev || !v_dev || !valid_dtype(in_dtype) || n_tok < 0) return WUSHKV_EINVAL;
+wushkv_status check_append_args(const wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                int32_t in_dtype, const float* T_k_dev, int32_t bits, int32_t quantizer) {
+  if (!cache || !k_rope_dev || !v_dev || !valid_dtype(in_dtype)) return WUSHKV_EINVAL;
   if (reinterpret_cast<uintptr_t>(T_k_dev) & 15) return WUSHKV_EINVAL;  // read as float4
   const wushkv_config& c = cache->cfg;
   if (bits != c.bits || quantizer != c.quantizer) return WUSHKV_EINVAL;
-  if (cache->n + n_tok > c.max_ctx) return WUSHKV_ECAPACITY;
+  if (c.num_pages > 0 && cache->page_table == nullptr) return WUSHKV_EINVAL;
+  return WUSHKV_OK;
+}
+
+size_t dtype_bytes(int32_t dtype) { return dtype == WUSHKV_F32 ? 4 : 2; }
+
+// Plan the append of n_tok tokens to every sequence of `view` (the whole
+// cache, or one sequence's batch-1 view), all holding n0 tokens.
+void plan_append_view(const wushkv_cache* cache, const DevCache& view, int batch, int64_t n0, int32_t n_tok,
+                      const void* k_rope_dev, const void* v_dev, int32_t in_dtype, const float* T_k_dev,
+                      AppendPlan* p) {
+  const wushkv_config& c = cache->cfg;
   std::memset(p, 0, sizeof(*p));
-  const int64_t n0 = cache->n, n1 = n0 + n_tok;
+  const int64_t n1 = n0 + n_tok;
   p->n1 = n1;
-  if (n_tok == 0) return WUSHKV_OK;
+  if (n_tok == 0) return;
   const int64_t S = c.sink, W = c.recent + c.chunk;
   const int64_t P0 = packed_count(n0, c), P1 = packed_count(n1, c);
 
   AppendArgs& a = p->a;
-  a.c = dev_view(cache);
+  a.c = view;
   a.k = k_rope_dev;
   a.v = v_dev;
   a.dtype = in_dtype;
@@ -428,7 +523,7 @@ wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const voi
   const int64_t ta = (n0 + 3) / 4 * 4;
   const uintptr_t kv_addr = reinterpret_cast<uintptr_t>(k_rope_dev) | reinterpret_cast<uintptr_t>(v_dev);
   p->tc = T_k_dev != nullptr && in_dtype == WUSHKV_BF16 && n1 - ta >= TC_MIN_TOKENS &&
-          (kv_addr & 15) == 0 && (int64_t)c.batch * n_tok < 2147483647LL &&
+          (kv_addr & 15) == 0 && (int64_t)batch * n_tok < 2147483647LL &&
           (c.quantizer == WUSHKV_QUEST_INT || (c.clip_lo_rank <= 2 && c.clip_hi_rank >= 127));
   const int64_t tc_qa = p->tc ? ta / 4 : 0;
   // the FMA kernel takes every quad before the tensor-core range
@@ -458,7 +553,7 @@ wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const voi
     pf.tb = (int)n1;
     pf.packed1 = (int)P1;
     pf.tiles_per_unit = (int)((n1 - ta + 127) / 128);
-    const int64_t head_tiles = (int64_t)c.batch * pf.tiles_per_unit;
+    const int64_t head_tiles = (int64_t)batch * pf.tiles_per_unit;
     // one CTA per SM shared among the heads, each CTA at least
     // TC_MIN_CTA_TILES tiles (the T split into smem is paid once per CTA)
     int64_t per_head = device_sms() / c.n_kv_heads;
@@ -467,6 +562,19 @@ wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const voi
     if (per_head < 1) per_head = 1;
     pf.ctas_per_head = (int)per_head;
   }
+}
+
+// The whole-cache plan of a one-call append when every sequence holds the
+// same number of tokens; ECAPACITY if it would exceed max_ctx.
+wushkv_status plan_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev, int32_t in_dtype,
+                          const float* T_k_dev, int32_t n_tok, int32_t bits, int32_t quantizer,
+                          AppendPlan* p) {
+  wushkv_status st = check_append_args(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, bits, quantizer);
+  if (st != WUSHKV_OK) return st;
+  if (n_tok < 0) return WUSHKV_EINVAL;
+  if (cache->n + n_tok > cache->cfg.max_ctx) return WUSHKV_ECAPACITY;
+  plan_append_view(cache, dev_view(cache), cache->cfg.batch, cache->n, n_tok, k_rope_dev, v_dev, in_dtype,
+                   T_k_dev, p);
   return WUSHKV_OK;
 }
 
@@ -478,6 +586,36 @@ cudaError_t run_append(AppendPlan& p, const void* k_rope_dev, const void* v_dev,
   }
   if (p.tc) return launch_prefill_tc(p.pf, k_rope_dev, v_dev, device_sms(), s);
   return cudaSuccess;
+}
+
+void set_uniform(wushkv_cache* cache) {
+  const auto& v = cache->seq_n;
+  cache->uniform = true;
+  for (size_t b = 1; b < v.size(); ++b) cache->uniform &= v[b] == v[0];
+  cache->n = cache->uniform ? v[0] : -1;
+}
+
+// Append n_new[b] tokens to sequence b (token-major input, the sequences'
+// tokens one after another), each sequence through its own batch-1 view.
+// The caller has checked the arguments and the capacity.
+wushkv_status append_per_sequence(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                  int32_t in_dtype, const float* T_k_dev, const int32_t* n_new,
+                                  cudaStream_t s) {
+  const wushkv_config& c = cache->cfg;
+  const size_t row = (size_t)c.n_kv_heads * D * dtype_bytes(in_dtype);
+  size_t off = 0;
+  for (int b = 0; b < c.batch; ++b) {
+    if (n_new[b] == 0) continue;
+    AppendPlan p;
+    const uint8_t* kb = static_cast<const uint8_t*>(k_rope_dev) + off * row;
+    const uint8_t* vb = static_cast<const uint8_t*>(v_dev) + off * row;
+    plan_append_view(cache, seq_view(cache, b), 1, cache->seq_n[b], n_new[b], kb, vb, in_dtype, T_k_dev, &p);
+    if (run_append(p, kb, vb, s) != cudaSuccess) return WUSHKV_ECUDA;
+    cache->seq_n[b] += n_new[b];
+    off += (size_t)n_new[b];
+  }
+  set_uniform(cache);
+  return WUSHKV_OK;
 }
 
 wushkv_status check_query_args(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
@@ -507,11 +645,59 @@ extern "C" {
 wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
                             int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
                             int32_t quantizer, void* stream) {
+  if (cache && !cache->uniform) {   // sequences of unequal lengths: one plan per sequence
+    wushkv_status st = check_append_args(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, bits, quantizer);
+    if (st != WUSHKV_OK) return st;
+    if (n_tok < 0) return WUSHKV_EINVAL;
+    for (int64_t n : cache->seq_n)
+      if (n + n_tok > cache->cfg.max_ctx) return WUSHKV_ECAPACITY;
+    if (n_tok == 0) return WUSHKV_OK;
+    std::vector<int32_t> counts((size_t)cache->cfg.batch, n_tok);
+    return append_per_sequence(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, counts.data(),
+                               static_cast<cudaStream_t>(stream));
+  }
   AppendPlan p;
   const wushkv_status st = plan_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, n_tok, bits, quantizer, &p);
   if (st != WUSHKV_OK || n_tok == 0) return st;
   if (run_append(p, k_rope_dev, v_dev, static_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSHKV_ECUDA;
   cache->n = p.n1;
+  for (auto& n : cache->seq_n) n = p.n1;
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_append_varlen(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                   int32_t in_dtype, const float* T_k_dev, const int32_t* n_new_host,
+                                   int32_t bits, int32_t quantizer, void* stream) {
+  wushkv_status st = check_append_args(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, bits, quantizer);
+  if (st != WUSHKV_OK) return st;
+  if (!n_new_host) return WUSHKV_EINVAL;
+  const wushkv_config& c = cache->cfg;
+  bool equal = true;
+  for (int b = 0; b < c.batch; ++b) {
+    if (n_new_host[b] < 0) return WUSHKV_EINVAL;
+    if (cache->seq_n[b] + n_new_host[b] > c.max_ctx) return WUSHKV_ECAPACITY;
+    equal &= n_new_host[b] == n_new_host[0];
+  }
+  // equal counts on equal lengths: the packed input is [batch][n][Hkv][128],
+  // one plan for the whole cache
+  if (equal && cache->uniform)
+    return wushkv_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, n_new_host[0], bits, quantizer, stream);
+  return append_per_sequence(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, n_new_host,
+                             static_cast<cudaStream_t>(stream));
+}
+
+wushkv_status wushkv_reset_sequence(wushkv_cache* cache, int32_t seq) {
+  if (!cache || seq < 0 || seq >= cache->cfg.batch) return WUSHKV_EINVAL;
+  cache->seq_n[seq] = 0;
+  set_uniform(cache);
+  return WUSHKV_OK;
+}
+
+wushkv_status wushkv_set_page_table(wushkv_cache* cache, const int32_t* page_table_dev, int32_t max_pages_per_seq) {
+  if (!cache || cache->cfg.num_pages <= 0 || !page_table_dev) return WUSHKV_EINVAL;
+  if (max_pages_per_seq < cache->lay.packed_capacity / 64) return WUSHKV_EINVAL;
+  cache->page_table = page_table_dev;
+  cache->pt_stride = max_pages_per_seq;
   return WUSHKV_OK;
 }
 
@@ -526,10 +712,22 @@ wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, co
   if (st != WUSHKV_OK) return st;
   st = check_decode_args(q_prime_dev, cache, out_dev, scale);
   if (st != WUSHKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const RaggedTable* rt = nullptr;
+  DecodeArgs a;
+  if (!cache->uniform) {   // sequences of unequal lengths: per-sequence appends, then the query transform
+    st = wushkv_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, 1, c.bits, c.quantizer, stream);
+    if (st != WUSHKV_OK) return st;
+    if (launch_query_transform(q_dev, q_dtype, T_k_invT_dev, q_prime_dev, c.batch, c.n_q_heads, c.n_kv_heads,
+                               s) != cudaSuccess)
+      return WUSHKV_ECUDA;
+    st = plan_decode(cache, q_prime_dev, out_dev, scale, &a, &rt);
+    if (st != WUSHKV_OK) return st;
+    return cuda_status(launch_decode(a, cache->wmaps, rt, s));
+  }
   AppendPlan p;
   st = plan_append(cache, k_rope_dev, v_dev, in_dtype, T_k_dev, 1, c.bits, c.quantizer, &p);
   if (st != WUSHKV_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   const int64_t S = c.sink;
   const bool new_in_window = p.n1 - 1 < S || p.n1 - 1 >= S + p.a.packed1;
@@ -552,10 +750,10 @@ wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, co
   }
   if (e != cudaSuccess) return WUSHKV_ECUDA;
   cache->n = p.n1;
-  DecodeArgs a;
-  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  for (auto& n : cache->seq_n) n = p.n1;
+  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a, &rt);
   if (st != WUSHKV_OK) return st;
-  return cuda_status(launch_decode(a, cache->wmaps, s));
+  return cuda_status(launch_decode(a, cache->wmaps, rt, s));
 }
 
 wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
@@ -572,9 +770,10 @@ wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache,
   wushkv_status st = check_decode_args(q_prime_dev, cache, out_dev, scale);
   if (st != WUSHKV_OK) return st;
   DecodeArgs a;
-  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  const RaggedTable* rt = nullptr;
+  st = plan_decode(cache, q_prime_dev, out_dev, scale, &a, &rt);
   if (st != WUSHKV_OK) return st;
-  return cuda_status(launch_decode(a, cache->wmaps, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode(a, cache->wmaps, rt, static_cast<cudaStream_t>(stream)));
 }
 
 wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head, int32_t kv,
@@ -585,16 +784,34 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
   const wushkv_layout& L = cache->lay;
   if (seq < 0 || seq >= c.batch || head < 0 || head >= c.n_kv_heads || (kv != 0 && kv != 1))
     return WUSHKV_EINVAL;
-  if (tok0 < 0 || ntok < 0 || (int64_t)tok0 + ntok > cache->n) return WUSHKV_EINVAL;
+  const int64_t n = cache->seq_n[seq];
+  if (tok0 < 0 || ntok < 0 || (int64_t)tok0 + ntok > n) return WUSHKV_EINVAL;
   const size_t u = (size_t)seq * c.n_kv_heads + head;
-  const int64_t n = cache->n;
   const int64_t ns = n < c.sink ? n : c.sink;
   const int64_t P = packed_count(n, c);
   const int W = L.ring_slots;
-  // copy the unit's regions to host (its block records hold K and V)
-  std::vector<uint8_t> packed(L.unit_stride);
-  if (cudaMemcpy(packed.data(), cache->base + u * L.unit_stride, L.unit_stride, cudaMemcpyDeviceToHost))
+  // copy the unit's block records (they hold K and V) to host, one after
+  // another; a paged cache's through the sequence's page-table row
+  const int64_t nblk = (P + 63) / 64;
+  std::vector<uint8_t> packed((size_t)(nblk > 0 ? nblk : 1) * L.block_stride);
+  if (c.num_pages > 0 && nblk > 0) {
+    if (!cache->page_table) return WUSHKV_EINVAL;
+    std::vector<int32_t> pages((size_t)nblk);
+    if (cudaMemcpy(pages.data(), cache->page_table + (size_t)seq * cache->pt_stride, nblk * sizeof(int32_t),
+                   cudaMemcpyDeviceToHost))
+      return WUSHKV_ECUDA;
+    for (int64_t i = 0; i < nblk; ++i) {
+      if (pages[i] < 0 || pages[i] >= c.num_pages) return WUSHKV_EINVAL;
+      if (cudaMemcpy(packed.data() + i * L.block_stride,
+                     cache->base + ((size_t)pages[i] * c.n_kv_heads + head) * L.block_stride, L.block_stride,
+                     cudaMemcpyDeviceToHost))
+        return WUSHKV_ECUDA;
+    }
+  } else if (nblk > 0 &&
+             cudaMemcpy(packed.data(), cache->base + u * L.unit_stride, nblk * L.block_stride,
+                        cudaMemcpyDeviceToHost)) {
     return WUSHKV_ECUDA;
+  }
   auto word_at = [&](uint64_t part_off, int64_t blk, size_t byte) {
     uint32_t wd;
     std::memcpy(&wd, packed.data() + (size_t)blk * L.block_stride + part_off + byte, 4);
@@ -707,7 +924,6 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   if (!q_prime_dev || !cache || !out_dev) return WUSHKV_EINVAL;
   if ((reinterpret_cast<uintptr_t>(out_dev) | reinterpret_cast<uintptr_t>(q_prime_dev)) & 15)
     return WUSHKV_EINVAL;  // read and written as float4
-  if (cache->n == 0) return WUSHKV_EINVAL;
   if (!(scale >= 0.f) || std::isinf(scale)) return WUSHKV_EINVAL;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WUSHKV_ECUDA;
@@ -718,12 +934,17 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
     g_noalloc_addr[dev].store(scratch, std::memory_order_release);
   }
   DecodeArgs a;
-  const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a);
+  const RaggedTable* rt = nullptr;
+  const wushkv_status st = plan_decode(cache, q_prime_dev, out_dev, scale, &a, &rt);
   if (st != WUSHKV_OK) return st;
   // Partials are packed densely, as many per unit as CTAs of this call can
   // touch one unit.
-  const int total = (int)parts_per_unit_bound((int64_t)a.items_per_unit * a.c.units, a.grid,
-                                              a.items_per_unit);
+  const int64_t items = (int64_t)a.cta_q * a.grid + a.cta_r;
+  int64_t ni_max = a.items_per_unit;
+  if (rt)
+    for (int b = 0; b < rt->nseq; ++b)
+      ni_max = std::max<int64_t>(ni_max, (rt->item_start[b + 1] - rt->item_start[b]) / cache->cfg.n_kv_heads);
+  const int total = (int)parts_per_unit_bound(items, a.grid, ni_max);
   a.c.max_splits = total;
   const size_t units = (size_t)a.c.units;
   const size_t partial_bytes = units * (size_t)total * a.c.group * PARTIAL_FLOATS * sizeof(float);
@@ -740,5 +961,5 @@ extern "C" wushkv_status wushkv_decode_noalloc(const float* q_prime_dev, const w
   // The array keeps the previous call's contents: arrival counters must
   // start at zero.
   if (cudaMemsetAsync(a.counters, 0, units * sizeof(int), s) != cudaSuccess) return WUSHKV_ECUDA;
-  return cuda_status(launch_decode(a, cache->wmaps, s));
+  return cuda_status(launch_decode(a, cache->wmaps, rt, s));
 }

@@ -69,9 +69,18 @@ struct StageBytes {
   static constexpr int BYTES = (RAW + 1023) / 1024 * 1024;
 };
 
+// Items of one unit segment of a CTA's batch: its first global item, item
+// count and window split (the same for every unit when all sequences hold
+// the same number of tokens).
+struct SegGeom {
+  uint32_t start;
+  int ni, win_chunks, n_sink, n_win, n_packed, ring_first;
+};
+
 template <int BITS, int G>
 struct Smem {
   static constexpr int NW = Warps<BITS>::N;
+  SegGeom geom[UMAX];
   static constexpr int NT = (G + 3) / 4;   // n-tiles of 8 columns (4 heads x 2 terms)
   alignas(1024) unsigned char stage[NW][NSTAGE][StageBytes<BITS>::BYTES];
   int8_t qterm[UMAX][NT * 4][2][D];        // two int8 terms per head (padded heads = 0)
@@ -259,18 +268,17 @@ __device__ __forceinline__ uint32_t cta_of(const DecodeArgs& a, uint32_t y) {
 // compare per item.
 struct ItemCursor {
   int i, w, rem;   // current item, W(i), i nw - W(i) ni
-  __device__ __forceinline__ void start(const DecodeArgs& a, int i0) {
-    const uint32_t ni = a.items_per_unit;
-    const uint32_t x = (uint32_t)i0 * (uint32_t)a.win_chunks;   // < 2^32 (host check)
+  __device__ __forceinline__ void start(int ni_, int win_chunks, int i0) {
+    const uint32_t ni = ni_;
+    const uint32_t x = (uint32_t)i0 * (uint32_t)win_chunks;   // < 2^32 (host check)
     i = i0;
-    w = (int)(x / ni);
+    w = ni ? (int)(x / ni) : 0;
     rem = (int)(x - (uint32_t)w * ni);
   }
   // Classify the current item (window chunk or packed block, and its
   // number), then step to the next.
-  __device__ __forceinline__ bool take(const DecodeArgs& a, int* idx) {
-    const int ni = a.items_per_unit;
-    rem += a.win_chunks;
+  __device__ __forceinline__ bool take(int ni, int win_chunks, int* idx) {
+    rem += win_chunks;
     const bool win = rem >= ni;
     *idx = win ? w : i - w;
     if (win) { rem -= ni; ++w; }
@@ -279,11 +287,10 @@ struct ItemCursor {
   }
 };
 
-__device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const __half* sink,
-                                                    const __half* ring, int u, int w) {
-  const DevCache& c = a.c;
-  if (w < a.n_sink) return sink + ((size_t)u * c.sink + w) * D;
-  int slot = a.ring_first + (w - a.n_sink);   // < 2 ring_slots
+__device__ __forceinline__ const __half* window_row(const DevCache& c, int n_sink, int ring_first,
+                                                    const __half* sink, const __half* ring, int u, int w) {
+  if (w < n_sink) return sink + ((size_t)u * c.sink + w) * D;
+  int slot = ring_first + (w - n_sink);   // < 2 ring_slots
   if (slot >= c.ring_slots) slot -= c.ring_slots;
   return ring + ((size_t)u * c.ring_slots + slot) * D;
 }
@@ -297,21 +304,22 @@ __device__ __forceinline__ const __half* window_row(const DecodeArgs& a, const _
 // whatever the box covers there (zeros outside the array, else stale but
 // finite rows, the buffer being zeroed at creation) or, when gathered, the
 // window's last row; their scores are masked.
-template <int BITS, bool AFFINE>
-__device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps& wm, int u, bool win,
-                                           int idx, unsigned char* st, uint64_t* bar, int lane) {
+template <int BITS, bool AFFINE, class GEO>
+__device__ __forceinline__ void issue_item(const DecodeArgs& a, const GEO& geo, int j, const WindowMaps& wm,
+                                           bool win, int idx, unsigned char* st, uint64_t* bar, int lane) {
   using SL = StageLayout<BITS, AFFINE>;
   const DevCache& c = a.c;
+  const int u = geo.u_first + j;
   if (win) {
-    const int nwin = a.n_sink + a.n_recent;
+    const int nwin = geo.n_win(j), n_sink = geo.n_sink(j);
     const int w0 = idx * WC, w1 = min(w0 + WC, nwin) - 1;
     const CUtensorMap* mk = nullptr;
     const CUtensorMap* mv = nullptr;
     int y = 0;
-    if (w1 < a.n_sink) {
+    if (w1 < n_sink) {
       if (wm.has_sink) { mk = &wm.sink_k; mv = &wm.sink_v; y = u * c.sink + w0; }
-    } else if (w0 >= a.n_sink) {
-      int s0 = a.ring_first + (w0 - a.n_sink);
+    } else if (w0 >= n_sink) {
+      int s0 = geo.ring_first(j) + (w0 - n_sink);
       if (s0 >= c.ring_slots) s0 -= c.ring_slots;
       if (wm.has_ring && s0 + (w1 - w0) < c.ring_slots) {
         mk = &wm.ring_k; mv = &wm.ring_v; y = u * c.ring_slots + s0;
@@ -331,7 +339,8 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const WindowMaps
     for (int e = lane; e < 2 * WC * 16; e += 32) {
       const int kv = e / (WC * 16), j = (e / 16) % WC, q = e % 16;
       const int w = min(w0 + j, nwin - 1);
-      const __half* row = window_row(a, kv ? c.sink_v : c.sink_k, kv ? c.ring_v : c.ring_k, u, w);
+      const __half* row = window_row(c, n_sink, geo.ring_first(j), kv ? c.sink_v : c.sink_k,
+                                     kv ? c.ring_v : c.ring_k, u, w);
       const uint4 val = *reinterpret_cast<const uint4*>(row + 8 * q);
       *reinterpret_cast<uint4*>(st + kv * WIN_V + (q / 8) * 1024 + j * 128 + (((q % 8) ^ j) * 16)) = val;
     }
@@ -387,11 +396,12 @@ template <int BITS, int G, bool AFFINE, bool FULL, bool KEEP>
 __device__ __forceinline__ void packed_block_compute(
     const DecodeArgs& a, Smem<BITS, G>& sh, const unsigned char* st, int blk, int warp, int lane,
     const uint32_t (&qb)[(G + 3) / 4][4][2], const float (&qscale)[(G + 3) / 4],
-    const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], SoftmaxState<(G + 3) / 4>& S) {
+    const float (&qoff)[(G + 3) / 4], const float (&qsum)[(G + 3) / 4], SoftmaxState<(G + 3) / 4>& S,
+    int n_packed) {
   constexpr int NT = (G + 3) / 4;
   using SL = StageLayout<BITS, AFFINE>;
   const int r = lane >> 2, c4 = lane & 3;
-  const int nvalid = a.n_packed - blk * PB;  // used when !FULL
+  const int nvalid = n_packed - blk * PB;  // used when !FULL
 
   // ---- scores ----------------------------------------------------------------
   // Lane 4r + c owns tokens 8r .. 8r + 7 of the block (slot j = 2 mt + th is
@@ -607,10 +617,10 @@ __device__ __forceinline__ float row_factor(int rho) {
 template <int BITS, int G, bool KEEP>
 __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<BITS, G>& sh,
                                                      const unsigned char* st, int wc, int j, int lane,
-                                                     SoftmaxState<(G + 3) / 4>& S) {
+                                                     SoftmaxState<(G + 3) / 4>& S, int n_win) {
   constexpr int NT = (G + 3) / 4;
   const int r = lane >> 2, c4 = lane & 3;
-  const bool valid = wc * WC + r < a.n_sink + a.n_recent;
+  const bool valid = wc * WC + r < n_win;
   // lane supplies row j = lane % 8 of matrix lane / 8 (dims 32kk + 8 (lane / 8)
   // .. +7: 16-byte chunk 4 (kk % 2) + lane / 8 of tile kk / 2, swizzled with j;
   // odd kk flips bit 2 of the chunk, i.e. bit 6 of the 1 KB-aligned address)
@@ -681,33 +691,70 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
   }
 }
 
-// Cursor over items laid end to end across units (global item y is item
-// y mod NI of unit y / NI).
-struct GCursor {
-  int u;
-  ItemCursor ic;
-  __device__ __forceinline__ void start(const DecodeArgs& a, uint32_t y) {
-    u = (int)(y / (uint32_t)a.items_per_unit);
-    ic.start(a, (int)(y - (uint32_t)u * (uint32_t)a.items_per_unit));
+// Item geometry of the batch's unit segments: from the kernel arguments
+// when every sequence holds the same number of tokens, else from the
+// per-batch table in shared memory.
+template <bool RAGGED, int BITS, int G>
+struct Geo {
+  const Smem<BITS, G>& sh;
+  const DecodeArgs& a;
+  int u_first;
+  // (uniform sequences read the kernel arguments at each use)
+  __device__ __forceinline__ int ni(int j) const { return RAGGED ? sh.geom[j].ni : a.items_per_unit; }
+  __device__ __forceinline__ int win_chunks(int j) const { return RAGGED ? sh.geom[j].win_chunks : a.win_chunks; }
+  __device__ __forceinline__ int n_sink(int j) const { return RAGGED ? sh.geom[j].n_sink : a.n_sink; }
+  __device__ __forceinline__ int n_win(int j) const { return RAGGED ? sh.geom[j].n_win : a.n_sink + a.n_recent; }
+  __device__ __forceinline__ int n_packed(int j) const { return RAGGED ? sh.geom[j].n_packed : a.n_packed; }
+  __device__ __forceinline__ int ring_first(int j) const { return RAGGED ? sh.geom[j].ring_first : a.ring_first; }
+  __device__ __forceinline__ uint32_t start(int j) const {
+    return RAGGED ? sh.geom[j].start : (uint32_t)(u_first + j) * (uint32_t)a.items_per_unit;
   }
-  __device__ __forceinline__ bool take(const DecodeArgs& a, int* idx, int* unit) {
-    if (ic.i == a.items_per_unit) { ++u; ic.start(a, 0); }
-    *unit = u;
-    return ic.take(a, idx);
+  __device__ __forceinline__ SegGeom operator()(int j) const {
+    SegGeom g;
+    g.ni = ni(j); g.start = start(j); g.win_chunks = win_chunks(j); g.n_sink = n_sink(j);
+    g.n_win = n_win(j); g.n_packed = n_packed(j); g.ring_first = ring_first(j);
+    return g;
+  }
+  // segment holding global item y (segments without items are stepped over)
+  __device__ __forceinline__ int segment_of(uint32_t y) const {
+    if constexpr (RAGGED) {
+      int j = 0;
+      while (y >= sh.geom[j].start + (uint32_t)sh.geom[j].ni) ++j;
+      return j;
+    } else {
+      return (int)(y / (uint32_t)a.items_per_unit) - u_first;
+    }
+  }
+};
+
+// Cursor over items laid end to end across the batch's unit segments.
+struct GCursor {
+  int j;
+  ItemCursor ic;
+  template <class GEO>
+  __device__ __forceinline__ void start(const GEO& geo, uint32_t y) {
+    j = geo.segment_of(y);
+    ic.start(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
+  }
+  template <class GEO>
+  __device__ __forceinline__ bool take(const GEO& geo, int* idx, int* seg) {
+    while (ic.i == geo.ni(j)) { ++j; ic.start(geo.ni(j), geo.win_chunks(j), 0); }
+    *seg = j;
+    return ic.take(geo.ni(j), geo.win_chunks(j), idx);
   }
 };
 
 // First copies of the warp's items [y0, y1), issued before the query prologue.
-template <int BITS, bool AFFINE, int G>
+template <int BITS, bool AFFINE, int G, class GEO>
 __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const WindowMaps& wm,
-                                                    Smem<BITS, G>& sh, uint32_t y0, uint32_t y1,
+                                                    Smem<BITS, G>& sh, const GEO& geo, uint32_t y0, uint32_t y1,
                                                     int warp, int lane, uint32_t it, GCursor& ic) {
-  ic.start(a, y0);
+  ic.start(geo, y0);
   for (uint32_t j = 0; j < (uint32_t)NSTAGE && y0 + j < y1; ++j) {
     const int stg = (it + j) % NSTAGE;
-    int idx, unit;
-    const bool win = ic.take(a, &idx, &unit);
-    issue_item<BITS, AFFINE>(a, wm, unit, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+    int idx, seg;
+    const bool win = ic.take(geo, &idx, &seg);
+    issue_item<BITS, AFFINE>(a, geo, seg, wm, win, idx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
   }
 }
 
@@ -775,8 +822,8 @@ __device__ __forceinline__ void state_to_slot(const SoftmaxState<(G + 3) / 4>& S
 // When the items move on to the next unit, the finished unit's state goes
 // to that segment's boundary slot.  Returns the segment of the final state
 // in S (-1 if the warp had no items).
-template <int BITS, int G, bool AFFINE>
-__device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, int u_first,
+template <int BITS, int G, bool AFFINE, class GEO>
+__device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>& sh, const GEO& geo,
                         uint32_t y0, uint32_t y1, int warp, int lane, uint32_t& it, GCursor& ic,
                         SoftmaxState<(G + 3) / 4>& S) {
   constexpr int NT = (G + 3) / 4;
@@ -787,13 +834,11 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
   uint32_t qb[NT][4][2];
   float qscale[NT], qsum[NT], qoff[NT];
   if (y1 <= y0) return -1;
-  const uint32_t NI = (uint32_t)a.items_per_unit;
   int cur = -1;
   uint32_t y = y0;
   while (y < y1) {   // one piece per unit the range touches
-    const int unit = (int)(y / NI);
-    const uint32_t yend = min(y1, (uint32_t)(unit + 1) * NI);
-    const int j = unit - u_first;
+    const int j = geo.segment_of(y);
+    const uint32_t yend = min(y1, geo.start(j) + (uint32_t)geo.ni(j));
     if (cur >= 0) {   // leaving segment cur: its state goes to the boundary slot
       if constexpr (KEEP) {
 #pragma unroll
@@ -807,7 +852,7 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
     begin_segment<BITS, G>(sh, j, lane, qb, qscale, qsum, qoff, S);
     cur = j;
     ItemCursor cc;
-    cc.start(a, (int)(y - (uint32_t)unit * NI));
+    cc.start(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
     for (; y < yend; ++y, ++it) {
       const int stg = it % NSTAGE;
       // (fault injection for tests: the warp's first wait is made on a
@@ -828,19 +873,21 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
       }
       const unsigned char* st = sh.stage[warp][stg];
       int idx;
-      if (cc.take(a, &idx)) {
-        window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, j, lane, S);
-      } else if ((idx + 1) * PB <= a.n_packed) {
-        packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+      if (cc.take(geo.ni(j), geo.win_chunks(j), &idx)) {
+        window_chunk_compute<BITS, G, KEEP>(a, sh, st, idx, j, lane, S, geo.n_win(j));
+      } else if ((idx + 1) * PB <= geo.n_packed(j)) {
+        packed_block_compute<BITS, G, AFFINE, true, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S,
+                                                          geo.n_packed(j));
       } else {
-        packed_block_compute<BITS, G, AFFINE, false, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S);
+        packed_block_compute<BITS, G, AFFINE, false, KEEP>(a, sh, st, idx, warp, lane, qb, qscale, qoff, qsum, S,
+                                                           geo.n_packed(j));
       }
       __syncwarp();
       if (y + NSTAGE < y1) {
         fence_proxy_async();
-        int nidx, nunit;
-        const bool nwin = ic.take(a, &nidx, &nunit);
-        issue_item<BITS, AFFINE>(a, wm, nunit, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
+        int nidx, nseg;
+        const bool nwin = ic.take(geo, &nidx, &nseg);
+        issue_item<BITS, AFFINE>(a, geo, nseg, wm, nwin, nidx, sh.stage[warp][stg], &sh.bar[warp][stg], lane);
       }
     }
   }
@@ -860,9 +907,52 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
 // boundary when its range does; the warps' states are merged per segment
 // into the CTA's partial for that unit, and the last CTA to finish a unit
 // merges its partials into the output.
-template <int BITS, int G, bool AFFINE>
+// Kernel parameter of the per-sequence token counts (empty when every
+// sequence holds the same number of tokens).
+template <bool RAGGED> struct RaggedParam {};
+template <> struct RaggedParam<true> { RaggedTable t; };
+
+// Item geometry of unit u, and the unit holding global item y.
+template <bool RAGGED>
+__device__ __forceinline__ SegGeom unit_geom(const DecodeArgs& a, const RaggedParam<RAGGED>& rp, int u) {
+  SegGeom g;
+  if constexpr (RAGGED) {
+    const DevCache& c = a.c;
+    const int b = u / c.n_kv_heads, h = u - b * c.n_kv_heads;
+    const SeqGeom s = seq_geom(rp.t.n[b], c.sink, c.recent, c.chunk, c.ring_slots);
+    g.ni = s.win_chunks + s.pack_blocks;
+    g.start = rp.t.item_start[b] + (uint32_t)h * (uint32_t)g.ni;
+    g.win_chunks = s.win_chunks; g.n_sink = s.n_sink; g.n_win = s.n_sink + s.n_recent;
+    g.n_packed = s.n_packed; g.ring_first = s.ring_first;
+  } else {
+    g.ni = a.items_per_unit;
+    g.start = (uint32_t)u * (uint32_t)a.items_per_unit;
+    g.win_chunks = a.win_chunks; g.n_sink = a.n_sink; g.n_win = a.n_sink + a.n_recent;
+    g.n_packed = a.n_packed; g.ring_first = a.ring_first;
+  }
+  return g;
+}
+template <bool RAGGED>
+__device__ __forceinline__ int unit_of(const DecodeArgs& a, const RaggedParam<RAGGED>& rp, uint32_t y) {
+  if constexpr (RAGGED) {
+    int lo = 0, hi = rp.t.nseq - 1;   // last sequence whose first item is <= y
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (rp.t.item_start[mid] <= y) lo = mid; else hi = mid - 1;
+    }
+    const DevCache& c = a.c;
+    const SeqGeom s = seq_geom(rp.t.n[lo], c.sink, c.recent, c.chunk, c.ring_slots);
+    const uint32_t ni = (uint32_t)(s.win_chunks + s.pack_blocks);
+    return lo * c.n_kv_heads + (int)((y - rp.t.item_start[lo]) / ni);
+  } else {
+    return (int)(y / (uint32_t)a.items_per_unit);
+  }
+}
+
+template <int BITS, int G, bool AFFINE, bool RAGGED>
 __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
-    decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm) {
+    decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm,
+                  const __grid_constant__ RaggedParam<RAGGED> rp) {
   constexpr int NW = Warps<BITS>::N;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // stages on 1 KB boundaries (swizzle atoms): the launch adds 1 KB of slack
@@ -873,9 +963,8 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = c.n_kv_heads * G;
   const uint32_t cta = blockIdx.x;
-  const uint32_t NI = (uint32_t)a.items_per_unit;
   const uint32_t X0 = cta_begin(a, cta), X1 = X0 + a.cta_q + (cta < a.cta_r ? 1u : 0u);
-  const int U0 = (int)(X0 / NI), U1 = (int)((X1 - 1) / NI);
+  const int U0 = unit_of<RAGGED>(a, rp, X0), U1 = unit_of<RAGGED>(a, rp, X1 - 1);
 
   // the window maps' descriptors are kernel parameters: fetch them now
   if (tid == 0) {
@@ -896,8 +985,18 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
 
   for (int u_first = U0; u_first <= U1; u_first += UMAX) {
     const int nseg = min(UMAX, U1 - u_first + 1);
-    const uint32_t x0 = max(X0, (uint32_t)u_first * NI);
-    const uint32_t x1 = min(X1, (uint32_t)(u_first + nseg) * NI);
+    const Geo<RAGGED, BITS, G> geo{sh, a, u_first};
+    if constexpr (RAGGED) {   // the batch's segment geometry (the previous batch ended with a barrier)
+      if (tid < UMAX) {
+        SegGeom g = unit_geom<RAGGED>(a, rp, u_first + min(tid, nseg - 1));
+        if (tid >= nseg) { g.start += (uint32_t)g.ni; g.ni = 0; }   // unused slots: empty, past the end
+        sh.geom[tid] = g;
+      }
+      __syncthreads();
+    }
+    const SegGeom glast = geo(nseg - 1);
+    const uint32_t x0 = max(X0, geo(0).start);
+    const uint32_t x1 = min(X1, glast.start + (uint32_t)glast.ni);
     const uint32_t len = x1 - x0;
     const uint32_t y0 = x0 + (uint32_t)((uint64_t)len * (uint32_t)warp / NW);
     const uint32_t y1 = x0 + (uint32_t)((uint64_t)len * (uint32_t)(warp + 1) / NW);
@@ -919,7 +1018,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     // (the previous batch ended with a barrier: its slot reads are complete
     // before these copies land in the stage area)
     GCursor ic;
-    warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, y0, y1, warp, lane, it, ic);
+    warp_items_prefetch<BITS, AFFINE, G>(a, wm, sh, geo, y0, y1, warp, lane, it, ic);
     if (tid < UMAX - 1) sh.bused[tid] = 0;
     if (tid < UMAX * G) sh.segMi[tid / G][tid % G] = float_order(-INFINITY);
 
@@ -964,7 +1063,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
 
     // ---- this warp's items -----------------------------------------------------------
     SoftmaxState<NT> S;
-    const int jl = warp_run<BITS, G, AFFINE>(a, wm, sh, u_first, y0, y1, warp, lane, it, ic, S);
+    const int jl = warp_run<BITS, G, AFFINE>(a, wm, sh, geo, y0, y1, warp, lane, it, ic, S);
     // The warp's ring has drained: its final state goes into its own stages
     // (an idle warp's slot, maximum and sum are neutral: every slot is read
     // below, with weight 0 where the warp is not a member).
@@ -989,9 +1088,10 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
                             ? merge_weight(sh.bm[jb][gb], order_float(sh.segMi[jb][gb])) : 0.f;
       }
     }
-    if (tid < nseg) {   // arrivals before the last one (0: the unit lies in this CTA alone)
-      const uint32_t ubj = (uint32_t)(u_first + tid) * NI;
-      sh.others[tid] = (int)(cta_of(a, ubj + NI - 1) - cta_of(a, ubj));
+    if (tid < nseg) {   // arrivals before the last one (0: the unit lies in this CTA alone;
+                        // -1: the unit has no tokens)
+      const SegGeom g = geo(tid);
+      sh.others[tid] = g.ni == 0 ? -1 : (int)(cta_of(a, g.start + (uint32_t)g.ni - 1) - cta_of(a, g.start));
     }
     __syncthreads();
 
@@ -1034,7 +1134,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
         }
         if (sh.others[jj] > 0) {
           const int uu = u_first + jj;
-          const uint32_t slot = cta - cta_of(a, (uint32_t)uu * NI);
+          const uint32_t slot = cta - cta_of(a, geo(jj).start);
           if (slot < (uint32_t)c.max_splits) {
             float* part = a.partials + (((size_t)uu * c.max_splits + slot) * G + g) * PART;
             part[d] = O;
@@ -1052,7 +1152,7 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     // arrival, make the other CTAs' partials visible (acquire).
     __syncthreads();
     if (tid < nseg) {
-      int last = 1;
+      int last = sh.others[tid] >= 0;   // a unit without tokens has no output
       if (sh.others[tid] > 0) {
         const int uu = u_first + tid;
         int prevc;
@@ -1118,9 +1218,9 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   }
 }
 
-template <int BITS, int G, bool AFFINE>
-cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
-  auto k = decode_kernel<BITS, G, AFFINE>;
+template <int BITS, int G, bool AFFINE, bool RAGGED>
+cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, const RaggedTable* rt, cudaStream_t s) {
+  auto k = decode_kernel<BITS, G, AFFINE, RAGGED>;
   static_assert(sizeof(Smem<BITS, G>) + 1024 <= 232448, "decode shared memory above the per-CTA limit");
   const int smem = (int)sizeof(Smem<BITS, G>) + 1024;
   static int attr_done[64] = {0};
@@ -1133,23 +1233,30 @@ cudaError_t launch_t(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  return launch_with_overlap(k, dim3((unsigned)a.grid), dim3(Warps<BITS>::N * 32), (size_t)smem, s, a, wm);
+  RaggedParam<RAGGED> rp;
+  if constexpr (RAGGED) rp.t = *rt;
+  return launch_with_overlap(k, dim3((unsigned)a.grid), dim3(Warps<BITS>::N * 32), (size_t)smem, s, a, wm, rp);
+}
+
+template <int BITS, int G, bool AFFINE>
+cudaError_t launch_r(const DecodeArgs& a, const WindowMaps& wm, const RaggedTable* rt, cudaStream_t s) {
+  return rt ? launch_t<BITS, G, AFFINE, true>(a, wm, rt, s) : launch_t<BITS, G, AFFINE, false>(a, wm, rt, s);
 }
 
 template <int BITS, bool AFFINE>
-cudaError_t launch_g(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
+cudaError_t launch_g(const DecodeArgs& a, const WindowMaps& wm, const RaggedTable* rt, cudaStream_t s) {
   switch (a.c.group) {
-    case 1: return launch_t<BITS, 1, AFFINE>(a, wm, s);
-    case 2: return launch_t<BITS, 2, AFFINE>(a, wm, s);
-    case 4: return launch_t<BITS, 4, AFFINE>(a, wm, s);
-    case 8: return launch_t<BITS, 8, AFFINE>(a, wm, s);
+    case 1: return launch_r<BITS, 1, AFFINE>(a, wm, rt, s);
+    case 2: return launch_r<BITS, 2, AFFINE>(a, wm, rt, s);
+    case 4: return launch_r<BITS, 4, AFFINE>(a, wm, rt, s);
+    case 8: return launch_r<BITS, 8, AFFINE>(a, wm, rt, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int BITS, int G, bool AFFINE>
 int occupancy_t() {
-  auto k = decode_kernel<BITS, G, AFFINE>;
+  auto k = decode_kernel<BITS, G, AFFINE, false>;
   const int smem = (int)sizeof(Smem<BITS, G>) + 1024;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
@@ -1160,12 +1267,12 @@ int occupancy_t() {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& wm, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& wm, const RaggedTable* rt, cudaStream_t s) {
   const bool affine = a.c.quantizer == WUSHKV_AFFINE_PCTCLIP;
   switch (a.c.bits) {
-    case 2: return affine ? launch_g<2, true>(a, wm, s) : launch_g<2, false>(a, wm, s);
-    case 3: return affine ? launch_g<3, true>(a, wm, s) : launch_g<3, false>(a, wm, s);
-    case 4: return affine ? launch_g<4, true>(a, wm, s) : launch_g<4, false>(a, wm, s);
+    case 2: return affine ? launch_g<2, true>(a, wm, rt, s) : launch_g<2, false>(a, wm, rt, s);
+    case 3: return affine ? launch_g<3, true>(a, wm, rt, s) : launch_g<3, false>(a, wm, rt, s);
+    case 4: return affine ? launch_g<4, true>(a, wm, rt, s) : launch_g<4, false>(a, wm, rt, s);
     default: return cudaErrorInvalidValue;
   }
 }

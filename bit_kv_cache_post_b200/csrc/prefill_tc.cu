@@ -477,10 +477,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
+      // (packed destinations are looked up only for packed rows)
+      const bool pkd = mode == ROW_PACKED;
       key_row<BITS, AFFINE>(
           taddr, unscale, c.alpha, lo_second, hi_second, mode,
-          k_row_at(c, 0, t.u, (int64_t)pkc), BITS == 3 ? k_row_at(c, 1, t.u, (int64_t)pkc) : nullptr,
-          k_meta_at(c, t.u, (int64_t)pkc), win);
+          pkd ? k_row_at(c, 0, t.u, (int64_t)pkc) : nullptr,
+          (BITS == 3 && pkd) ? k_row_at(c, 1, t.u, (int64_t)pkc) : nullptr,
+          pkd ? k_meta_at(c, t.u, (int64_t)pkc) : nullptr, win);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[g]);

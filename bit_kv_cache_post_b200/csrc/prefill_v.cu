@@ -49,7 +49,9 @@ __global__ void __launch_bounds__(VP_WARPS * 32) value_pack_kernel(const Prefill
   const int pkq = tq - c.sink;
   const bool packed_quad = tq >= c.sink && pkq < a.packed1;   // uniform per warp
   const int pk = pkq + beta;
-  const int u = b * Hkv + h;
+  // (lanes past the last head write nothing; their addresses are those of a
+  // real unit, so no lookup leaves the sequence's page-table row)
+  const int u = b * Hkv + min(h, Hkv - 1);
   const uint4* src =
       reinterpret_cast<const uint4*>(v + (((int64_t)b * a.n_tok + tok) * Hkv + h) * D + 64 * hf);
   if (!packed_quad) {

@@ -42,6 +42,13 @@ struct DevCache {
   int max_splits;
   int* status;                       // sticky device error word
   int units, n_kv_heads, group;
+  // Paged packed region (null page_table: dense, unit u's blocks at
+  // u * unit_stride).  Block blk of sequence b lives in page
+  // page_table[b * pt_stride + blk]; a page holds the n_kv_heads block
+  // records of that block, head h's at h * block_stride.  Page num_pages is
+  // a spare page that out-of-range ids are sent to (and reported).
+  const int32_t* page_table;
+  int pt_stride, num_pages;
   double alpha;                      // QuEST clip ratio
   int r_lo, r_hi;                    // affine ranks (1-indexed)
 };
@@ -57,24 +64,52 @@ __host__ __device__ __forceinline__ int k_row_pos(int64_t pk) {
   return (i & ~7) | ((i & 7) ^ ((i >> 3) & 3));
 }
 
+// Byte offset of block record blk of unit u from the start of the packed
+// region (the page table's entry when the region is paged).
+__device__ __forceinline__ uint64_t block_offset(const DevCache& c, int64_t u, int64_t blk) {
+  if (c.page_table == nullptr) return (uint64_t)u * c.unit_stride + (uint64_t)blk * c.block_stride;
+  const int64_t b = u / c.n_kv_heads, h = u - b * c.n_kv_heads;
+  int page = __ldg(c.page_table + b * c.pt_stride + blk);
+  if (page < 0 || page >= c.num_pages) {   // never touch another sequence's page
+    atomicOr(c.status, WUSHKV_DEV_RANGE);
+    page = c.num_pages;
+  }
+  return ((uint64_t)page * c.n_kv_heads + (uint64_t)h) * c.block_stride;
+}
+
 // Address of the K row (16 w bytes, plane p) of packed token pk of unit u.
-__host__ __device__ __forceinline__ uint8_t* k_row_at(const DevCache& c, int p, int64_t u, int64_t pk) {
-  return c.k_plane[p] + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
-         (uint64_t)k_row_pos(pk) * 16 * c.plane_bits[p];
+__device__ __forceinline__ uint8_t* k_row_at(const DevCache& c, int p, int64_t u, int64_t pk) {
+  return c.k_plane[p] + block_offset(c, u, pk >> 6) + (uint64_t)k_row_pos(pk) * 16 * c.plane_bits[p];
 }
 // Address of V quad `quad` (tokens 4 quad .. 4 quad + 3; 64 w bytes, plane p) of unit u.
-__host__ __device__ __forceinline__ uint8_t* v_quad_at(const DevCache& c, int p, int64_t u, int64_t quad) {
-  return c.v_plane[p] + (uint64_t)u * c.unit_stride + (uint64_t)(quad >> 4) * c.block_stride +
-         (uint64_t)(quad & 15) * 64 * c.plane_bits[p];
+__device__ __forceinline__ uint8_t* v_quad_at(const DevCache& c, int p, int64_t u, int64_t quad) {
+  return c.v_plane[p] + block_offset(c, u, quad >> 4) + (uint64_t)(quad & 15) * 64 * c.plane_bits[p];
 }
 // Addresses of the per-token meta of packed token pk of unit u.
-__host__ __device__ __forceinline__ uint8_t* k_meta_at(const DevCache& c, int64_t u, int64_t pk) {
-  return c.k_meta + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
-         (uint64_t)(pk & 63) * c.meta_bytes;
+__device__ __forceinline__ uint8_t* k_meta_at(const DevCache& c, int64_t u, int64_t pk) {
+  return c.k_meta + block_offset(c, u, pk >> 6) + (uint64_t)(pk & 63) * c.meta_bytes;
 }
-__host__ __device__ __forceinline__ uint8_t* v_meta_at(const DevCache& c, int64_t u, int64_t pk) {
-  return c.v_meta + (uint64_t)u * c.unit_stride + (uint64_t)(pk >> 6) * c.block_stride +
-         (uint64_t)(pk & 63) * c.meta_bytes;
+__device__ __forceinline__ uint8_t* v_meta_at(const DevCache& c, int64_t u, int64_t pk) {
+  return c.v_meta + block_offset(c, u, pk >> 6) + (uint64_t)(pk & 63) * c.meta_bytes;
+}
+
+// Window split of one sequence holding n tokens (the cache's policy: sink
+// S, recent R, flush chunk C, ring of W = R + C slots), with the decode's
+// items: 8-token window chunks and 64-token packed blocks.  Host and device
+// use this one definition.
+struct SeqGeom {
+  int n_sink, n_packed, n_recent, ring_first, win_chunks, pack_blocks;
+};
+__host__ __device__ __forceinline__ SeqGeom seq_geom(int64_t n, int S, int R, int C, int W) {
+  SeqGeom g;
+  g.n_sink = (int)(n < S ? n : S);
+  const int64_t m = n - g.n_sink;
+  g.n_packed = (int)((m >= (int64_t)R + C) ? (int64_t)C * ((m - R) / C) : 0);
+  g.n_recent = (int)(m - g.n_packed);
+  g.ring_first = W > 0 ? g.n_packed % W : 0;
+  g.win_chunks = (g.n_sink + g.n_recent + 7) / 8;
+  g.pack_blocks = (g.n_packed + 63) / 64;
+  return g;
 }
 
 // Status bits a kernel may set in the sticky word (values documented in
@@ -463,7 +498,18 @@ struct DecodeArgs {
   uint32_t inject_polls;   // 0, or fault injection for tests: each warp's first copy wait is made on a
                            // barrier nothing completes and gives up after this many polls
 };
-cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& m, cudaStream_t s);
+// Sequences of unequal lengths: each sequence's token count and the first
+// global item of its units (items laid end to end, unit by unit); a
+// kernel parameter of the decode, so the CTAs find their units without a
+// memory round trip.
+constexpr int MAX_RAGGED_SEQS = 1024;
+struct RaggedTable {
+  uint32_t item_start[MAX_RAGGED_SEQS + 1];   // [nseq] = total items
+  int32_t n[MAX_RAGGED_SEQS];
+  int32_t nseq;
+};
+// rt: null when every sequence holds the same number of tokens.
+cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& m, const RaggedTable* rt, cudaStream_t s);
 int decode_ctas_per_sm(int bits, int group, int quantizer);
 
 }  // namespace wushkv

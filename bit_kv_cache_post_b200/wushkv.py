@@ -21,6 +21,7 @@ EXPORTED = [
     "wushkv_cache_tokens", "wushkv_append", "wushkv_query_transform", "wushkv_decode",
     "wushkv_export", "wushkv_device_status", "wushkv_default_quest_alpha", "wushkv_strerror",
     "wushkv_decode_noalloc", "wushkv_decode_step", "wushkv_inject_decode_timeout",
+    "wushkv_sequence_tokens", "wushkv_reset_sequence", "wushkv_set_page_table", "wushkv_append_varlen",
 ]
 
 # bits of the sticky device status word; guard bands after each cache region
@@ -33,7 +34,8 @@ class Config(ctypes.Structure):
                 ("batch", "n_kv_heads", "n_q_heads", "head_dim", "max_ctx", "bits",
                  "quantizer", "sink", "recent", "chunk")] + \
                [("quest_alpha", ctypes.c_double),
-                ("clip_lo_rank", ctypes.c_int32), ("clip_hi_rank", ctypes.c_int32)]
+                ("clip_lo_rank", ctypes.c_int32), ("clip_hi_rank", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
 
 
 class Layout(ctypes.Structure):
@@ -50,6 +52,7 @@ class Layout(ctypes.Structure):
         ("ring_unit_stride", ctypes.c_uint64), ("ring_slots", ctypes.c_int32),
         ("workspace_off", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
         ("status_off", ctypes.c_uint64), ("total_bytes", ctypes.c_uint64),
+        ("num_pages", ctypes.c_int32), ("page_bytes", ctypes.c_uint64),
     ]
 
 
@@ -86,6 +89,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_export.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.wushkv_device_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
+    lib.wushkv_sequence_tokens.argtypes = [vp, i32] + [ctypes.POINTER(i64)] * 4
+    lib.wushkv_reset_sequence.argtypes = [vp, i32]
+    lib.wushkv_set_page_table.argtypes = [vp, vp, i32]
+    lib.wushkv_append_varlen.argtypes = [vp, vp, vp, i32, vp, ctypes.POINTER(i32), i32, i32, vp]
     lib.wushkv_inject_decode_timeout.argtypes = [ctypes.c_uint32]
     lib.wushkv_inject_decode_timeout.restype = None
     lib.wushkv_default_quest_alpha.argtypes = [i32]
@@ -124,11 +131,12 @@ def _stream_ptr(stream) -> int | None:
 
 
 def make_config(batch, n_kv_heads, n_q_heads, max_ctx, bits=2, quantizer=QUEST_INT, sink=64,
-                recent=256, chunk=8, quest_alpha=0.0, clip_lo_rank=2, clip_hi_rank=127) -> Config:
+                recent=256, chunk=8, quest_alpha=0.0, clip_lo_rank=2, clip_hi_rank=127,
+                num_pages=0) -> Config:
     return Config(batch=batch, n_kv_heads=n_kv_heads, n_q_heads=n_q_heads, head_dim=128,
                   max_ctx=max_ctx, bits=bits, quantizer=quantizer, sink=sink, recent=recent,
                   chunk=chunk, quest_alpha=quest_alpha, clip_lo_rank=clip_lo_rank,
-                  clip_hi_rank=clip_hi_rank)
+                  clip_hi_rank=clip_hi_rank, num_pages=num_pages)
 
 
 def cache_bytes(cfg: Config) -> int:
@@ -190,11 +198,36 @@ class Cache:
         _check(load().wushkv_cache_layout(self._handle, ctypes.byref(out)), "wushkv_cache_layout")
         return out
 
-    def tokens(self) -> tuple[int, int, int, int]:
+    def tokens(self, seq: int | None = None) -> tuple[int, int, int, int]:
+        """(total, sink, packed, recent) of sequence `seq` (default 0)."""
         v = [ctypes.c_int64() for _ in range(4)]
-        _check(load().wushkv_cache_tokens(self._handle, *[ctypes.byref(x) for x in v]),
-               "wushkv_cache_tokens")
+        _check(load().wushkv_sequence_tokens(self._handle, 0 if seq is None else seq,
+                                             *[ctypes.byref(x) for x in v]), "wushkv_sequence_tokens")
         return tuple(int(x.value) for x in v)
+
+    def reset_sequence(self, seq: int):
+        _check(load().wushkv_reset_sequence(self._handle, seq), "wushkv_reset_sequence")
+
+    def set_page_table(self, page_table, max_pages_per_seq: int):
+        """page_table: [batch][max_pages_per_seq] int32 device tensor (kept
+        referenced here so it outlives the cache's use of it)."""
+        import torch
+        assert page_table.is_contiguous() and page_table.dtype == torch.int32
+        self._page_table = page_table
+        _check(load().wushkv_set_page_table(self._handle, page_table.data_ptr(), max_pages_per_seq),
+               "wushkv_set_page_table")
+
+    def append_varlen(self, k, v, n_new, T=None, stream=None):
+        """k, v: [sum(n_new), Hkv, 128] device tensors (sequence 0's tokens,
+        then sequence 1's, ...); n_new: per-sequence counts (host)."""
+        assert k.is_contiguous() and v.is_contiguous() and k.dtype == v.dtype and k.shape == v.shape
+        assert len(n_new) == self.cfg.batch and k.shape[0] == sum(n_new)
+        if T is not None:
+            assert T.is_contiguous() and T.dtype.itemsize == 4
+        counts = (ctypes.c_int32 * len(n_new))(*[int(x) for x in n_new])
+        _check(load().wushkv_append_varlen(self._handle, k.data_ptr(), v.data_ptr(), _dtype_code(k),
+                                           None if T is None else T.data_ptr(), counts, self.cfg.bits,
+                                           self.cfg.quantizer, _stream_ptr(stream)), "wushkv_append_varlen")
 
     def append(self, k, v, T=None, stream=None, bits=None, quantizer=None):
         """k, v: [B, n_tok, Hkv, 128] device tensors (f16/bf16/f32); T:
@@ -265,7 +298,8 @@ class Cache:
         packed region, sink K, sink V, ring K, ring V and the workspace."""
         L = self.layout()
         U = self.cfg.batch * self.cfg.n_kv_heads
-        return [U * L.unit_stride, L.sink_k_off + U * L.sink_unit_stride,
+        packed = (L.num_pages + 1) * L.page_bytes if L.num_pages > 0 else U * L.unit_stride
+        return [packed, L.sink_k_off + U * L.sink_unit_stride,
                 L.sink_v_off + U * L.sink_unit_stride, L.ring_k_off + U * L.ring_unit_stride,
                 L.ring_v_off + U * L.ring_unit_stride, L.workspace_off + L.workspace_bytes]
 

@@ -95,6 +95,7 @@ typedef struct {
   int32_t sink, recent, chunk;
   double quest_alpha;
   int32_t clip_lo_rank, clip_hi_rank;
+  int32_t num_pages;   /* 0: dense packed region; > 0: paged (see wushkv_set_page_table) */
 } wushkv_config;
 
 typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
@@ -153,6 +154,8 @@ typedef struct {
   uint64_t workspace_off, workspace_bytes;
   uint64_t status_off;
   uint64_t total_bytes;
+  int32_t num_pages;                /* paged caches: pages in the pool (else 0) */
+  uint64_t page_bytes;              /* paged caches: n_kv_heads * block_stride */
 } wushkv_layout;
 
 /* Bytes of device memory a cache with this configuration needs (0 if the
@@ -172,10 +175,41 @@ WUSHKV_API wushkv_status wushkv_cache_destroy(wushkv_cache* cache);
 /* Fill *out with the byte layout of this cache. */
 WUSHKV_API wushkv_status wushkv_cache_layout(const wushkv_cache* cache, wushkv_layout* out);
 
-/* Current token counts per sequence: total, sink, packed, recent (host-side
+/* Token counts of sequence 0: total, sink, packed, recent (host-side
  * bookkeeping, no synchronisation).  Any pointer may be NULL. */
 WUSHKV_API wushkv_status wushkv_cache_tokens(const wushkv_cache* cache, int64_t* n_tokens, int64_t* n_sink,
                                   int64_t* n_packed, int64_t* n_recent);
+
+/* Token counts of sequence seq (0 <= seq < batch), as wushkv_cache_tokens.
+ * Sequences may hold different numbers of tokens (wushkv_append_varlen,
+ * wushkv_reset_sequence); the window policy applies to each on its own. */
+WUSHKV_API wushkv_status wushkv_sequence_tokens(const wushkv_cache* cache, int32_t seq, int64_t* n_tokens,
+                                                int64_t* n_sink, int64_t* n_packed, int64_t* n_recent);
+
+/* Empty sequence seq (its count drops to 0; its slots are reused by later
+ * appends), e.g. when a serving loop gives the batch slot to a new request.
+ * Host bookkeeping only: nothing is launched. */
+WUSHKV_API wushkv_status wushkv_reset_sequence(wushkv_cache* cache, int32_t seq);
+
+/* Paged caches (config num_pages > 0).  The packed tokens of a sequence live
+ * in 64-token blocks scattered over a pool of num_pages pages; a page holds
+ * the block records of all n_kv_heads heads of one block (page_bytes =
+ * n_kv_heads * block_stride, page p at byte p * page_bytes of the packed
+ * region; one spare page follows the pool).  The caller owns the page
+ * table, as a serving engine's cache manager does:
+ *   page_table_dev: [batch][max_pages_per_seq] int32 device array; entry
+ *     [b][i] is the page of block i (packed tokens 64i .. 64i + 63) of
+ *     sequence b.  It must map every block an append writes or a decode
+ *     reads (blocks 0 .. ceil(n_packed_after / 64) - 1 of each sequence)
+ *     before that call runs, and distinct sequences must not share a page.
+ *     A page id outside [0, num_pages) is redirected to the spare page and
+ *     reported as WUSHKV_DEV_RANGE.
+ *   max_pages_per_seq >= packed_capacity / 64 (EINVAL otherwise).
+ * The pointer is borrowed until the cache is destroyed or the table is
+ * replaced.  Sink and recent windows stay in the dense per-sequence regions.
+ * EINVAL on a dense cache. */
+WUSHKV_API wushkv_status wushkv_set_page_table(wushkv_cache* cache, const int32_t* page_table_dev,
+                                               int32_t max_pages_per_seq);
 
 /* Append n_tok tokens to every sequence.
  *   Source: summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
@@ -197,6 +231,21 @@ WUSHKV_API wushkv_status wushkv_append(wushkv_cache* cache, const void* k_rope_d
                             int32_t in_dtype, const float* T_k_dev, int32_t n_tok, int32_t bits,
                             int32_t quantizer, void* stream);
 
+/* Append a different number of tokens to each sequence.
+ *   Source: as wushkv_append; the window policy of the summary page
+ *   (sink, recent, chunked flush) applies to each sequence on its own.
+ *   k_rope_dev, v_dev: [sum_b n_new[b]][n_kv_heads][128] in_dtype, the
+ *     tokens of sequence 0, then those of sequence 1, ... (no padding).
+ *   n_new_host: [batch] host array of new-token counts (0 = sequence
+ *     unchanged).
+ *   Other arguments and results as wushkv_append; ECAPACITY (nothing
+ *   written) if any sequence would exceed max_ctx.  With equal counts on
+ *   sequences of equal length this is wushkv_append; otherwise each
+ *   sequence's tokens go through their own launches. */
+WUSHKV_API wushkv_status wushkv_append_varlen(wushkv_cache* cache, const void* k_rope_dev, const void* v_dev,
+                                              int32_t in_dtype, const float* T_k_dev, const int32_t* n_new_host,
+                                              int32_t bits, int32_t quantizer, void* stream);
+
 /* q' = T_k^{-T} q for every query head, with the transform of its KV group.
  *   Source: same page, 方法关键点 and 工作参考价值 (one d x d product per
  *   query; inverse transpose keeps q'.k' = q.k).
@@ -217,8 +266,13 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
  *   out_dev:     [batch][n_q_heads][128] fp32 = softmax(scale q'.k'^T) v
  *                in the transformed value space; 16-byte aligned (EINVAL otherwise).
  *   scale: softmax scale; 0 selects 1/sqrt(128).
+ * Each sequence attends to its own tokens: sequences of different lengths
+ * are decoded in the same launch (up to 1024 sequences when their lengths
+ * differ, else EUNSUPPORTED); the output rows of a sequence without tokens
+ * are left unchanged.
  * Uses the cache's workspace region for split-K partials; calls on the same
- * cache must therefore be stream-ordered.  EINVAL if the cache is empty. */
+ * cache must therefore be stream-ordered.  EINVAL if every sequence is
+ * empty, or the cache is paged and has no page table. */
 WUSHKV_API wushkv_status wushkv_decode(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
                             float scale, void* stream);
 

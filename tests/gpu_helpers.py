@@ -170,7 +170,7 @@ def unit_state_from_export(cache, b: int, h: int):
     wushkv_export and dequantised with the oracle's reconstruction rules:
     fp16 rows for window tokens, (codes, scales) for packed ones."""
     cfg = cache.cfg
-    n = cache.tokens()[0]
+    n = cache.tokens(b)[0]
     out = []
     for kv in (0, 1):
         codes, meta, rows, kinds = cache.export(b, h, kv, 0, n)
@@ -184,3 +184,27 @@ def unit_state_from_export(cache, b: int, h: int):
                 x[pk] = O.affine_dequantize(codes[pk], m[:, 0], m[:, 1])
         out.append(x)
     return out[0], out[1]
+
+
+def compare_unit_by_export(cache, b: int, h: int, oc: O.OracleCache, ou: int):
+    """Unit (b, h) of the GPU cache, read through wushkv_export, equals unit
+    ou of the oracle cache bit for bit: kinds, fp16 window rows, packed
+    codes and scales of K and V."""
+    cfg = cache.cfg
+    n = cache.tokens(b)[0]
+    ns, P, nr = oc.split()
+    assert (n, ns, P, nr) == (oc.n, *oc.split())
+    W = cfg.recent + cfg.chunk
+    nm = 2 if cfg.quantizer == O.AFFINE_PCTCLIP else 1
+    for kv in (0, 1):
+        codes, meta, rows, kinds = cache.export(b, h, kv, 0, n)
+        sink = oc.sink_k if kv == 0 else oc.sink_v
+        ring = oc.ring_k if kv == 0 else oc.ring_v
+        ocodes = oc.codes_k if kv == 0 else oc.codes_v
+        ometa = oc.meta_k if kv == 0 else oc.meta_v
+        assert np.array_equal(kinds, np.array([0] * ns + [1] * P + [2] * nr, np.int8)), (b, h, kv)
+        assert np.array_equal(rows[:ns], sink[ou, :ns].view(np.uint16)), (b, h, kv)
+        slots = [(t - cfg.sink) % W for t in range(ns + P, n)]
+        assert np.array_equal(rows[ns + P:], ring[ou, slots].view(np.uint16)), (b, h, kv)
+        assert np.array_equal(codes[ns:ns + P], ocodes[ou, :P]), (b, h, kv)
+        assert np.array_equal(meta[ns:ns + P, :nm], ometa[ou, :P, :nm].view(np.uint16)), (b, h, kv)
