@@ -303,7 +303,10 @@ wushkv_status plan_decode(const wushkv_cache* h, const float* q, float* out, flo
   const int W = c.recent + c.chunk;
   const int64_t units = a->c.units;
   int64_t items = 0, ni_max = 0, wc_max = 0;
-  if (h->uniform) {
+  // Uniform dense caches take the decode variant that reads the geometry
+  // from its arguments and addresses the packed region directly; ragged or
+  // paged ones the variant with the per-sequence table (and page lookups).
+  if (h->uniform && c.num_pages == 0) {
     const int64_t n = h->n;
     if (n == 0) return WUSHKV_EINVAL;
     const SeqGeom g = seq_geom(n, c.sink, c.recent, c.chunk, W);

@@ -268,11 +268,12 @@ __device__ __forceinline__ uint32_t cta_of(const DecodeArgs& a, uint32_t y) {
 // compare per item.
 struct ItemCursor {
   int i, w, rem;   // current item, W(i), i nw - W(i) ni
+  template <bool MAYBE_EMPTY = true>   // false: ni > 0 is known
   __device__ __forceinline__ void start(int ni_, int win_chunks, int i0) {
     const uint32_t ni = ni_;
     const uint32_t x = (uint32_t)i0 * (uint32_t)win_chunks;   // < 2^32 (host check)
     i = i0;
-    w = ni ? (int)(x / ni) : 0;
+    w = (!MAYBE_EMPTY || ni) ? (int)(x / ni) : 0;
     rem = (int)(x - (uint32_t)w * ni);
   }
   // Classify the current item (window chunk or packed block, and its
@@ -350,8 +351,10 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const GEO& geo, 
   }
   if (lane != 0) return;
   mbar_arrive_expect_tx(bar, (uint32_t)SL::PACKED);
-  bulk_copy_g2s_hint(st, k_row_at(c, 0, u, (int64_t)idx * PB), (uint32_t)SL::PACKED, bar,
-                     l2_evict_first_policy());
+  // (the general variant may read a paged region; the uniform one is dense)
+  const uint64_t off = GEO::kTable ? block_offset(c, u, idx)
+                                   : (uint64_t)u * c.unit_stride + (uint64_t)idx * c.block_stride;
+  bulk_copy_g2s_hint(st, c.k_plane[0] + off, (uint32_t)SL::PACKED, bar, l2_evict_first_policy());
 }
 
 // ---- packed blocks: copy ring + integer tensor cores ------------------------------
@@ -696,6 +699,7 @@ __device__ __forceinline__ void window_chunk_compute(const DecodeArgs& a, Smem<B
 // per-batch table in shared memory.
 template <bool RAGGED, int BITS, int G>
 struct Geo {
+  static constexpr bool kTable = RAGGED;
   const Smem<BITS, G>& sh;
   const DecodeArgs& a;
   int u_first;
@@ -734,11 +738,15 @@ struct GCursor {
   template <class GEO>
   __device__ __forceinline__ void start(const GEO& geo, uint32_t y) {
     j = geo.segment_of(y);
-    ic.start(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
+    ic.start<GEO::kTable>(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
   }
   template <class GEO>
   __device__ __forceinline__ bool take(const GEO& geo, int* idx, int* seg) {
-    while (ic.i == geo.ni(j)) { ++j; ic.start(geo.ni(j), geo.win_chunks(j), 0); }
+    if constexpr (GEO::kTable) {   // a table may hold units without items
+      while (ic.i == geo.ni(j)) { ++j; ic.start<true>(geo.ni(j), geo.win_chunks(j), 0); }
+    } else {
+      if (ic.i == geo.ni(j)) { ++j; ic.start<false>(geo.ni(j), geo.win_chunks(j), 0); }
+    }
     *seg = j;
     return ic.take(geo.ni(j), geo.win_chunks(j), idx);
   }
@@ -852,7 +860,7 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
     begin_segment<BITS, G>(sh, j, lane, qb, qscale, qsum, qoff, S);
     cur = j;
     ItemCursor cc;
-    cc.start(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
+    cc.start<false>(geo.ni(j), geo.win_chunks(j), (int)(y - geo.start(j)));
     for (; y < yend; ++y, ++it) {
       const int stg = it % NSTAGE;
       // (fault injection for tests: the warp's first wait is made on a
@@ -1091,7 +1099,9 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     if (tid < nseg) {   // arrivals before the last one (0: the unit lies in this CTA alone;
                         // -1: the unit has no tokens)
       const SegGeom g = geo(tid);
-      sh.others[tid] = g.ni == 0 ? -1 : (int)(cta_of(a, g.start + (uint32_t)g.ni - 1) - cta_of(a, g.start));
+      const int o = (int)(cta_of(a, g.start + (uint32_t)g.ni - 1) - cta_of(a, g.start));
+      if constexpr (RAGGED) sh.others[tid] = g.ni == 0 ? -1 : o;
+      else sh.others[tid] = o;
     }
     __syncthreads();
 
