@@ -210,6 +210,38 @@ def decode_graph_us(caches, qprime, out, torch, device, launches=4000):
     return us
 
 
+def step_graph_time_us(caches, step, dev_pool, i0, torch, device, reps=30):
+    """Microseconds per decode step (append + query transform + decode, two
+    launches) with one step per cache captured in a CUDA graph, replays
+    bracketed by CUDA events.  The capture call appends one token per cache
+    (indices i0 .. i0 + copies) after an untimed eager step per cache."""
+    stream = torch.cuda.current_stream()
+    n = len(caches)
+    capture = torch.cuda.Stream(device=device)
+    capture.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(capture):
+        for i in range(i0, i0 + n):
+            step(i, *dev_pool[i % STEP_POOL], stream=capture)
+        capture.synchronize()
+        with torch.cuda.graph(graph, stream=capture):
+            for i in range(i0 + n, i0 + 2 * n):
+                step(i, *dev_pool[i % STEP_POOL], stream=capture)
+    stream.wait_stream(capture)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    us = g0.elapsed_time(g1) * 1e3 / (reps * n)
+    del graph
+    return us
+
+
 def run_ours(args, rank, world, device, torch, dist):
     from bit_kv_cache_post_b200 import inputs as I
     from bit_kv_cache_post_b200 import wushkv as wk
@@ -217,7 +249,8 @@ def run_ours(args, rank, world, device, torch, dist):
     bits = args.bits
     stream = torch.cuda.current_stream()
     kd, vd, pool = build_inputs(w, torch, device)
-    total_steps = args.warmup + args.steps + args.e2e_steps
+    # set-up steps (one per cache) + warm-up + timed + e2e + the graph timing's
+    total_steps = args.copies + args.warmup + args.steps + args.e2e_steps + 2 * args.copies
     grow = math.ceil(total_steps / args.copies) + 8
     cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, w.context + grow, bits=bits,
                          sink=w.sink, recent=w.recent, chunk=w.chunk)
@@ -247,20 +280,25 @@ def run_ours(args, rank, world, device, torch, dist):
         rest = append_bytes(w, bits, after[2] > before[2]) + qtransform_bytes(w)
         return dec, rest
 
-    def step(i, k, v, q):
+    def step(i, k, v, q, stream=stream):
         # one call: append 1 token + query transform (one launch) + decode
         c = i % args.copies
         caches[c].decode_step(k, v, Ts[c], q, TinvTs[c], q_prime=qprime, out=out, stream=stream)
 
-    for i in range(args.warmup):
+    # set-up: every cache (layer) takes one decode step before the warm-up,
+    # as in a running server, so that no timed step is the first read of a
+    # layer's transforms since its prefill; then W warm-up steps
+    i0 = args.copies
+    for i in range(i0 + args.warmup):
         step_bytes(i)
         step(i, *dev_pool[i % STEP_POOL])
     torch.cuda.synchronize()
 
     # ---- timed region: K steps, device resident inputs ----------------------
     K = args.steps
+    first = i0 + args.warmup
     dec_total = rest_total = 0
-    for i in range(args.warmup, args.warmup + K):
+    for i in range(first, first + K):
         d, r = step_bytes(i)
         dec_total += d
         rest_total += r
@@ -272,7 +310,7 @@ def run_ours(args, rank, world, device, torch, dist):
     with ClockSampler(torch.cuda.current_device()) as clocks:
         t0.record(stream)
         h0 = time.perf_counter()
-        for i in range(args.warmup, args.warmup + K):
+        for i in range(first, first + K):
             step(i, *dev_pool[i % STEP_POOL])
         host_s = time.perf_counter() - h0
         t1.record(stream)
@@ -290,11 +328,19 @@ def run_ours(args, rank, world, device, torch, dist):
     dec_launch_bytes = [decode_bytes(w, bits, window_state(counts_after[c], w)) for c in range(args.copies)]
     counts = counts_after
 
+    # ---- the whole step with no host in the loop: one decode_step per cache
+    # captured in a CUDA graph (each replay re-appends the captured tokens at
+    # the captured positions); minus the decode alone = the step kernel
+    step_graph_us = step_graph_time_us(caches, step, dev_pool, first + K, torch, device)
+    for i in range(first + K, first + K + 2 * args.copies):
+        step_bytes(i)
+    e_first = first + K + 2 * args.copies
+
     # ---- e2e: host buffers, copies inside the timed region --------------------
     E = args.e2e_steps
     host_out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory()
     e_dec = 0
-    for i in range(args.warmup + K, args.warmup + K + E):
+    for i in range(e_first, e_first + E):
         e_dec += sum(step_bytes(i))
     # each step's k, v and q packed back to back in one pinned host buffer:
     # one host->device copy per step, one device->host copy of the output
@@ -313,7 +359,7 @@ def run_ours(args, rank, world, device, torch, dist):
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for i in range(args.warmup + K, args.warmup + K + E):
+    for i in range(e_first, e_first + E):
         dbuf.copy_(packed[i % STEP_POOL], non_blocking=True)
         step(i, *parts)
         host_out.copy_(out, non_blocking=True)
@@ -324,7 +370,7 @@ def run_ours(args, rank, world, device, torch, dist):
         e_ms = max_over_ranks(e_ms, dist, device)
 
     return dict(w=w, bits=bits, K=K, ms=ms, dec_total=dec_total, rest_total=rest_total, host_s=host_s,
-                dec_ms=dec_ms, dec_launch_bytes=dec_launch_bytes, clocks=clocks.summary(),
+                dec_ms=dec_ms, step_graph_us=step_graph_us, dec_launch_bytes=dec_launch_bytes, clocks=clocks.summary(),
                 launches=launches_per_step * K,
                 status=status, e2e=(E, e_ms, e_dec, h2d, d2h), copies=args.copies,
                 l2_bytes=sum(decode_bytes(w, bits, window_state(c, w)) for c in counts))
@@ -445,6 +491,68 @@ def run_append_steps(caches, w, Td, device, torch, steps=64):
             "timing": "one-token wushkv_append calls back to back, CUDA events around the run"}
 
 
+def ragged_lengths(w, seed=0):
+    """Per-sequence token counts with the workload's mean: pairs context +- d
+    with d drawn uniformly from [0, context / 2] (seeded), so the batch holds
+    the same number of tokens as the uniform one."""
+    g = np.random.default_rng(seed)
+    d = g.integers(0, w.context // 2 + 1, size=w.batch // 2)
+    n = np.concatenate([w.context + d, w.context - d])
+    if w.batch % 2:
+        n = np.append(n, w.context)
+    return [int(x) for x in g.permutation(n)]
+
+
+def run_ragged_decode(device, torch, paged: bool, copies=8, bits=2):
+    """Decode GB/s of the batch-16 Qwen3-8B-shaped layer when its sequences
+    hold different numbers of tokens (ragged_lengths), optionally with the
+    packed region paged through a random page table; same total tokens as
+    the uniform workload, so the GB/s compare directly."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[WORKLOAD]
+    lens = ragged_lengths(w)
+    nmax = max(lens)
+    k, v = I.device_kv(w, 0, nmax, device=device)
+    kf = torch.cat([k[b, :n] for b, n in enumerate(lens)]).contiguous()
+    vf = torch.cat([v[b, :n] for b, n in enumerate(lens)]).contiguous()
+    del k, v
+    T, TinvT = I.key_transforms(w, 0)
+    Td, TinvTd = torch.from_numpy(T).to(device), torch.from_numpy(TinvT).to(device)
+    max_ctx = nmax + 128
+    pages_per_seq = (max_ctx + 127) // 128 * 2
+    cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, max_ctx, bits=bits, sink=w.sink,
+                         recent=w.recent, chunk=w.chunk,
+                         num_pages=w.batch * pages_per_seq if paged else 0)
+    caches = []
+    for c in range(copies):
+        cache = wk.Cache(cfg, device=device)
+        if paged:
+            perm = np.random.default_rng(100 + c).permutation(cfg.num_pages).astype(np.int32)
+            cache.set_page_table(torch.from_numpy(perm.reshape(w.batch, pages_per_seq)).to(device),
+                                 pages_per_seq)
+        cache.append_varlen(kf, vf, lens, Td)
+        caches.append(cache)
+    del kf, vf
+    qprime = wk.query_transform(I.device_queries(w, 0, 0, device=device), TinvTd)
+    out = torch.empty_like(qprime)
+    torch.cuda.synchronize()
+    us = decode_graph_us(caches, qprime, out, torch, device)
+    status = max(c.device_status() for c in caches)
+    per_seq = 0
+    for n in lens:
+        _, ns, P, nr = window_state(n, w)
+        per_seq += w.n_kv_heads * (P * 2 * (16 * bits + meta_bytes(w.quantizer)) + (ns + nr) * 2 * 256)
+    nbytes = per_seq + 2 * w.batch * w.n_q_heads * 128 * 4
+    peak, _ = peaks()
+    del caches
+    torch.cuda.empty_cache()
+    return {"workload": f"{WORKLOAD} with per-sequence lengths {min(lens)}..{max(lens)} "
+                        f"(mean {sum(lens) / len(lens):.0f}){', paged packed region' if paged else ''}",
+            "lengths": lens, "decode_us": us, "bytes_per_launch": nbytes, "gbs": nbytes / us / 1e3,
+            "frac": nbytes / us / 1e3 / peak, "copies": copies, "device_status": status}
+
+
 def run_extra(device, torch):
     """Decode GB/s of the 32B-shaped, 4B-shaped long-context and 36-layer
     (one layer, affine) workloads, config-1 decode at 3 and 4 bits, and the
@@ -463,6 +571,8 @@ def run_extra(device, torch):
         out[key] = res
         del caches
         torch.cuda.empty_cache()
+    out["ragged_" + WORKLOAD] = run_ragged_decode(device, torch, paged=False)
+    out["ragged_paged_" + WORKLOAD] = run_ragged_decode(device, torch, paged=True)
     return out
 
 
@@ -645,7 +755,9 @@ def config_block(w, bits, copies):
     c = {"workload": w.name, "layers": 1, "batch": w.batch, "n_q_heads": w.n_q_heads,
          "n_kv_heads": w.n_kv_heads, "head_dim": 128, "context": w.context, "bits": bits,
          "quantizer": "QuEST INT", "sink": w.sink, "recent": w.recent, "chunk": w.chunk,
-         "input_dtype": w.dtype, "step": "append 1 token/seq + query transform + decode"}
+         "input_dtype": w.dtype, "step": "append 1 token/seq + query transform + decode",
+         "state": "each cache holds context - 1 prefilled tokens and takes one decode step "
+                  "before the warm-up steps"}
     if copies is not None:
         c["l2"] = (f"inputs larger than L2: {copies} independent caches cycled "
                    "(one per layer), ~90 MB of cache bytes each")
@@ -705,11 +817,15 @@ def main():
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": E, "counts": "step bytes / step time incl. pinned host<->device copies"},
         "step_breakdown": {"host_enqueue_us_per_step": r["host_s"] * 1e6 / K,
+                           "step_us_timed_region": r["ms"] * 1e3 / K,
+                           "step_us_graph": r["step_graph_us"],
                            "decode_us": dec_avg_ms * 1e3,
-                           "append_and_query_transform_us": r["ms"] * 1e3 / K - dec_avg_ms * 1e3,
+                           "step_kernel_us": r["step_graph_us"] - dec_avg_ms * 1e3,
                            "note": "per step: the step kernel (key append, query transform, chunk flush "
-                                   "every 8th step) runs before the decode; its time here is the step "
-                                   "time minus the decode launch time"},
+                                   "every 8th step) runs before the decode; step_us_graph is one step per "
+                                   "cache in a CUDA graph (no host in the loop), step_kernel_us = "
+                                   "step_us_graph - decode_us; the timed region's steps are issued from "
+                                   "the host one call at a time"},
         "gpu_launches": r["launches"], "clocks": r["clocks"], "device_status": r["status"],
     }
     if rank == 0 and world == 1 and not args.no_prefill:

@@ -44,6 +44,10 @@ constexpr int WC = WIN_BOX_ROWS; // window tokens per chunk
 constexpr int WIN_V = 2048;      // offset of the V tiles of a window chunk
 constexpr int PS_LD = PB + 16;   // bytes per row of the per-warp P tile
 constexpr int NSTAGE = 2;        // per-warp copy stages
+// Copies a warp issues before its first item; the rest of its ring fills
+// once the first copy has landed (at G = 8 that start measured faster, and
+// its code allocates registers without spills).
+template <int G> struct FirstCopies { static constexpr int N = G == 8 ? 1 : NSTAGE; };
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr unsigned FULL_MASK = 0xffffffffu;
 constexpr int PART = PARTIAL_FLOATS;  // floats per partial record (16-byte rows)
@@ -758,7 +762,7 @@ __device__ __forceinline__ void warp_items_prefetch(const DecodeArgs& a, const W
                                                     Smem<BITS, G>& sh, const GEO& geo, uint32_t y0, uint32_t y1,
                                                     int warp, int lane, uint32_t it, GCursor& ic) {
   ic.start(geo, y0);
-  for (uint32_t j = 0; j < (uint32_t)NSTAGE && y0 + j < y1; ++j) {
+  for (uint32_t j = 0; j < (uint32_t)FirstCopies<G>::N && y0 + j < y1; ++j) {
     const int stg = (it + j) % NSTAGE;
     int idx, seg;
     const bool win = ic.take(geo, &idx, &seg);
@@ -871,13 +875,19 @@ __device__ int warp_run(const DecodeArgs& a, const WindowMaps& wm, Smem<BITS, G>
         // A copy never completed: report it, drain what is still in flight
         // (bounded, at the full limit), and contribute nothing more.
         if (lane == 0) atomicOr(a.c.status, DEV_ERR_TIMEOUT);
-        const uint32_t inflight = min((uint32_t)NSTAGE, y1 - y);
+        const uint32_t inflight = y == y0 ? min((uint32_t)FirstCopies<G>::N, y1 - y) : min((uint32_t)NSTAGE, y1 - y);
         for (uint32_t q = 0; q < inflight; ++q)
           mbar_wait_bounded(&sh.bar[warp][(it + q) % NSTAGE], ((it + q) / NSTAGE) & 1, WAIT_POLLS);
         it += inflight;   // the ring is empty again, its phases in step
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) { S.m[nt] = -INFINITY; S.l[nt] = 0.f; S.e[nt] = 0.f; }
         return cur;
+      }
+      if (FirstCopies<G>::N < NSTAGE && y == y0 && y0 + 1 < y1) {   // the ring's second copy
+        int nidx, nseg;
+        const bool nwin = ic.take(geo, &nidx, &nseg);
+        const int s1 = (it + 1) % NSTAGE;
+        issue_item<BITS, AFFINE>(a, geo, nseg, wm, nwin, nidx, sh.stage[warp][s1], &sh.bar[warp][s1], lane);
       }
       const unsigned char* st = sh.stage[warp][stg];
       int idx;
@@ -957,6 +967,18 @@ __device__ __forceinline__ int unit_of(const DecodeArgs& a, const RaggedParam<RA
   }
 }
 
+// Segment geometry of the batch of nseg units from u_first into shared
+// memory (threads tid < UMAX; unused slots empty, past the batch's end).
+template <bool RAGGED, class SM>
+__device__ __forceinline__ void fill_batch_geom(const DecodeArgs& a, const RaggedParam<RAGGED>& rp, SM& sh,
+                                                int u_first, int nseg, int tid) {
+  if (tid < UMAX) {
+    SegGeom g = unit_geom<RAGGED>(a, rp, u_first + min(tid, nseg - 1));
+    if (tid >= nseg) { g.start += (uint32_t)g.ni; g.ni = 0; }
+    sh.geom[tid] = g;
+  }
+}
+
 template <int BITS, int G, bool AFFINE, bool RAGGED>
 __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ WindowMaps wm,
@@ -985,6 +1007,8 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
     if (warp == 0 && lane == 0) mbar_init(&sh.never, 1);
     fence_barrier_init();
   }
+  // the first batch's segment geometry depends on the parameters alone
+  if constexpr (RAGGED) fill_batch_geom<RAGGED>(a, rp, sh, U0, min(UMAX, U1 - U0 + 1), tid);
   __syncthreads();
   uint32_t it = 0;
   // q' and the cache may come from the kernel launched just before this one
@@ -994,13 +1018,11 @@ __global__ void __launch_bounds__(Warps<BITS>::N * 32, 1)
   for (int u_first = U0; u_first <= U1; u_first += UMAX) {
     const int nseg = min(UMAX, U1 - u_first + 1);
     const Geo<RAGGED, BITS, G> geo{sh, a, u_first};
-    if constexpr (RAGGED) {   // the batch's segment geometry (the previous batch ended with a barrier)
-      if (tid < UMAX) {
-        SegGeom g = unit_geom<RAGGED>(a, rp, u_first + min(tid, nseg - 1));
-        if (tid >= nseg) { g.start += (uint32_t)g.ni; g.ni = 0; }   // unused slots: empty, past the end
-        sh.geom[tid] = g;
+    if constexpr (RAGGED) {   // later batches' geometry (the previous batch ended with a barrier)
+      if (u_first != U0) {
+        fill_batch_geom<RAGGED>(a, rp, sh, u_first, nseg, tid);
+        __syncthreads();
       }
-      __syncthreads();
     }
     const SegGeom glast = geo(nseg - 1);
     const uint32_t x0 = max(X0, geo(0).start);
