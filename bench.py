@@ -280,10 +280,11 @@ def run_ours(args, rank, world, device, torch, dist):
         rest = append_bytes(w, bits, after[2] > before[2]) + qtransform_bytes(w)
         return dec, rest
 
-    def step(i, k, v, q, stream=stream):
+    def step(i, k, v, q, stream=stream, o=None):
         # one call: append 1 token + query transform (one launch) + decode
         c = i % args.copies
-        caches[c].decode_step(k, v, Ts[c], q, TinvTs[c], q_prime=qprime, out=out, stream=stream)
+        caches[c].decode_step(k, v, Ts[c], q, TinvTs[c], q_prime=qprime, out=out if o is None else o,
+                              stream=stream)
 
     # set-up: every cache (layer) takes one decode step before the warm-up,
     # as in a running server, so that no timed step is the first read of a
@@ -341,32 +342,70 @@ def run_ours(args, rank, world, device, torch, dist):
     e_first = first + K + 2 * args.copies
 
     # ---- e2e: host buffers, copies inside the timed region --------------------
+    # Each step's k, v and q sit back to back in one pinned host buffer: one
+    # host->device copy per step (on a copy stream, one step ahead, into one
+    # of two device buffers) and one device->host copy of the step's output
+    # (on a second copy stream, from one of two output buffers), ordered by
+    # events so neither buffer is reused before its copy or step is done.
     E = args.e2e_steps
-    host_out = torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory()
+    NB = 2
+    host_outs = [torch.empty((w.batch, w.n_q_heads, 128), dtype=torch.float32).pin_memory() for _ in range(NB)]
+    outs = [torch.empty_like(out) for _ in range(NB)]
     e_dec = 0
     for i in range(e_first, e_first + E):
         e_dec += sum(step_bytes(i))
-    # each step's k, v and q packed back to back in one pinned host buffer:
-    # one host->device copy per step, one device->host copy of the output
     shapes = [x.shape for x in pool[0]]
     sizes = [x.numel() for x in pool[0]]
     packed = [torch.cat([x.reshape(-1) for x in p]).pin_memory() for p in pool]
     h2d = packed[0].numel() * packed[0].element_size()
-    d2h = host_out.numel() * 4
-    dbuf = torch.empty_like(packed[0], device=device)
-    parts, off = [], 0
-    for shp, n in zip(shapes, sizes):
-        parts.append(dbuf[off:off + n].view(shp))
-        off += n
+    d2h = host_outs[0].numel() * 4
+    dbufs = [torch.empty_like(packed[0], device=device) for _ in range(NB)]
+    parts = []
+    for dbuf in dbufs:
+        pb, off = [], 0
+        for shp, n in zip(shapes, sizes):
+            pb.append(dbuf[off:off + n].view(shp))
+            off += n
+        parts.append(pb)
+    h2d_stream = torch.cuda.Stream(device=device)
+    d2h_stream = torch.cuda.Stream(device=device)
+    h2d_done = [torch.cuda.Event() for _ in range(NB)]
+    step_done = [torch.cuda.Event() for _ in range(NB)]
+    d2h_done = [torch.cuda.Event() for _ in range(NB)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+
+    def h2d_copy(j):
+        b = j % NB
+        with torch.cuda.stream(h2d_stream):
+            if j >= NB:
+                h2d_stream.wait_event(step_done[b])   # step j - NB has read this buffer
+            dbufs[b].copy_(packed[(e_first + j) % STEP_POOL], non_blocking=True)
+            h2d_done[b].record(h2d_stream)
+
     e0.record(stream)
-    for i in range(e_first, e_first + E):
-        dbuf.copy_(packed[i % STEP_POOL], non_blocking=True)
-        step(i, *parts)
-        host_out.copy_(out, non_blocking=True)
+    h2d_stream.wait_event(e0)
+    if E:
+        h2d_copy(0)
+    for j in range(E):
+        b = j % NB
+        if j + 1 < E:
+            h2d_copy(j + 1)
+        stream.wait_event(h2d_done[b])
+        if j >= NB:
+            stream.wait_event(d2h_done[b])                # output buffer b has been read back
+        step(e_first + j, *parts[b], o=outs[b])
+        step_done[b].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(step_done[b])
+            host_outs[b].copy_(outs[b], non_blocking=True)
+            d2h_done[b].record(d2h_stream)
+    if E:
+        stream.wait_event(d2h_done[(E - 1) % NB])
+        if E > 1:
+            stream.wait_event(d2h_done[(E - 2) % NB])
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
@@ -819,7 +858,9 @@ def main():
                                "replays on the launching stream, time / launches"},
         "e2e": {"value": world * e_dec / (e_ms / 1e3) / 1e9 if E else None,
                 "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": E, "counts": "step bytes / step time incl. pinned host<->device copies"},
+                "steps": E, "counts": "step bytes / step time incl. each step's pinned host->device input copy and "
+                                    "device->host output copy (two copy streams, double-buffered, ordered by "
+                                    "events)"},
         "step_breakdown": {"host_enqueue_us_per_step": r["host_s"] * 1e6 / K,
                            "step_us_timed_region": r["ms"] * 1e3 / K,
                            "step_us_graph": r["step_graph_us"],

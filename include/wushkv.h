@@ -33,8 +33,13 @@
  *     device status word read by wushkv_device_status.
  *   - head_dim is 128.  KV head of query head h is floor(h / G), G =
  *     n_q_heads / n_kv_heads (contiguous groups).
- *   - One cache object holds one layer for `batch` sequences that all hold
- *     the same number of tokens (every append adds n_tok to each sequence).
+ *   - One cache object holds one layer for `batch` sequences.  wushkv_append
+ *     adds n_tok tokens to every sequence; wushkv_append_varlen adds a
+ *     per-sequence count, and wushkv_reset_sequence empties one sequence, so
+ *     sequences may hold different numbers of tokens (the window policy
+ *     applies to each sequence on its own).  With num_pages > 0 the packed
+ *     region is paged through a caller-owned page table
+ *     (wushkv_set_page_table).
  *   - A "unit" is one (sequence b, KV head h); unit index u = b*n_kv_heads+h.
  */
 #ifndef WUSHKV_H
