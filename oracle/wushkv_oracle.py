@@ -639,6 +639,36 @@ class OracleCache:
         return out
 
 
+    def prefill_attention(self, q_prime: np.ndarray, scale: float | None = None,
+                          units: list[int] | None = None) -> np.ndarray:
+        """Causal attention of a chunk of queries over the cache (chunked
+        prefill), q' [B, n_q, Hq, 128] -> [B, n_q, Hq, 128].
+
+        READING (the pages describe no prefill attention; this is the plain
+        reading that the decode's rules give): the chunk's tokens are the last
+        n_q tokens of every sequence and have been appended first; the query
+        of token p = n - n_q + i attends to tokens 0 .. p as the cache holds
+        them (fp16 windows, dequantised packed tokens), just as a decode query
+        attends after its own token was appended.  ``units`` restricts the
+        work; other outputs are left NaN.
+        """
+        cfg = self.cfg
+        if scale is None:
+            scale = 1.0 / math.sqrt(HEAD_DIM)
+        B, nq, Hq, d = q_prime.shape
+        G = cfg.group
+        n = self.n
+        out = np.full((B, nq, Hq, d), np.nan)
+        for u in (range(cfg.units) if units is None else units):
+            b, h = divmod(u, cfg.n_kv_heads)
+            K, V = self.unit_kv(u)
+            for i in range(nq):
+                p = n - nq + i
+                out[b, i, h * G:(h + 1) * G] = attention_f64(q_prime[b, i, h * G:(h + 1) * G],
+                                                             K[:p + 1], V[:p + 1], scale)
+        return out
+
+
 # ---------------------------------------------------------------------------
 # Module-output error (summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
 # 关键实验, first bullet: the relative error of the attention module's output
