@@ -759,6 +759,30 @@ wushkv_status wushkv_decode_step(wushkv_cache* cache, const void* k_rope_dev, co
   return cuda_status(launch_decode(a, cache->wmaps, rt, s));
 }
 
+wushkv_status wushkv_prefill_attention(const float* q_prime_dev, const wushkv_cache* cache, float* out_dev,
+                                       int32_t n_q, float scale, void* stream) {
+  wushkv_status st = check_decode_args(q_prime_dev, cache, out_dev, scale);
+  if (st != WUSHKV_OK) return st;
+  const wushkv_config& c = cache->cfg;
+  if (!cache->uniform) return WUSHKV_EUNSUPPORTED;   // one count for every sequence
+  if (n_q < 1 || n_q > cache->n) return WUSHKV_EINVAL;
+  if (c.num_pages > 0 && cache->page_table == nullptr) return WUSHKV_EINVAL;
+  const int64_t units = (int64_t)c.batch * c.n_kv_heads;
+  if (units > 65535) return WUSHKV_EUNSUPPORTED;   // one grid row per unit
+  PaArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.c = dev_view(cache);
+  a.q = q_prime_dev;
+  a.out = out_dev;
+  a.n = (int)cache->n;
+  a.n_q = n_q;
+  a.ns = (int)std::min<int64_t>(cache->n, c.sink);
+  a.P = (int)packed_count(cache->n, c);
+  const float sc = scale > 0.f ? scale : 0.08838834764831845f;  // 1/sqrt(128)
+  a.scale_log2 = sc * 1.4426950408889634f;
+  return cuda_status(launch_prefill_attention(a, static_cast<cudaStream_t>(stream)));
+}
+
 wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dtype, const float* T_k_invT_dev,
                                      float* q_out_dev, int32_t batch, int32_t n_q_heads,
                                      int32_t n_kv_heads, void* stream) {

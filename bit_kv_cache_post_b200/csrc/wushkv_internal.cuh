@@ -512,4 +512,16 @@ struct RaggedTable {
 cudaError_t launch_decode(const DecodeArgs& a, const WindowMaps& m, const RaggedTable* rt, cudaStream_t s);
 int decode_ctas_per_sm(int bits, int group, int quantizer);
 
+// Chunked-prefill attention: q [batch][n_q][n_q_heads][128] fp32 (the last
+// n_q tokens' transformed queries), out likewise; every sequence holds n
+// tokens (ns sink, P packed, the rest in the ring).
+struct PaArgs {
+  DevCache c;
+  const float* q;
+  float* out;
+  int n, n_q, ns, P;
+  float scale_log2;
+};
+cudaError_t launch_prefill_attention(const PaArgs& a, cudaStream_t s);
+
 }  // namespace wushkv

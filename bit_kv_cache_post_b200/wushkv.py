@@ -22,6 +22,7 @@ EXPORTED = [
     "wushkv_export", "wushkv_device_status", "wushkv_default_quest_alpha", "wushkv_strerror",
     "wushkv_decode_noalloc", "wushkv_decode_step", "wushkv_inject_decode_timeout",
     "wushkv_sequence_tokens", "wushkv_reset_sequence", "wushkv_set_page_table", "wushkv_append_varlen",
+    "wushkv_prefill_attention",
 ]
 
 # bits of the sticky device status word; guard bands after each cache region
@@ -86,6 +87,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_query_transform.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp]
     lib.wushkv_decode.argtypes = [vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_decode_noalloc.argtypes = [vp, vp, vp, ctypes.c_float, vp]
+    lib.wushkv_prefill_attention.argtypes = [vp, vp, vp, i32, ctypes.c_float, vp]
     lib.wushkv_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp]
     lib.wushkv_export.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     lib.wushkv_device_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
@@ -267,6 +269,18 @@ class Cache:
                                          T.data_ptr(), q.data_ptr(), _dtype_code(q), TinvT.data_ptr(),
                                          q_prime.data_ptr(), out.data_ptr(), scale, _stream_ptr(stream)),
                "wushkv_decode_step")
+        return out
+
+    def prefill_attention(self, q_prime, n_q: int, out=None, scale: float = 0.0, stream=None):
+        """Causal attention of the last n_q tokens' queries (q_prime:
+        [B, n_q, Hq, 128] fp32, transformed) over the cache; returns out of
+        the same shape."""
+        import torch
+        assert q_prime.is_contiguous() and q_prime.dtype == torch.float32 and q_prime.shape[1] == n_q
+        if out is None:
+            out = torch.empty_like(q_prime)
+        _check(load().wushkv_prefill_attention(q_prime.data_ptr(), self._handle, out.data_ptr(), int(n_q),
+                                               scale, _stream_ptr(stream)), "wushkv_prefill_attention")
         return out
 
     def decode_noalloc(self, q_prime, out=None, scale: float = 0.0, stream=None):

@@ -263,6 +263,26 @@ WUSHKV_API wushkv_status wushkv_query_transform(const void* q_dev, int32_t q_dty
                                      float* q_out_dev, int32_t batch, int32_t n_q_heads,
                                      int32_t n_kv_heads, void* stream);
 
+/* Chunked-prefill attention: the queries of the last n_q tokens of every
+ * sequence attend causally to the cache.
+ *   Source: not on the pages (they describe decoding); the decode's rules
+ *   apply (summary page "WUSH-KV：数据自适应变换的 KV Cache 低比特量化",
+ *   方法关键点: keys through T_k after RoPE, queries through T_k^{-T}).  The
+ *   chunk's tokens have been appended first (wushkv_append); the query of
+ *   token p = n - n_q + i attends to tokens 0 .. p as the cache holds them
+ *   (fp16 sink and recent rows, dequantised packed tokens).
+ *   q_prime_dev: [batch][n_q][n_q_heads][128] fp32 transformed queries
+ *                (wushkv_query_transform with batch * n_q rows), 16-byte
+ *                aligned (EINVAL otherwise).
+ *   out_dev:     [batch][n_q][n_q_heads][128] fp32, 16-byte aligned.
+ *   n_q: 1 .. tokens per sequence (EINVAL otherwise); scale as wushkv_decode.
+ * Every sequence must hold the same number of tokens (EUNSUPPORTED
+ * otherwise); dense and paged caches; at most 65535 (sequence, KV head)
+ * units.  Reads the cache only (no workspace), so it may run concurrently
+ * with other readers of the cache. */
+WUSHKV_API wushkv_status wushkv_prefill_attention(const float* q_prime_dev, const wushkv_cache* cache,
+                                                  float* out_dev, int32_t n_q, float scale, void* stream);
+
 /* GQA decode attention of one query per query head over the whole cache.
  *   Source: review "[논문리뷰] WUSH-KV ..." (secrett2633), Key Terms (GQA);
  *   dequantisation happens inside the score and PV loops.
