@@ -596,6 +596,80 @@ def run_ragged_decode(device, torch, paged: bool, copies=8, bits=2):
             "frac": nbytes / us / 1e3 / peak, "copies": copies, "device_status": status}
 
 
+def run_prefill_attention(device, torch, nq=512, copies=4, bits=2):
+    """Chunked-prefill attention at the batch-16 Qwen3-8B-shaped layer: each
+    sequence holds 8192 tokens of which the last nq are the chunk; its
+    queries attend causally over the quantised cache.  Launches back to back
+    in a CUDA graph over `copies` caches.  Algorithmic flops: 4 x 128 per
+    (query head, visible token) (q.k and p.v)."""
+    from bit_kv_cache_post_b200 import inputs as I
+    from bit_kv_cache_post_b200 import wushkv as wk
+    w = I.WORKLOADS[WORKLOAD]
+    n = w.context
+    k, v = I.device_kv(w, 0, n, device=device)
+    T, TinvT = I.key_transforms(w, 0)
+    Td, TinvTd = torch.from_numpy(T).to(device), torch.from_numpy(TinvT).to(device)
+    cfg = wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, n, bits=bits, sink=w.sink,
+                         recent=w.recent, chunk=w.chunk)
+    caches = []
+    for _ in range(copies):
+        c = wk.Cache(cfg, device=device)
+        c.append(k, v, Td)
+        caches.append(c)
+    del k, v
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([w.wid, 7]).generate_state(1)[0]))
+    q = torch.randn((w.batch * nq, w.n_q_heads, 128), generator=g, device=device).bfloat16()
+    qp = wk.query_transform(q, TinvTd).view(w.batch, nq, w.n_q_heads, 128).contiguous()
+    out = torch.empty_like(qp)
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream(device=device)
+    cap.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        for c in caches:
+            c.prefill_attention(qp, nq, out=out, stream=cap)
+        cap.synchronize()
+        with torch.cuda.graph(graph, stream=cap):
+            for c in caches:
+                c.prefill_attention(qp, nq, out=out, stream=cap)
+    stream.wait_stream(cap)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    reps = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    del graph
+    status = max(c.device_status() for c in caches)
+    visible = nq * (n - nq) + nq * (nq + 1) // 2          # (query, token) pairs per head
+    flops = 4.0 * 128 * visible * w.batch * w.n_q_heads
+    peak_tf = peaks_tensor()
+    tf = flops / us / 1e6
+    return {"workload": f"{WORKLOAD}: chunk of the last {nq} of {n} tokens per sequence, {bits}-bit QuEST, G {w.group}",
+            "us_per_launch": us, "query_tokens_per_s": w.batch * nq / (us / 1e6),
+            "algorithmic_tflops": tf, "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf[0],
+                                                   "unit": "TFLOP/s", "frac": tf / peak_tf[0],
+                                                   "peak_source": peak_tf[1]},
+            "kernel": "fp16 mma.sync (m16n8k16), scores with the query as hi + lo terms",
+            "copies": copies, "device_status": status,
+            "timing": "launches back to back in a CUDA graph over the cycled caches, CUDA events"}
+
+
+def peaks_tensor():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "of measured (MEASURED_PEAKS.json bf16_tflops, burst; fp16 runs at the bf16 rate)"
+    except Exception:
+        return 1590.0, "of fallback (1.59 PFLOP/s)"
+
+
 def run_extra(device, torch):
     """Decode GB/s of the 32B-shaped, 4B-shaped long-context and 36-layer
     (one layer, affine) workloads, config-1 decode at 3 and 4 bits, and the
@@ -614,6 +688,7 @@ def run_extra(device, torch):
         out[key] = res
         del caches
         torch.cuda.empty_cache()
+    out["prefill_attention_" + WORKLOAD] = run_prefill_attention(device, torch)
     out["ragged_" + WORKLOAD] = run_ragged_decode(device, torch, paged=False)
     out["ragged_paged_" + WORKLOAD] = run_ragged_decode(device, torch, paged=True)
     return out

@@ -182,3 +182,37 @@ def test_prefill_attention_last_row_is_decode(wk):
     dec = cache.decode(torch.from_numpy(np.ascontiguousarray(q[:, -1])).cuda()).cpu().numpy()
     rms = math.sqrt(float(np.mean(dec.astype(np.float64) ** 2)))
     assert np.abs(out[:, -1] - dec).max() / rms <= DECODE_TOL
+
+
+@pytest.mark.gpu
+def test_prefill_attention_qwen3_8b_layer_chunk512(wk):
+    """Full-size Qwen3-8B-shaped layer (batch 16, 8 KV heads, G 4, bf16):
+    8192 tokens appended through the key transform, the last 512 of them
+    the chunk.  Sampled units and queries against float64 causal attention
+    over the GPU cache's own state (read through wushkv_export and
+    dequantised with the oracle's rules)."""
+    import torch
+    from bit_kv_cache_post_b200 import inputs as I
+    w = I.WORKLOADS["qwen3-8b-layer-b16-ctx8192"]
+    n, nq, G = w.context, 512, w.group
+    k, v = I.device_kv(w, 0, n)
+    T, TinvT = I.key_transforms(w, 0)
+    cache = wk.Cache(wk.make_config(w.batch, w.n_kv_heads, w.n_q_heads, n, bits=2))
+    cache.append(k, v, torch.from_numpy(T).cuda())
+    del k, v
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    q = torch.randn((w.batch * nq, w.n_q_heads, 128), generator=g, device="cuda").bfloat16()
+    qp = wk.query_transform(q, torch.from_numpy(TinvT).cuda()).view(w.batch, nq, w.n_q_heads, 128)
+    out = cache.prefill_attention(qp.contiguous(), nq).cpu().numpy()
+    qp = qp.cpu().numpy().astype(np.float64)
+    assert cache.device_status() == 0
+    rng = np.random.default_rng(5)
+    for b, h in [(0, 0), (15, 7), (int(rng.integers(16)), int(rng.integers(8)))]:
+        Kg, Vg = H.unit_state_from_export(cache, b, h)
+        for i in sorted(set([0, nq - 1] + list(rng.integers(0, nq, 6)))):
+            p = n - nq + i
+            want = O.attention_f64(qp[b, i, h * G:(h + 1) * G], Kg[:p + 1], Vg[:p + 1], 1.0 / np.sqrt(128.0))
+            got = out[b, i, h * G:(h + 1) * G]
+            assert np.abs(got - want).max() / math.sqrt(float(np.mean(want ** 2))) <= DECODE_TOL, (b, h, i)
+    H.check_guards(cache)
