@@ -870,7 +870,12 @@ wushkv_status wushkv_export(const wushkv_cache* cache, int32_t seq, int32_t head
         for (int d = 0; d < 128; ++d) {
           uint32_t wd;
           int bit;
-          if (kv == 0) {
+          if (kv == 0 && c.bits == 2) {   // K quads
+            const int64_t quad = pk / 4;
+            wd = word_at(L.k_plane_off[p], quad / 16,
+                         (size_t)(quad % 16) * 128 + 4 * (size_t)k2_word_pos(quad, d / 4));
+            bit = 8 * (d % 4) + 2 * (int)(pk % 4);
+          } else if (kv == 0) {
             const int ks = d / 32, rem = d % 32, h2 = rem / 16, c4 = (rem % 16) / 4, beta = d % 4;
             const int rho = 4 * h2 + ks;
             wd = word_at(L.k_plane_off[p], pk / 64, (size_t)k_row_pos(pk) * 16 * w + 4 * (c4 * w + rho / F));

@@ -179,7 +179,18 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, int64_t bx, int
       __syncthreads();
       for (int p = 0; p < c.n_planes; ++p) {
         const int w = c.plane_bits[p], P = 8 / w;
-        if (kv == 0) {
+        if (kv == 0 && c.bits == 2) {
+          // one K quad, 32 words: thread tid builds word omega = tid from the
+          // four tokens' codes of dims 4 tid .. 4 tid + 3
+          if (tid < 32) {
+            uint32_t word = 0;
+            for (int f = 0; f < 4; ++f)
+              for (int beta = 0; beta < 4; ++beta)
+                word |= (uint32_t)codes[f * D + 4 * tid + beta] << (8 * beta + 2 * f);
+            const int64_t quad = pk / 4;
+            reinterpret_cast<uint32_t*>(k_quad_at(c, u, quad))[k2_word_pos(quad, tid)] = word;
+          }
+        } else if (kv == 0) {
           // four K rows, 4w words each: warp = token, lane = word
           if (lane < 4 * w) {
             uint32_t word = 0;

@@ -395,6 +395,15 @@ __device__ __forceinline__ VWords<BITS> stage_v_words(const unsigned char* st, i
 }
 
 
+// Token (within the block) of slot j = 2 mt + th of lane row r: 2-bit keys
+// come in quads (m-tile mt = field mt of quads r and r + 8), wider keys in
+// rows (8 consecutive tokens per lane).
+template <int BITS>
+__device__ __forceinline__ int slot_token(int r, int j) {
+  if constexpr (BITS == 2) return 4 * r + 32 * (j & 1) + (j >> 1);
+  else return 8 * r + j;
+}
+
 // Lane = 4r + c.  Score m-tile rows r, r+8 are tokens; columns are (head,
 // term) pairs, so thread c owns head 4nt + c of n-tile nt.  PV m-tile rows
 // are dims 16mt + r (+8); the PV B operand comes back through the warp's P
@@ -425,18 +434,35 @@ __device__ __forceinline__ void packed_block_compute(
     float ks_[8], ko_[8];
     if constexpr (AFFINE) {
 #pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
-        const uint4 km = *reinterpret_cast<const uint4*>(st + SL::K_META + 32 * r + 16 * hq);
-        const uint4 vm = *reinterpret_cast<const uint4*>(st + SL::V_META + 32 * r + 16 * hq);
+      for (int hq = 0; hq < 2; ++hq) {   // four consecutive tokens per load (slot_token)
+        const int off = BITS == 2 ? 16 * r + 128 * hq : 32 * r + 16 * hq;
+        const uint4 km = *reinterpret_cast<const uint4*>(st + SL::K_META + off);
+        const uint4 vm = *reinterpret_cast<const uint4*>(st + SL::V_META + off);
         const uint32_t kw[4] = {km.x, km.y, km.z, km.w}, vw[4] = {vm.x, vm.y, vm.z, vm.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          const int j = BITS == 2 ? 2 * e + hq : 4 * hq + e;
           const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&kw[e]));
           const float2 vf = __half22float2(*reinterpret_cast<const __half2*>(&vw[e]));
-          ks_[4 * hq + e] = kf.x; ko_[4 * hq + e] = kf.y;
-          vs[4 * hq + e] = vf.x; vo[4 * hq + e] = vf.y;
+          ks_[j] = kf.x; ko_[j] = kf.y;
+          vs[j] = vf.x; vo[j] = vf.y;
         }
       }
+    } else if constexpr (BITS == 2) {
+      // the lane's tokens 4r .. 4r + 3 (th = 0) and 4r + 32 .. 4r + 35 (th = 1)
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+        const uint2 km = *reinterpret_cast<const uint2*>(st + SL::K_META + 8 * r + 64 * th);
+        const uint2 vm = *reinterpret_cast<const uint2*>(st + SL::V_META + 8 * r + 64 * th);
+        const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&km.x));
+        const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&km.y));
+        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vm.x));
+        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vm.y));
+        ks_[th] = k01.x; ks_[2 + th] = k01.y; ks_[4 + th] = k23.x; ks_[6 + th] = k23.y;
+        vs[th] = v01.x; vs[2 + th] = v01.y; vs[4 + th] = v23.x; vs[6 + th] = v23.y;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ko_[j] = vo[j] = 0.f;
     } else {
       const uint4 km = *reinterpret_cast<const uint4*>(st + SL::K_META + 16 * r);
       const uint4 vm = *reinterpret_cast<const uint4*>(st + SL::V_META + 16 * r);
@@ -450,31 +476,61 @@ __device__ __forceinline__ void packed_block_compute(
         ko_[2 * e] = ko_[2 * e + 1] = vo[2 * e] = vo[2 * e + 1] = 0.f;
       }
     }
+    // K fragments of m-tile mt, k-step ks: rows r, r + 8 are tokens
+    // slot_token(r, 2 mt), slot_token(r, 2 mt + 1); 2-bit words carry the
+    // m-tile's field in place (times 4^mt, removed with the query scale)
+    uint32_t wr[4][2], w8[4][2];   // 2-bit: words [ks][h] of quads r and r + 8
+    if constexpr (BITS == 2) {
+      const int xq = r & 1;
+      const unsigned char* q0 = st + SL::K_LO + r * 128;
+      const unsigned char* q1 = st + SL::K_LO + (r + 8) * 128;
+      const uint4 a0 = *reinterpret_cast<const uint4*>(q0 + ((2 * c4) ^ xq) * 16);
+      const uint4 a1 = *reinterpret_cast<const uint4*>(q0 + ((2 * c4 + 1) ^ xq) * 16);
+      const uint4 b0 = *reinterpret_cast<const uint4*>(q1 + ((2 * c4) ^ xq) * 16);
+      const uint4 b1 = *reinterpret_cast<const uint4*>(q1 + ((2 * c4 + 1) ^ xq) * 16);
+      wr[0][0] = a0.x; wr[0][1] = a0.y; wr[1][0] = a0.z; wr[1][1] = a0.w;
+      wr[2][0] = a1.x; wr[2][1] = a1.y; wr[3][0] = a1.z; wr[3][1] = a1.w;
+      w8[0][0] = b0.x; w8[0][1] = b0.y; w8[1][0] = b0.z; w8[1][1] = b0.w;
+      w8[2][0] = b1.x; w8[2][1] = b1.y; w8[3][0] = b1.z; w8[3][1] = b1.w;
+    }
     const int x = r & 3;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
-      const KWords<BITS> kw0 = stage_k_words<BITS>(st, 8 * r + ((2 * mt) ^ x), c4);
-      const KWords<BITS> kw1 = stage_k_words<BITS>(st, 8 * r + ((2 * mt + 1) ^ x), c4);
       int acc[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+      if constexpr (BITS == 2) {
+        const uint32_t m = 0x03030303u << (2 * mt);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint32_t a0 = k_frag<BITS>(kw0, ks, 0), a1 = k_frag<BITS>(kw1, ks, 0);
-        const uint32_t a2 = k_frag<BITS>(kw0, ks, 1), a3 = k_frag<BITS>(kw1, ks, 1);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t a0 = wr[ks][0] & m, a1 = w8[ks][0] & m, a2 = wr[ks][1] & m, a3 = w8[ks][1] & m;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+        }
+      } else {
+        const KWords<BITS> kw0 = stage_k_words<BITS>(st, 8 * r + ((2 * mt) ^ x), c4);
+        const KWords<BITS> kw1 = stage_k_words<BITS>(st, 8 * r + ((2 * mt + 1) ^ x), c4);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t a0 = k_frag<BITS>(kw0, ks, 0), a1 = k_frag<BITS>(kw1, ks, 0);
+          const uint32_t a2 = k_frag<BITS>(kw0, ks, 1), a3 = k_frag<BITS>(kw1, ks, 1);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_u8s8(acc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+        }
       }
+      constexpr float kf4[4] = {1.f, 0.25f, 0.0625f, 0.015625f};
+      const float fmt = BITS == 2 ? kf4[mt] : 1.f;   // 4^-mt (exact)
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
         const int j = 2 * mt + th;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const float xf = (float)(acc[nt][2 * th] * 254 + acc[nt][2 * th + 1]);
+          const float qsc = qscale[nt] * fmt;
           float d;   // score minus the reference maximum in use
-          if constexpr (AFFINE) d = fmaf(ks_[j], qscale[nt] * xf, fmaf(ko_[j], qsum[nt], nm[nt]));
-          else d = fmaf(ks_[j], fmaf(qscale[nt], xf, qoff[nt]), nm[nt]);   // delta (q.c + beta sum q) - m
-          if constexpr (!FULL) d = (8 * r + j < nvalid) ? d : -INFINITY;
+          if constexpr (AFFINE) d = fmaf(ks_[j], qsc * xf, fmaf(ko_[j], qsum[nt], nm[nt]));
+          else d = fmaf(ks_[j], fmaf(qsc, xf, qoff[nt]), nm[nt]);   // delta (q.c + beta sum q) - m
+          if constexpr (!FULL) d = (slot_token<BITS>(r, j) < nvalid) ? d : -INFINITY;
           sc[j][nt] = d;
         }
       }
@@ -508,7 +564,7 @@ __device__ __forceinline__ void packed_block_compute(
     for (int j = 0; j < 8; ++j) {
       const float p = ex2(sc[j][nt]);   // masked tokens: exp2(-inf) = 0
       float pt = p * vs[j];
-      if constexpr (!FULL) pt = (8 * r + j < nvalid) ? pt : 0.f;
+      if constexpr (!FULL) pt = (slot_token<BITS>(r, j) < nvalid) ? pt : 0.f;
       ls += p;
       if constexpr (AFFINE) es = fmaf(p, vo[j], es);
       else es += pt;                                 // times beta at the end
@@ -552,15 +608,23 @@ __device__ __forceinline__ void packed_block_compute(
     for (int j = 0; j < 8; ++j) bw[j] = __float_as_uint(fmaf(sc[j][nt], inv, 12582912.f));
     uint32_t t0w[2], t1w[2];
 #pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-      const uint32_t x01 = __byte_perm(bw[4 * hq], bw[4 * hq + 1], 0x5140);      // lo0 lo1 hi0 hi1
-      const uint32_t x23 = __byte_perm(bw[4 * hq + 2], bw[4 * hq + 3], 0x5140);  // lo2 lo3 hi2 hi3
+    for (int hq = 0; hq < 2; ++hq) {   // four consecutive tokens (slot_token) per word
+      const int j0 = BITS == 2 ? hq : 4 * hq, dj = BITS == 2 ? 2 : 1;
+      const uint32_t x01 = __byte_perm(bw[j0], bw[j0 + dj], 0x5140);               // lo0 lo1 hi0 hi1
+      const uint32_t x23 = __byte_perm(bw[j0 + 2 * dj], bw[j0 + 3 * dj], 0x5140);  // lo2 lo3 hi2 hi3
       t1w[hq] = __byte_perm(x01, x23, 0x5410);
       t0w[hq] = __byte_perm(x01, x23, 0x7632);
     }
     const int col = nt * 8 + 2 * c4;
-    *reinterpret_cast<uint2*>(ps + col * PS_LD + 8 * r) = make_uint2(t0w[0], t0w[1]);
-    *reinterpret_cast<uint2*>(ps + (col + 1) * PS_LD + 8 * r) = make_uint2(t1w[0], t1w[1]);
+    if constexpr (BITS == 2) {   // tokens 4r .. 4r + 3 and 4r + 32 .. 4r + 35
+      *reinterpret_cast<uint32_t*>(ps + col * PS_LD + 4 * r) = t0w[0];
+      *reinterpret_cast<uint32_t*>(ps + col * PS_LD + 4 * r + 32) = t0w[1];
+      *reinterpret_cast<uint32_t*>(ps + (col + 1) * PS_LD + 4 * r) = t1w[0];
+      *reinterpret_cast<uint32_t*>(ps + (col + 1) * PS_LD + 4 * r + 32) = t1w[1];
+    } else {
+      *reinterpret_cast<uint2*>(ps + col * PS_LD + 8 * r) = make_uint2(t0w[0], t0w[1]);
+      *reinterpret_cast<uint2*>(ps + (col + 1) * PS_LD + 8 * r) = make_uint2(t1w[0], t1w[1]);
+    }
   }
   __syncwarp();
 

@@ -93,8 +93,15 @@ __device__ __forceinline__ void load_block(const DevCache& c, int u, int blk, in
     const int nk = p == 0 ? PL::K0 : PL::K1, nv = p == 0 ? PL::V0 : PL::V1;
 #pragma unroll
     for (int j = 0; j < (p == 0 ? PL::K0 : PL::K1); ++j) {
-      const int e = tid + PA_THREADS * j, i = e / (4 * w), wi = e % (4 * w);
-      const uint32_t x = i < cnt ? __ldg(reinterpret_cast<const uint32_t*>(kb + (size_t)k_row_pos(i) * 16 * w) + wi) : 0u;
+      const int e = tid + PA_THREADS * j;
+      uint32_t x;
+      if constexpr (BITS == 2) {   // K quads: quad e / 32, word omega = e % 32
+        const int q = e >> 5, om = e & 31;
+        x = 4 * q < cnt ? __ldg(reinterpret_cast<const uint32_t*>(kb + (size_t)q * 128) + k2_word_pos(q, om)) : 0u;
+      } else {
+        const int i = e / (4 * w), wi = e % (4 * w);
+        x = i < cnt ? __ldg(reinterpret_cast<const uint32_t*>(kb + (size_t)k_row_pos(i) * 16 * w) + wi) : 0u;
+      }
       if (p == 0) r.k0[j] = x; else r.k1[j] = x;
     }
 #pragma unroll
@@ -135,16 +142,26 @@ __device__ __forceinline__ void write_block(const DevCache& c, PaSmem& sh, int c
     const float mul = p == 0 ? 1.f : 4.f;
 #pragma unroll
     for (int j = 0; j < (p == 0 ? PL::K0 : PL::K1); ++j) {
-      const int e = tid + PA_THREADS * j, i = e / (4 * w), wi = e % (4 * w);
+      const int e = tid + PA_THREADS * j;
       const uint32_t word = p == 0 ? r.k0[j] : r.k1[j];
+      if constexpr (BITS == 2) {   // K quads: field f = token 4q + f, byte beta = dim 4 omega + beta
+        const int q = e >> 5, om = e & 31;
 #pragma unroll
-      for (int beta = 0; beta < 4; ++beta)
+        for (int f = 0; f < 4; ++f)
 #pragma unroll
-        for (int s = 0; s < F; ++s) {
-          const float v = (float)((word >> (8 * beta + w * s)) & mask) * mul;
-          __half* dst = &sh.kr[i][k_field_dim(wi, w, s, beta)];
-          *dst = p == 0 ? __float2half_rn(v) : __float2half_rn(__half2float(*dst) + v);
-        }
+          for (int beta = 0; beta < 4; ++beta)
+            sh.kr[4 * q + f][4 * om + beta] = __float2half_rn((float)((word >> (8 * beta + 2 * f)) & 3u));
+      } else {
+        const int i = e / (4 * w), wi = e % (4 * w);
+#pragma unroll
+        for (int beta = 0; beta < 4; ++beta)
+#pragma unroll
+          for (int s = 0; s < F; ++s) {
+            const float v = (float)((word >> (8 * beta + w * s)) & mask) * mul;
+            __half* dst = &sh.kr[i][k_field_dim(wi, w, s, beta)];
+            *dst = p == 0 ? __float2half_rn(v) : __float2half_rn(__half2float(*dst) + v);
+          }
+      }
     }
 #pragma unroll
     for (int j = 0; j < (p == 0 ? PL::V0 : PL::V1); ++j) {

@@ -192,7 +192,7 @@ __device__ __forceinline__ void key_codes(uint32_t taddr, const QParams& q, bool
 template <int BITS, bool AFFINE>
 __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double alpha,
                                         bool lo_second, bool hi_second, int mode, uint8_t* row0,
-                                        uint8_t* row1, uint8_t* meta_p, __half* win) {
+                                        uint8_t* row1, uint8_t* meta_p, __half* win, int64_t quad) {
   const bool packed = mode == ROW_PACKED;
   AffineStats ast;
   QuestStats qst;
@@ -234,8 +234,31 @@ __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double a
 #pragma unroll
   for (int i = 0; i < 4; ++i) w1[i] = 0u;
   key_codes<BITS, AFFINE>(taddr, q, packed, w0, w1, row0);
+  if constexpr (BITS == 2) {
+    // 2-bit keys are stored in quads of 4 tokens (the four lanes 4k .. 4k + 3
+    // hold a quad's rows): word (c, h) of lane f holds k-step ks at field ks;
+    // the quad's word omega = 8 ks + 4 h + c holds token f at field f.  Lane
+    // f collects the words of k-step f from the four lanes.
+    const int lane = threadIdx.x & 31, f = lane & 3;
+    uint32_t qw[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {   // x = 2 c + h
+      uint32_t acc = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int dst = (f - j) & 3;   // the lane that takes this round's value
+        const uint32_t send = ((w0[x] >> (2 * dst)) & 0x03030303u) << (2 * f);
+        acc |= __shfl_sync(FULL, send, (lane & ~3) | ((f + j) & 3));
+      }
+      qw[x] = acc;
+    }
+    if (!packed) return;
+    uint32_t* o = reinterpret_cast<uint32_t*>(row0);   // the quad's 128 bytes
+#pragma unroll
+    for (int x = 0; x < 8; ++x) o[k2_word_pos(quad, 8 * f + 4 * (x & 1) + (x >> 1))] = qw[x];
+  }
   if (!packed) return;
-  if constexpr (BITS != 4) {
+  if constexpr (BITS == 3) {
     uint4* o0 = reinterpret_cast<uint4*>(row0);
     o0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
     o0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
@@ -481,9 +504,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool pkd = mode == ROW_PACKED;
       key_row<BITS, AFFINE>(
           taddr, unscale, c.alpha, lo_second, hi_second, mode,
-          pkd ? k_row_at(c, 0, t.u, (int64_t)pkc) : nullptr,
+          pkd ? (BITS == 2 ? k_quad_at(c, t.u, (int64_t)pkc / 4) : k_row_at(c, 0, t.u, (int64_t)pkc)) : nullptr,
           (BITS == 3 && pkd) ? k_row_at(c, 1, t.u, (int64_t)pkc) : nullptr,
-          pkd ? k_meta_at(c, t.u, (int64_t)pkc) : nullptr, win);
+          pkd ? k_meta_at(c, t.u, (int64_t)pkc) : nullptr, win, (int64_t)pkc / 4);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[g]);

@@ -77,7 +77,22 @@ __device__ __forceinline__ uint64_t block_offset(const DevCache& c, int64_t u, i
   return ((uint64_t)page * c.n_kv_heads + (uint64_t)h) * c.block_stride;
 }
 
-// Address of the K row (16 w bytes, plane p) of packed token pk of unit u.
+// 2-bit keys are packed in quads of 4 consecutive tokens (128 bytes, 32
+// words): word omega holds dims 4 omega .. 4 omega + 3 at its bytes and token
+// 4 quad + f at field f of each byte; with omega = 8 ks + 4 h + c it sits at
+// this position of the quad (the decode's lane c reads its eight words of a
+// quad as two 16-byte chunks, adjacent quads on alternating chunks).
+__host__ __device__ __forceinline__ int k2_word_pos(int64_t quad, int omega) {
+  const int ks = omega >> 3, h = (omega >> 2) & 1, c = omega & 3;
+  return 4 * ((2 * c + (ks >> 1)) ^ (int)(quad & 1)) + 2 * (ks & 1) + h;
+}
+// Address of 2-bit K quad `quad` (packed tokens 4 quad .. 4 quad + 3) of unit u.
+__device__ __forceinline__ uint8_t* k_quad_at(const DevCache& c, int64_t u, int64_t quad) {
+  return c.k_plane[0] + block_offset(c, u, quad >> 4) + (uint64_t)(quad & 15) * 128;
+}
+
+// Address of the K row (16 w bytes, plane p) of packed token pk of unit u
+// (3- and 4-bit keys).
 __device__ __forceinline__ uint8_t* k_row_at(const DevCache& c, int p, int64_t u, int64_t pk) {
   return c.k_plane[p] + block_offset(c, u, pk >> 6) + (uint64_t)k_row_pos(pk) * 16 * c.plane_bits[p];
 }

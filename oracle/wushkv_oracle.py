@@ -324,9 +324,13 @@ def affine_dequantize(codes: np.ndarray, s_h: np.ndarray, lo_h: np.ndarray) -> n
 #           (code >> 2).  A plane of width w packs P = 8 / w fields in each
 #           byte; field s of byte beta of a 32-bit little-endian word sits at
 #           bit 8*beta + w*s.
-#   K rows (one token, 128 dims, 4w words per plane): for c in 0..3,
-#     h in 0..1, ks in 0..3, beta in 0..3, rho = 4h + ks:
+#   K rows, 3 and 4 bits (one token, 128 dims, 4w words per plane): for c in
+#     0..3, h in 0..1, ks in 0..3, beta in 0..3, rho = 4h + ks:
 #       word = c*w + rho // P, field s = rho % P, dim = 32ks + 4c + 16h + beta.
+#   K quads, 2 bits (4 consecutive tokens, 32 words): word omega holds dims
+#     4 omega + beta at byte beta, and token 4*quad + f at field f; with
+#     omega = 8ks + 4h + c it is stored at position
+#     4 ((2c + ks // 2) xor (quad mod 2)) + 2 (ks mod 2) + h of the quad.
 #   V quads (4 consecutive tokens, 8*2w words per plane): for r in 0..7,
 #     rho in 0..15 (mt = rho // 2, rh = rho % 2), beta in 0..3:
 #       unit word j = rho // P, field s = rho % P,
@@ -348,8 +352,28 @@ def _plane_values(codes: np.ndarray, bits: int) -> list[np.ndarray]:
     return [c]
 
 
+def k2_word_pos(quad: int, omega: int) -> int:
+    """Position of word omega (dims 4 omega .. 4 omega + 3) in a 2-bit K quad."""
+    ks, h, c = omega // 8, (omega // 4) % 2, omega % 4
+    return 4 * ((2 * c + ks // 2) ^ (quad % 2)) + 2 * (ks % 2) + h
+
+
 def pack_k_rows(codes: np.ndarray, bits: int) -> list[np.ndarray]:
-    """codes [N, 128] -> one uint32 array [N, 4w] per plane."""
+    """codes [N, 128] -> one uint32 array per plane: [N, 4w] token rows at 3
+    and 4 bits; [N / 4, 32] quads at 2 bits (N a multiple of 4)."""
+    if bits == 2:
+        n = codes.shape[0]
+        assert n % 4 == 0, "2-bit K codes are packed in quads of 4 tokens"
+        c = codes.astype(np.uint32).reshape(n // 4, 4, HEAD_DIM)
+        words = np.zeros((n // 4, 32), dtype=np.uint32)
+        for q in range(n // 4):
+            for omega in range(32):
+                wd = np.uint32(0)
+                for beta in range(4):
+                    for f in range(4):
+                        wd |= c[q, f, 4 * omega + beta] << np.uint32(8 * beta + 2 * f)
+                words[q, k2_word_pos(q, omega)] = wd
+        return [words]
     out = []
     for w, vals in zip(plane_widths(bits), _plane_values(codes, bits)):
         P = 8 // w
@@ -367,7 +391,18 @@ def pack_k_rows(codes: np.ndarray, bits: int) -> list[np.ndarray]:
 
 
 def unpack_k_rows(planes: list[np.ndarray], bits: int) -> np.ndarray:
-    """Inverse of :func:`pack_k_rows`."""
+    """Inverse of :func:`pack_k_rows`: -> codes [N, 128]."""
+    if bits == 2:
+        words = planes[0]
+        nq = words.shape[0]
+        codes = np.zeros((nq, 4, HEAD_DIM), dtype=np.uint32)
+        for q in range(nq):
+            for omega in range(32):
+                wd = words[q, k2_word_pos(q, omega)]
+                for beta in range(4):
+                    for f in range(4):
+                        codes[q, f, 4 * omega + beta] = (wd >> np.uint32(8 * beta + 2 * f)) & np.uint32(3)
+        return codes.reshape(nq * 4, HEAD_DIM).astype(np.uint8)
     n = planes[0].shape[:-1]
     codes = np.zeros(n + (HEAD_DIM,), dtype=np.uint32)
     shift = 0

@@ -42,7 +42,8 @@ def _unit_blocks(cache, u: int, n_packed: int) -> np.ndarray:
 def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
     """The packed plane bytes of unit u for its first n_packed tokens,
     gathered from the block records into uint32 arrays shaped like the
-    oracle's pack_* output (token rows for K, quads for V)."""
+    oracle's pack_* output (token rows for 3- and 4-bit K, quads for 2-bit K
+    and for V)."""
     L = cache.layout()
     blocks = _unit_blocks(cache, u, n_packed)
     out = []
@@ -50,7 +51,10 @@ def unit_packed_planes(cache, u: int, kv: int, n_packed: int):
         w = L.plane_bits[p]
         off = L.k_plane_off[p] if kv == 0 else L.v_plane_off[p]
         part = np.ascontiguousarray(blocks[:, off:off + 64 * 16 * w]).view(np.uint32)
-        if kv == 0:
+        if kv == 0 and cache.cfg.bits == 2:
+            # 2-bit K quads: 16 quads of 32 words per block record, in order
+            out.append(part.reshape(-1, 32)[:n_packed // 4])
+        elif kv == 0:
             # K rows sit at the swizzled position 8r + (j ^ (r & 3)) of token
             # 8r + j of each 64-token block
             rows = part.reshape(-1, 64, 4 * w)

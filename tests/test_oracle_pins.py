@@ -89,14 +89,14 @@ def test_attention_through_transforms():
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_pack_roundtrip_and_bijection(bits):
     g = np.random.default_rng(bits)
-    c = g.integers(0, 1 << bits, (7, 128)).astype(np.uint8)
+    c = g.integers(0, 1 << bits, (8, 128)).astype(np.uint8)
     assert (O.unpack_k_rows(O.pack_k_rows(c, bits), bits) == c).all()
     cq = g.integers(0, 1 << bits, (3, 4, 128)).astype(np.uint8)
     assert (O.unpack_v_quads(O.pack_v_quads(cq, bits), bits) == cq).all()
     # every (dim) of a row and every (token, dim) of a quad owns distinct bits
     total = sum(int(np.unpackbits(p.view(np.uint8)).sum())
-                for p in O.pack_k_rows(np.full((1, 128), (1 << bits) - 1, np.uint8), bits))
-    assert total == 128 * bits
+                for p in O.pack_k_rows(np.full((4, 128), (1 << bits) - 1, np.uint8), bits))
+    assert total == 4 * 128 * bits
     total = sum(int(np.unpackbits(p.view(np.uint8)).sum())
                 for p in O.pack_v_quads(np.full((1, 4, 128), (1 << bits) - 1, np.uint8), bits))
     assert total == 512 * bits
@@ -118,8 +118,8 @@ def test_pack_positions_golden():
     for kind, bits, plane, tok, dim, word, bit in _golden_positions():
         code = (1 << bits) - 1
         if kind == "K":
-            c = np.zeros((1, 128), np.uint8)
-            c[0, dim] = code
+            c = np.zeros(((tok // 4 + 1) * 4 if bits == 2 else 1, 128), np.uint8)
+            c[tok if bits == 2 else 0, dim] = code
             planes = O.pack_k_rows(c, bits)
         else:
             c = np.zeros((tok // 4 + 1, 4, 128), np.uint8)
