@@ -420,10 +420,11 @@ __device__ __forceinline__ void packed_block_compute(
   const int nvalid = n_packed - blk * PB;  // used when !FULL
 
   // ---- scores ----------------------------------------------------------------
-  // Lane 4r + c owns tokens 8r .. 8r + 7 of the block (slot j = 2 mt + th is
-  // token 8r + j, row r + 8 th of m-tile mt).  Its K rows sit at positions
-  // 8r + (j ^ (r & 3)) (the cache's row swizzle), which spreads each load
-  // over all shared-memory banks.
+  // Lane 4r + c owns eight tokens of the block: slot j = 2 mt + th is row
+  // r + 8 th of m-tile mt, token slot_token(r, j).  2-bit keys: the lane
+  // reads its eight words of quads r and r + 8 as four 16-byte chunks.
+  // Wider keys: its K rows sit at positions 8r + (j ^ (r & 3)) (the cache's
+  // row swizzle), which spreads each load over all shared-memory banks.
   // sc[j]: score minus the reference in use (m, or 0 while m = -inf)
   float sc[8][NT];
   float vs[8], vo[8];

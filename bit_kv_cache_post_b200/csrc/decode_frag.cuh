@@ -1,10 +1,14 @@
 // Register-level access to the packed cache for the tensor-core decode.
 //
 // The packed format (include/wushkv.h) is laid out so that the integer
-// mma.sync fragments fall out of one shift and one mask per register:
-//   * K rows: thread c of a quad of lanes (lane = 4r + c) reads 8 bytes per
-//     2-bit plane of a token row; field ks of word (2c + h) holds dims
-//     32ks + 4c + 16h + beta at byte beta -- exactly the A fragment
+// mma.sync fragments fall out of at most one shift and one mask per register:
+//   * 2-bit K quads: word (ks, h, c) of a quad holds dims 32ks + 16h + 4c +
+//     beta at byte beta for its four tokens at fields 0..3 -- masked to field
+//     f it is the A fragment A[token 4 quad + f][k = 4c + 16h + beta] of
+//     k-step ks (times 4^f), so m-tile f's fragments need no shift.
+//   * 3- and 4-bit K rows: thread c of a quad of lanes (lane = 4r + c) reads
+//     8 bytes per 2-bit plane of a token row; field ks of word (2c + h) holds
+//     dims 32ks + 4c + 16h + beta at byte beta -- exactly the A fragment
 //     A[token][k = 4c + 16h + beta] of k-step ks of an m16n8k32 product.
 //   * V quads: word (r, j) field s holds dim 16mt + r + 8rh (rho = 2mt + rh)
 //     of the quad's 4 tokens at bytes 0..3 -- the A fragment

@@ -114,19 +114,25 @@ typedef struct wushkv_cache wushkv_cache; /* opaque host handle */
  *     copy fetches everything the decode needs for those tokens.
  *     k_plane_off[p], v_plane_off[p], k_meta_off and v_meta_off are the
  *     offsets of these parts in unit 0's block 0; block b of unit u adds
- *     u * unit_stride + b * block_stride.  Within a record, the K row of
- *     packed token b * 64 + i sits at 16 * w * pos(i) with the row swizzle
+ *     u * unit_stride + b * block_stride.  Within a record, 2-bit K quad
+ *     b * 16 + q sits at 128 * q; at 3 and 4 bits the K row of packed token
+ *     b * 64 + i sits at 16 * w * pos(i) with the row swizzle
  *     pos(i) = (i & 56) | ((i & 7) ^ ((i >> 3) & 3)) (spreads the decode's
- *     shared-memory reads over all banks), V quads b * 16 + q at 64 * w * q,
+ *     shared-memory reads over all banks); V quads b * 16 + q at 64 * w * q,
  *     meta entries at meta_bytes * i.
  * Formats:
  *   planes: 2-bit codes -> one 2-bit plane, 4-bit -> one 4-bit plane, 3-bit
  *     -> a 2-bit plane of (code & 3) and a 1-bit plane of (code >> 2).  A
  *     plane of width w packs 8/w fields per byte; field s of byte beta of a
  *     little-endian 32-bit word is at bit 8*beta + w*s.
- *   K (token rows, 16*w bytes per token per plane): c in 0..3, h in 0..1,
- *     ks in 0..3, beta in 0..3, rho = 4h + ks: word c*w + rho/(8/w), field
- *     rho % (8/w), dim 32ks + 4c + 16h + beta.
+ *   K, 2 bits (4-token quads, 128 bytes per quad): word omega holds dims
+ *     4*omega + beta at byte beta and token 4*quad + f at field f; with
+ *     omega = 8ks + 4h + c it sits at word 4*((2c + ks/2) xor (quad mod 2))
+ *     + 2*(ks mod 2) + h of the quad (the decode's score fragment of m-tile
+ *     f is the word masked to field f).
+ *   K, 3 and 4 bits (token rows, 16*w bytes per token per plane): c in 0..3,
+ *     h in 0..1, ks in 0..3, beta in 0..3, rho = 4h + ks: word c*w +
+ *     rho/(8/w), field rho % (8/w), dim 32ks + 4c + 16h + beta.
  *   V (4-token quads, 64*w bytes per quad per plane): r in 0..7, rho in
  *     0..15 (mt = rho/2, rh = rho%2), beta in 0..3: unit word j = rho/(8/w),
  *     field rho % (8/w), dim 16mt + r + 8rh, token 4*quad + beta.  Row unit
