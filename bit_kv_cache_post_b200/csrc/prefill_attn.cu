@@ -40,10 +40,12 @@ constexpr int PA_THREADS = PA_WARPS * 32;
 constexpr int PA_ROWS = 16 * PA_WARPS;   // (query, head) rows per CTA
 constexpr int PA_TOK = 64;               // tokens per staged block (one packed block record)
 constexpr int PA_LD = D + 8;             // halves per shared row (272 bytes: conflict-free ldmatrix)
+constexpr int PA_LDT = PA_TOK + 8;       // halves per transposed value row (144 bytes)
 
 struct PaSmem {
   __half qhi[PA_ROWS][PA_LD], qlo[PA_ROWS][PA_LD];
-  __half kr[PA_TOK][PA_LD], vr[PA_TOK][PA_LD];
+  __half kr[PA_TOK][PA_LD];      // key rows [token][dim]
+  __half vt[D][PA_LDT];          // value rows transposed [dim][token]
   float ks[PA_TOK], ko[PA_TOK], vs[PA_TOK], vo[PA_TOK];
   float qsum[PA_ROWS];
 };
@@ -126,7 +128,7 @@ __device__ __forceinline__ void load_block(const DevCache& c, int u, int blk, in
   }
 }
 
-// The block's codes into kr / vr as fp16 values -- key codes as they are,
+// The block's codes into kr / vt as fp16 values -- key codes as they are,
 // value codes minus (L - 1) / 2 -- (the second plane of 3-bit codes adds
 // 4 x its bit after a barrier) and the (scale, offset) pairs; key rows past
 // cnt come out zero (their words were loaded as zero), value rows past cnt
@@ -147,10 +149,14 @@ __device__ __forceinline__ void write_block(const DevCache& c, PaSmem& sh, int c
       if constexpr (BITS == 2) {   // K quads: field f = token 4q + f, byte beta = dim 4 omega + beta
         const int q = e >> 5, om = e & 31;
 #pragma unroll
-        for (int f = 0; f < 4; ++f)
-#pragma unroll
-          for (int beta = 0; beta < 4; ++beta)
-            sh.kr[4 * q + f][4 * om + beta] = __float2half_rn((float)((word >> (8 * beta + 2 * f)) & 3u));
+        for (int f = 0; f < 4; ++f) {   // dims 4 omega .. 4 omega + 3 of token 4q + f: one 8-byte store
+          const __half2 lo = __floats2half2_rn((float)((word >> (2 * f)) & 3u), (float)((word >> (8 + 2 * f)) & 3u));
+          const __half2 hi = __floats2half2_rn((float)((word >> (16 + 2 * f)) & 3u), (float)((word >> (24 + 2 * f)) & 3u));
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(&sh.kr[4 * q + f][4 * om]) = pk;
+        }
       } else {
         const int i = e / (4 * w), wi = e % (4 * w);
 #pragma unroll
@@ -170,14 +176,25 @@ __device__ __forceinline__ void write_block(const DevCache& c, PaSmem& sh, int c
 #pragma unroll
       for (int s = 0; s < F; ++s) {
         const int dim = v_field_dim(rj, w, s);
+        // the quad's four tokens of this dim (bytes 0..3): one 8-byte store;
+        // value codes centred on the grid's middle (the first plane takes the
+        // shift): half the magnitude, so P's fp16 rounding counts half
+        float v[4];
 #pragma unroll
-        for (int beta = 0; beta < 4; ++beta) {
-          // value codes centred on the grid's middle (the first plane takes
-          // the shift): half the magnitude, so P's fp16 rounding counts half
-          const float v = (float)((word >> (8 * beta + w * s)) & mask) * mul - (p == 0 ? CMID : 0.f);
-          __half* dst = &sh.vr[4 * q + beta][dim];
-          *dst = p == 0 ? __float2half_rn(v) : __float2half_rn(__half2float(*dst) + v);
+        for (int beta = 0; beta < 4; ++beta)
+          v[beta] = (float)((word >> (8 * beta + w * s)) & mask) * mul - (p == 0 ? CMID : 0.f);
+        uint2* dst = reinterpret_cast<uint2*>(&sh.vt[dim][4 * q]);
+        if (p != 0) {   // the second plane adds to the first
+          const uint2 old = *dst;
+          const float2 o01 = __half22float2(*reinterpret_cast<const __half2*>(&old.x));
+          const float2 o23 = __half22float2(*reinterpret_cast<const __half2*>(&old.y));
+          v[0] += o01.x; v[1] += o01.y; v[2] += o23.x; v[3] += o23.y;
         }
+        const __half2 lo = __floats2half2_rn(v[0], v[1]), hi = __floats2half2_rn(v[2], v[3]);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *dst = pk;
       }
     }
     if (PL::N > 1 && p == 0) __syncthreads();   // the second plane adds to what the first wrote
@@ -201,7 +218,7 @@ __device__ __forceinline__ void write_block(const DevCache& c, PaSmem& sh, int c
   }
 }
 
-// Rows [0, cnt) of a block of fp16 window rows (sink or ring) into kr / vr;
+// Rows [0, cnt) of a block of fp16 window rows (sink or ring) into kr / vt;
 // rows past cnt are zero.  Scales 1, offsets 0.
 __device__ __forceinline__ void stage_window(const DevCache& c, PaSmem& sh, int u, int kind, int t0, int cnt,
                                              int tid) {
@@ -219,7 +236,13 @@ __device__ __forceinline__ void stage_window(const DevCache& c, PaSmem& sh, int 
       }
       val = __ldg(reinterpret_cast<const uint4*>(row) + ch);
     }
-    *reinterpret_cast<uint4*>(&(kv ? sh.vr : sh.kr)[i][8 * ch]) = val;
+    if (kv == 0) {
+      *reinterpret_cast<uint4*>(&sh.kr[i][8 * ch]) = val;
+    } else {   // values transposed: dims 8 ch .. 8 ch + 7 of token i
+      const __half* hv = reinterpret_cast<const __half*>(&val);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sh.vt[8 * ch + k][i] = hv[k];
+    }
   }
   if (tid < PA_TOK) {
     const bool ok = tid < cnt;
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __grid_c
   const uint32_t qaddr_hi = smem_addr(&sh.qhi[16 * warp + (lane & 15)][8 * (lane >> 4)]);
   const uint32_t qaddr_lo = smem_addr(&sh.qlo[16 * warp + (lane & 15)][8 * (lane >> 4)]);
   const uint32_t kaddr = smem_addr(&sh.kr[(lane & 7) + 8 * (lane >> 4)][8 * ((lane >> 3) & 1)]);
-  const uint32_t vaddr = smem_addr(&sh.vr[(lane & 7) + 8 * ((lane >> 3) & 1)][8 * (lane >> 4)]);
+  const uint32_t vaddr = smem_addr(&sh.vt[(lane & 7) + 8 * (lane >> 4)][8 * ((lane >> 3) & 1)]);
 
   for (int ib = 0; ib < nblocks; ++ib) {
     const BlockSpan sp = block_span(a, ib, nb_sink, nb_pk, n_rec);
@@ -410,7 +433,7 @@ __global__ void __launch_bounds__(PA_THREADS) prefill_attn_kernel(const __grid_c
 #pragma unroll
       for (int dp = 0; dp < 8; ++dp) {
         uint32_t bv[4];
-        ldmatrix_x4_trans(bv, vaddr + kt * 16 * PA_LD * 2 + dp * 32);
+        ldmatrix_x4(bv, vaddr + dp * 16 * PA_LDT * 2 + kt * 32);
         mma_f16_k16(O[2 * dp], a0, a1, a2, a3, bv[0], bv[1]);
         mma_f16_k16(O[2 * dp + 1], a0, a1, a2, a3, bv[2], bv[3]);
       }
