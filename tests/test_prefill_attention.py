@@ -34,33 +34,82 @@ def _filled(n, G=4, Hkv=2, B=2, bits=2, quantizer=O.QUEST_INT, sink=16, recent=3
     return c, k, v, T
 
 
-def test_last_query_is_the_decode():
-    """The chunk's last query sees the whole cache: it is the decode of that
-    query."""
+def _oracle(c, q):
+    return c.prefill_attention(q)
+
+
+def check_last_query_is_the_decode(prefill):
     c, *_ = _filled(120)
     q = np.random.default_rng(1).standard_normal((2, 5, 8, 128))
-    out = c.prefill_attention(q)
+    out = prefill(c, q)
     dec = c.decode(q[:, -1])
     assert np.abs(out[:, -1] - dec).max() <= 1e-12
 
 
-def test_causal():
-    """Replacing the last token changes only the last query's output."""
+def check_causal(prefill):
     q = np.random.default_rng(2).standard_normal((2, 6, 8, 128))
     a, *_ = _filled(130, last_token_seed=5)
     b, *_ = _filled(130, last_token_seed=6)
-    oa, ob = a.prefill_attention(q), b.prefill_attention(q)
+    oa, ob = prefill(a, q), prefill(b, q)
     assert np.array_equal(oa[:, :-1], ob[:, :-1])
     assert np.abs(oa[:, -1] - ob[:, -1]).max() > 1e-3
+
+
+def test_last_query_is_the_decode():
+    """The chunk's last query sees the whole cache: it is the decode of that
+    query."""
+    check_last_query_is_the_decode(_oracle)
+
+
+def test_causal():
+    """Replacing the last token changes only the last query's output."""
+    check_causal(_oracle)
+
+
+def _mutant(first_visible=0, extra=1, shift=0):
+    """prefill_attention with a planted mistake: the query of token p sees
+    tokens first_visible .. p + extra - 1 (with p moved by shift)."""
+    def f(c, q):
+        B, nq, Hq, d = q.shape
+        G = c.cfg.group
+        out = np.full((B, nq, Hq, d), np.nan)
+        for u in range(c.cfg.units):
+            b, h = divmod(u, c.cfg.n_kv_heads)
+            K, V = c.unit_kv(u)
+            for i in range(nq):
+                p = c.n - nq + i + shift
+                hi = min(c.n, max(p + extra, first_visible + 1))
+                out[b, i, h * G:(h + 1) * G] = O.attention_f64(q[b, i, h * G:(h + 1) * G], K[first_visible:hi],
+                                                               V[first_visible:hi], 1.0 / math.sqrt(128.0))
+        return out
+    return f
+
+
+@pytest.mark.parametrize("mut", [dict(extra=0), dict(extra=10 ** 9), dict(shift=-1), dict(first_visible=1)],
+                         ids=["sees-one-less", "not-causal", "position-off-by-one", "drops-token-0"])
+def test_prefill_mistakes_are_caught(mut):
+    """Each planted mistake fails at least one pin."""
+    bad = _mutant(**mut)
+    caught = 0
+    for check in (check_last_query_is_the_decode, check_causal, check_brute_force_tiny):
+        try:
+            check(bad)
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, mut
 
 
 def test_brute_force_tiny():
     """Explicit loops over tokens (max, exponentials, sums) on a tiny cache
     with sink, packed and recent tokens."""
+    check_brute_force_tiny(_oracle)
+
+
+def check_brute_force_tiny(prefill):
     c, *_ = _filled(45, G=2, Hkv=1, B=1, sink=4, recent=8, chunk=4, seed=3)
     assert c.split()[1] > 0
     q = np.random.default_rng(4).standard_normal((1, 7, 2, 128))
-    out = c.prefill_attention(q)
+    out = prefill(c, q)
     K, V = c.unit_kv(0)
     s = 1.0 / math.sqrt(128.0)
     for i in range(7):
