@@ -362,13 +362,14 @@ __device__ __forceinline__ void issue_item(const DecodeArgs& a, const GEO& geo, 
 }
 
 // ---- packed blocks: copy ring + integer tensor cores ------------------------------
+// K row words of token row t for lane c4 (3- and 4-bit keys; 2-bit keys are
+// read as quads in packed_block_compute).
 template <int BITS>
 __device__ __forceinline__ KWords<BITS> stage_k_words(const unsigned char* st, int t, int c4) {
+  static_assert(BITS == 3 || BITS == 4, "2-bit keys are packed in quads");
   using SL = StageLayout<BITS>;
   KWords<BITS> w;
-  if constexpr (BITS == 2) {
-    w.lo = *reinterpret_cast<const uint2*>(st + SL::K_LO + t * 32 + 8 * c4);
-  } else if constexpr (BITS == 3) {
+  if constexpr (BITS == 3) {
     w.lo = *reinterpret_cast<const uint2*>(st + SL::K_LO + t * 32 + 8 * c4);
     w.hi = *reinterpret_cast<const uint32_t*>(st + SL::K_HI + t * 16 + 4 * c4);
   } else {

@@ -67,17 +67,14 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&v)[4], uint32_t add
 }
 
 // ---- K rows -------------------------------------------------------------------
-template <int BITS> struct KWords;
-template <> struct KWords<2> { uint2 lo; };
+template <int BITS> struct KWords;   // 3- and 4-bit K rows
 template <> struct KWords<3> { uint2 lo; uint32_t hi; };
 template <> struct KWords<4> { uint4 w; };
 
 // A fragment register of k-step ks, half h (k columns 16h + 4c .. +3).
 template <int BITS>
 __device__ __forceinline__ uint32_t k_frag(const KWords<BITS>& w, int ks, int h) {
-  if constexpr (BITS == 2) {
-    return ((h ? w.lo.y : w.lo.x) >> (2 * ks)) & 0x03030303u;
-  } else if constexpr (BITS == 3) {
+  if constexpr (BITS == 3) {
     const uint32_t lo = ((h ? w.lo.y : w.lo.x) >> (2 * ks)) & 0x03030303u;
     const int rho = 4 * h + ks;
     return lo | (((w.hi >> rho) & 0x01010101u) << 2);
