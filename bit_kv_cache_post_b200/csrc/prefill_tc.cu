@@ -239,18 +239,20 @@ __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double a
     // hold a quad's rows): word (c, h) of lane f holds k-step ks at field ks;
     // the quad's word omega = 8 ks + 4 h + c holds token f at field f.  Lane
     // f collects the words of k-step f from the four lanes.
-    const int lane = threadIdx.x & 31, f = lane & 3;
+    // A 4 x 4 transpose of 2-bit fields (lane f, field ks) -> (lane ks,
+    // field f) in two exchange rounds: with lane f ^ 1 the fields of the
+    // other parity, then with lane f ^ 2 the other half of each byte.
+    const int f = threadIdx.x & 3;
     uint32_t qw[8];
 #pragma unroll
     for (int x = 0; x < 8; ++x) {   // x = 2 c + h
-      uint32_t acc = 0u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int dst = (f - j) & 3;   // the lane that takes this round's value
-        const uint32_t send = ((w0[x] >> (2 * dst)) & 0x03030303u) << (2 * f);
-        acc |= __shfl_sync(FULL, send, (lane & ~3) | ((f + j) & 3));
-      }
-      qw[x] = acc;
+      const uint32_t X = w0[x];
+      const uint32_t P = __shfl_xor_sync(FULL, X, 1);
+      const uint32_t Xa = (f & 1) ? (((P & 0xCCCCCCCCu) >> 2) | (X & 0xCCCCCCCCu))
+                                  : ((X & 0x33333333u) | ((P & 0x33333333u) << 2));
+      const uint32_t Q = __shfl_xor_sync(FULL, Xa, 2);
+      qw[x] = (f & 2) ? (((Q & 0xF0F0F0F0u) >> 4) | (Xa & 0xF0F0F0F0u))
+                      : ((Xa & 0x0F0F0F0Fu) | ((Q & 0x0F0F0F0Fu) << 4));
     }
     if (!packed) return;
     uint32_t* o = reinterpret_cast<uint32_t*>(row0);   // the quad's 128 bytes
