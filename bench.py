@@ -596,6 +596,13 @@ def run_ragged_decode(device, torch, paged: bool, copies=8, bits=2):
             "frac": nbytes / us / 1e3 / peak, "copies": copies, "device_status": status}
 
 
+def prefill_attention_flops(n, nq, batch, n_q_heads):
+    """4 x 128 flop (q.k and p.v) per (query head, visible token); the
+    chunk's query i sees n - nq + i + 1 tokens."""
+    visible = nq * (n - nq) + nq * (nq + 1) // 2
+    return 4.0 * 128 * visible * batch * n_q_heads
+
+
 def run_prefill_attention(device, torch, nq=512, copies=4, bits=2):
     """Chunked-prefill attention at the batch-16 Qwen3-8B-shaped layer: each
     sequence holds 8192 tokens of which the last nq are the chunk; its
@@ -647,8 +654,7 @@ def run_prefill_attention(device, torch, nq=512, copies=4, bits=2):
     us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
     del graph
     status = max(c.device_status() for c in caches)
-    visible = nq * (n - nq) + nq * (nq + 1) // 2          # (query, token) pairs per head
-    flops = 4.0 * 128 * visible * w.batch * w.n_q_heads
+    flops = prefill_attention_flops(n, nq, w.batch, w.n_q_heads)
     peak_tf = peaks_tensor()
     tf = flops / us / 1e6
     return {"workload": f"{WORKLOAD}: chunk of the last {nq} of {n} tokens per sequence, {bits}-bit QuEST, G {w.group}",
