@@ -187,8 +187,10 @@ __device__ __forceinline__ void key_codes(uint32_t taddr, const QParams& q, bool
 // format of wushkv.h): dim d = 32 ks + 4 c + 16 h + beta goes to word
 // c w + rho / (8/w), field rho mod (8/w), byte beta, with rho = 4 h + ks; the
 // two codes of a pair (beta, beta + 1) share a word and a field and are
-// placed together with one byte permute.  Every lane of the warp must call
-// (the TMEM accesses are warp-wide).
+// placed together with one byte permute.  At 2 bits the four lanes holding a
+// quad's rows then exchange fields so that each stores its share of the
+// quad's words (K quads: field = token).  Every lane of the warp must call
+// (the TMEM accesses and the exchange are warp-wide).
 template <int BITS, bool AFFINE>
 __device__ __forceinline__ void key_row(uint32_t taddr, float2 unscale, double alpha,
                                         bool lo_second, bool hi_second, int mode, uint8_t* row0,
