@@ -92,7 +92,6 @@ __device__ __forceinline__ void load_block(const DevCache& c, int u, int blk, in
     const int w = p == 0 ? PL::W0 : PL::W1;
     const uint8_t* kb = c.k_plane[p] + boff;
     const uint8_t* vb = c.v_plane[p] + boff;
-    const int nk = p == 0 ? PL::K0 : PL::K1, nv = p == 0 ? PL::V0 : PL::V1;
 #pragma unroll
     for (int j = 0; j < (p == 0 ? PL::K0 : PL::K1); ++j) {
       const int e = tid + PA_THREADS * j;
@@ -114,7 +113,6 @@ __device__ __forceinline__ void load_block(const DevCache& c, int u, int blk, in
                                      : 0u;   // the block starts at a multiple of 16 quads
       if (p == 0) r.v0[j] = x; else r.v1[j] = x;
     }
-    (void)nk; (void)nv;
   }
   r.km = r.vm = 0u;
   if (tid < cnt) {
